@@ -1,0 +1,219 @@
+"""Python binding of the smgemm C-ABI (libsmgemm.so, built for sm_100a).
+
+Argument marshalling only: torch tensors give device pointers, leading dimensions
+and the current CUDA stream; every computation runs in the library's kernels. There
+is no fallback: if the library is missing or a call fails, an exception is raised.
+
+    import sm_gemm_b200 as sg
+    C = sg.gemm_bf16(A, B, bias=b, act="gelu_tanh", out_dtype=torch.bfloat16)
+    Q, S = sg.quantize_fp8_blockwise(X, group_rows=1)
+    C = sg.gemm_fp8_blockscaled(Aq, sa, Bq, sb, out_dtype=torch.bfloat16)
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsmgemm.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(7)
+F32, BF16, F16, E4M3 = 0, 1, 2, 3
+ROW_MAJOR, COL_MAJOR = 0, 1
+ACTS = {"none": 0, None: 0, "gelu_tanh": 1, "gelu": 1, "silu": 2}
+
+_lock = threading.Lock()
+_lib = None
+_ws_cache: dict = {}
+
+
+class SmgemmError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"smgemm {what}: status {status} ({status_string(status)})")
+
+
+def lib():
+    """The loaded C library (built in-tree by ``python -m sm_gemm_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sm_gemm_b200.build`")
+            L = C.CDLL(LIB_PATH)
+            I64, P, I, SZ = C.c_int64, C.c_void_p, C.c_int, C.c_size_t
+            L.gemm_bf16.argtypes = [I64, I64, I64, P, I, I, I64, P, I, I64, P, I, I, P, I, I64, P, SZ, P]
+            L.gemm_bf16.restype = I
+            L.gemm_fp8_blockscaled.argtypes = [I64, I64, I64, P, P, P, P, P, I, I, P, I, I64, P, SZ, P]
+            L.gemm_fp8_blockscaled.restype = I
+            L.quantize_fp8_blockwise.argtypes = [P, I64, I64, I, I64, I, P, P, P]
+            L.quantize_fp8_blockwise.restype = I
+            L.smgemm_workspace_size.argtypes = [I64, I64, I64, I]
+            L.smgemm_workspace_size.restype = SZ
+            L.smgemm_status_string.argtypes = [I]
+            L.smgemm_status_string.restype = C.c_char_p
+            L.smgemm_check.argtypes = [P]
+            L.smgemm_check.restype = I
+            L.smgemm_last_config.argtypes = []
+            L.smgemm_last_config.restype = C.c_char_p
+            L.smgemm_selftest_wait_timeout.argtypes = [C.c_uint32, P]
+            L.smgemm_selftest_wait_timeout.restype = I
+            L.smgemm_schedule_dump.argtypes = [I64, I64, I64, I, I, I, P, I64]
+            L.smgemm_schedule_dump.restype = I64
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().smgemm_status_string(status).decode()
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(dt) -> int:
+    torch = _torch()
+    return {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}[dt]
+
+
+def _layout(t, name):
+    """(layout, leading dimension) of a 2-D tensor; one of its strides must be 1."""
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D")
+    if t.stride(1) == 1 and (t.shape[0] <= 1 or t.stride(0) >= t.shape[1]):
+        return ROW_MAJOR, max(t.stride(0), t.shape[1])
+    if t.stride(0) == 1:
+        return COL_MAJOR, max(t.stride(1), t.shape[0])
+    raise ValueError(f"{name} must have a unit stride in one dimension")
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if hasattr(stream, "cuda_stream"):
+        return C.c_void_p(stream.cuda_stream)
+    return C.c_void_p(stream)
+
+
+def _workspace(nbytes: int, device):
+    if nbytes == 0:
+        return None, 0
+    torch = _torch()
+    key = (device.index if device.index is not None else torch.cuda.current_device())
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws, ws.numel()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise SmgemmError(status, what)
+
+
+def workspace_size(M: int, N: int, K: int, kind: int = 0) -> int:
+    return int(lib().smgemm_workspace_size(M, N, K, kind))
+
+
+def gemm_bf16(A, B, *, bias=None, act="none", out=None, out_dtype=None, workspace=None, stream=None):
+    """C = act(A @ B + bias) for bf16/f16 A[M,K], B[K,N] (any unit-stride layout).
+
+    ``out`` (row-major [M,N]) is allocated when not given; ``out_dtype`` defaults to
+    A's dtype. Returns ``out``."""
+    torch = _torch()
+    M, K = A.shape
+    K2, N = B.shape
+    if K != K2 or A.dtype != B.dtype:
+        raise ValueError("A and B must agree in K and dtype")
+    la, lda = _layout(A, "A")
+    lb, ldb = _layout(B, "B")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or A.dtype, device=A.device)
+    if out.stride(1) != 1:
+        raise ValueError("out must be row-major")
+    ldc = max(out.stride(0), N)
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
+        _workspace(workspace_size(M, N, K, 0), A.device)
+    st = lib().gemm_bf16(M, N, K, A.data_ptr(), _dtype_code(A.dtype), la, lda, B.data_ptr(), lb, ldb,
+                         None if bias is None else bias.data_ptr(),
+                         _dtype_code(bias.dtype) if bias is not None else 0, ACTS[act],
+                         out.data_ptr(), _dtype_code(out.dtype), ldc,
+                         None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+    _check(st, "gemm_bf16")
+    return out
+
+
+def gemm_fp8_blockscaled(Aq, sa, Bq, sb, *, bias=None, act="none", out=None, out_dtype=None,
+                         workspace=None, stream=None):
+    """C = act(sum_kb sa*sb*(Aq @ Bq^T)_kb + bias) from E4M3 codes Aq[M,K], Bq[N,K] (uint8 or
+    float8_e4m3fn, K contiguous) and FP32 scales sa[KB,M], sb[KB,NB]."""
+    torch = _torch()
+    M, K = Aq.shape
+    N, K2 = Bq.shape
+    if K != K2:
+        raise ValueError("Aq and Bq must agree in K")
+    for t, n in ((Aq, "Aq"), (Bq, "Bq"), (sa, "sa"), (sb, "sb")):
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=Aq.device)
+    ldc = max(out.stride(0), N)
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
+        _workspace(workspace_size(M, N, K, 1), Aq.device)
+    st = lib().gemm_fp8_blockscaled(M, N, K, Aq.data_ptr(), sa.data_ptr(), Bq.data_ptr(), sb.data_ptr(),
+                                    None if bias is None else bias.data_ptr(),
+                                    _dtype_code(bias.dtype) if bias is not None else 0, ACTS[act],
+                                    out.data_ptr(), _dtype_code(out.dtype), ldc,
+                                    None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+    _check(st, "gemm_fp8_blockscaled")
+    return out
+
+
+def quantize_fp8_blockwise(X, group_rows: int = 1, *, Q=None, scales=None, stream=None):
+    """FP32 X[rows, cols] -> (codes uint8, scales float32). group_rows=1: 1x128 groups,
+    codes [rows, cols], scales [ceil(cols/128), rows]. group_rows=128: 128x128 blocks of
+    the weight X[K, N], codes written transposed [N, K], scales [ceil(K/128), ceil(N/128)]."""
+    torch = _torch()
+    rows, cols = X.shape
+    lx, ldx = _layout(X, "X")
+    if group_rows == 1:
+        qshape, sshape = (rows, cols), (-(-cols // 128), rows)
+    else:
+        qshape, sshape = (cols, rows), (-(-rows // 128), -(-cols // 128))
+    if Q is None:
+        Q = torch.empty(qshape, dtype=torch.uint8, device=X.device)
+    if scales is None:
+        scales = torch.empty(sshape, dtype=torch.float32, device=X.device)
+    st = lib().quantize_fp8_blockwise(X.data_ptr(), rows, cols, lx, ldx, group_rows, Q.data_ptr(),
+                                      scales.data_ptr(), _stream(stream))
+    _check(st, "quantize_fp8_blockwise")
+    return Q, scales
+
+
+def check(stream=None) -> int:
+    """Synchronise the stream and return the library status (ERR_TIMEOUT if a kernel
+    abandoned a barrier wait since the last check)."""
+    return int(lib().smgemm_check(_stream(stream)))
+
+
+def last_config() -> str:
+    return lib().smgemm_last_config().decode()
+
+
+def selftest_wait_timeout(limit_us: int, stream=None) -> int:
+    return int(lib().smgemm_selftest_wait_timeout(limit_us, _stream(stream)))
+
+
+def schedule_dump(M: int, N: int, K: int, kind: int = 0, layout_a: int = ROW_MAJOR, num_sms: int = 148):
+    """Segments (cta, tile, m_tile, n_tile, kb_begin, kb_end, slot) of the persistent
+    schedule a call with these sizes uses on a GPU with ``num_sms`` SMs (host only)."""
+    import numpy as np
+    n = lib().smgemm_schedule_dump(M, N, K, kind, layout_a, num_sms, None, 0)
+    out = np.zeros((max(n, 1), 7), dtype=np.int32)
+    lib().smgemm_schedule_dump(M, N, K, kind, layout_a, num_sms, out.ctypes.data_as(C.c_void_p), n)
+    return out[:n]

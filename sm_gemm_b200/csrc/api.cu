@@ -1,0 +1,455 @@
+// C-ABI of the GEMM library: argument validation, TMA descriptor encoding, schedule
+// planning (tile grid, data-parallel / stream-K split, workspace) and dispatch to the
+// sm_100a kernels. Declared in include/smgemm.h.
+//
+// The library links the CUDA runtime statically and reaches the one driver function it
+// needs (cuTensorMapEncodeTiled) through the runtime's entry-point query, so the shared
+// object loads on machines without a GPU driver; every entry point that needs the GPU
+// fails with SMGEMM_ERR_CUDA there.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/smgemm.h"
+#include "kernels.h"
+
+using namespace smg;
+
+namespace {
+
+// ------------------------------------------------------------------ driver entry point
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                    CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                    CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled encode_fn() {
+  static PFN_encodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  });
+  return fn;
+}
+
+// ------------------------------------------------------------------ device info
+
+struct DevInfo {
+  bool ok = false;
+  int sms = 0;
+};
+
+smgemm_status current_device(DevInfo& out) {
+  static std::mutex mu;
+  static DevInfo cache[64];
+  static bool filled[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return SMGEMM_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> g(mu);
+  if (!filled[dev]) {
+    cudaDeviceProp prop;
+    DevInfo d;
+    if (cudaGetDeviceProperties(&prop, dev) == cudaSuccess) {
+      d.ok = (prop.major == 10 && prop.minor == 0);
+      d.sms = prop.multiProcessorCount;
+    } else {
+      cudaGetLastError();
+    }
+    cache[dev] = d;
+    filled[dev] = true;
+  }
+  out = cache[dev];
+  return out.ok ? SMGEMM_OK : SMGEMM_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ config / logging
+
+thread_local char g_last_config[256] = "none";
+
+long long env_ll(const char* name, long long dflt) {
+  const char* v = std::getenv(name);
+  if (v == nullptr || *v == 0) return dflt;
+  return std::atoll(v);
+}
+
+enum class SchedMode { kAuto, kDP, kSK };
+
+SchedMode sched_mode() {
+  const char* v = std::getenv("SMGEMM_SCHED");
+  if (v == nullptr) return SchedMode::kAuto;
+  if (std::strcmp(v, "dp") == 0) return SchedMode::kDP;
+  if (std::strcmp(v, "sk") == 0) return SchedMode::kSK;
+  return SchedMode::kAuto;
+}
+
+// Tile-grid plan. Large tile counts run data-parallel waves with the ragged last
+// wave(s) handed to stream-K; small tile counts with a long K are split by stream-K
+// so every SM streams an equal share of the K-blocks (the page's concern that small
+// shapes leave SMs idle: "为什么我们要死磕GEMM", kwkr.cn, section 3.3).
+struct Plan {
+  TileSched s;
+  int grid = 0;
+  size_t counter_bytes = 0;
+  size_t slot_bytes = 0;  // all slots
+  size_t ws_bytes() const { return counter_bytes + slot_bytes; }
+};
+
+Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, size_t slot_floats) {
+  Plan pl;
+  const long long T = static_cast<long long>(m_tiles) * n_tiles;
+  long long max_ctas = env_ll("SMGEMM_GRID", sms);
+  if (max_ctas < 1) max_ctas = 1;
+  if (max_ctas > sms) max_ctas = sms;
+  const SchedMode mode = sched_mode();
+  constexpr int kMinItersPerCta = 8;
+
+  long long dp = T, sk_iters = 0, grid = std::min<long long>(T, max_ctas);
+  if (mode == SchedMode::kSK) {
+    dp = 0;
+    sk_iters = T * kb_total;
+    grid = std::min<long long>(max_ctas, sk_iters);
+  } else if (mode == SchedMode::kAuto) {
+    if (T >= max_ctas) {
+      if (T % max_ctas != 0 && kb_total >= kMinItersPerCta) {
+        dp = (T / max_ctas - 1) * max_ctas;
+        sk_iters = (T - dp) * kb_total;
+        grid = max_ctas;
+      }
+    } else {
+      const long long want = std::min<long long>(max_ctas, T * kb_total / kMinItersPerCta);
+      if (want > T) {
+        dp = 0;
+        sk_iters = T * kb_total;
+        grid = want;
+      }
+    }
+  }
+  pl.s.m_tiles = m_tiles;
+  pl.s.n_tiles = n_tiles;
+  pl.s.kb_total = kb_total;
+  pl.s.dp_tiles = static_cast<int>(dp);
+  pl.s.num_ctas = static_cast<int>(grid);
+  pl.s.group_m = std::max(1, std::min(group_m, m_tiles));
+  pl.s.sk_iters = sk_iters;
+  pl.grid = static_cast<int>(grid);
+  if (sk_iters > 0) {
+    pl.counter_bytes = ((static_cast<size_t>(T - dp) * sizeof(int)) + 255) / 256 * 256;
+    pl.slot_bytes = static_cast<size_t>(grid) * 2 * slot_floats * sizeof(float);
+  }
+  return pl;
+}
+
+// ------------------------------------------------------------------ TMA maps
+
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  PFN_encodeTiled fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_size(int dt) { return dt == kF32 ? 4 : (dt == kE4M3 ? 1 : 2); }
+
+bool valid_out_dtype(int dt) { return dt == kF32 || dt == kBF16 || dt == kF16; }
+bool valid_bias_dtype(int dt) { return dt == kF32 || dt == kBF16 || dt == kF16; }
+bool valid_act(int a) { return a == kActNone || a == kActGeluTanh || a == kActSilu; }
+bool valid_layout(int l) { return l == SMGEMM_ROW_MAJOR || l == SMGEMM_COL_MAJOR; }
+
+smgemm_status check_output(int64_t M, int64_t N, const void* C, int c_dtype, int64_t ldc, const void* bias,
+                           int bias_dtype, int act) {
+  if (!valid_out_dtype(c_dtype) || !valid_act(act)) return SMGEMM_ERR_INVALID_ARG;
+  if (bias != nullptr && !valid_bias_dtype(bias_dtype)) return SMGEMM_ERR_INVALID_ARG;
+  if (C == nullptr || ldc < N) return SMGEMM_ERR_INVALID_ARG;
+  if (!aligned16(C) || (ldc * elem_size(c_dtype)) % 16 != 0) return SMGEMM_ERR_ALIGNMENT;
+  if (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) % elem_size(bias_dtype)) != 0)
+    return SMGEMM_ERR_ALIGNMENT;
+  (void)M;
+  return SMGEMM_OK;
+}
+
+bool fits_int(int64_t v) { return v >= 0 && v <= 0x7FFFFFFF; }
+
+smgemm_status launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return SMGEMM_OK;
+  cudaGetLastError();
+  return SMGEMM_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ 16-bit GEMM plan
+
+struct Gemm16Plan {
+  Tc16Variant v;
+  bool skinny;
+  Plan pl;
+  int mma_n, bk;
+};
+
+Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms) {
+  Gemm16Plan g;
+  const bool force_large = env_ll("SMGEMM_FORCE_LARGE", 0) != 0;
+  g.skinny = (M <= 64 && layout_a == SMGEMM_ROW_MAJOR && !force_large);
+  if (g.skinny) g.v = M <= 16 ? Tc16Variant::kSkinny16 : (M <= 32 ? Tc16Variant::kSkinny32 : Tc16Variant::kSkinny64);
+  else g.v = Tc16Variant::kLarge;
+  g.mma_n = tc16_mma_n(g.v);
+  g.bk = tc16_bk(g.v);
+  const int kb = static_cast<int>((K + g.bk - 1) / g.bk);
+  int m_tiles, n_tiles;
+  if (g.skinny) {
+    m_tiles = static_cast<int>((N + 127) / 128);  // MMA rows run over the output columns
+    n_tiles = 1;
+  } else {
+    m_tiles = static_cast<int>((M + 127) / 128);
+    n_tiles = static_cast<int>((N + g.mma_n - 1) / g.mma_n);
+  }
+  g.pl = make_plan(m_tiles, n_tiles, std::max(kb, 1), sms, static_cast<int>(env_ll("SMGEMM_GROUP_M", 8)),
+                   static_cast<size_t>(128) * g.mma_n);
+  return g;
+}
+
+Plan plan_fp8(int64_t M, int64_t N, int64_t K, int sms) {
+  const int kb = static_cast<int>((K + kFp8BK - 1) / kFp8BK);
+  return make_plan(static_cast<int>((M + kFp8BM - 1) / kFp8BM), static_cast<int>((N + kFp8BN - 1) / kFp8BN),
+                   std::max(kb, 1), sms, static_cast<int>(env_ll("SMGEMM_GROUP_M", 8)),
+                   static_cast<size_t>(kFp8BM) * kFp8BN);
+}
+
+smgemm_status prepare_workspace(const Plan& pl, void* ws, size_t ws_bytes, cudaStream_t stream, float** slots,
+                                int** counters) {
+  *slots = nullptr;
+  *counters = nullptr;
+  if (pl.ws_bytes() == 0) return SMGEMM_OK;
+  if (ws == nullptr || ws_bytes < pl.ws_bytes()) return SMGEMM_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SMGEMM_ERR_ALIGNMENT;
+  *counters = static_cast<int*>(ws);
+  *slots = reinterpret_cast<float*>(static_cast<char*>(ws) + pl.counter_bytes);
+  return launch_status(cudaMemsetAsync(ws, 0, pl.counter_bytes, stream));
+}
+
+void note_config(const char* path, const Plan& pl, int mma_n) {
+  std::snprintf(g_last_config, sizeof(g_last_config),
+                "path=%s tile=128x%d tiles=%dx%d kb=%d grid=%d dp_tiles=%d sk_iters=%lld ws=%zu", path, mma_n,
+                pl.s.m_tiles, pl.s.n_tiles, pl.s.kb_total, pl.grid, pl.s.dp_tiles, pl.s.sk_iters, pl.ws_bytes());
+  if (env_ll("SMGEMM_LOG", 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
+}
+
+unsigned long long wait_limit() {
+  return static_cast<unsigned long long>(env_ll("SMGEMM_WAIT_LIMIT_NS", static_cast<long long>(kWaitLimitNs)));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* smgemm_status_string(smgemm_status st) {
+  switch (st) {
+    case SMGEMM_OK: return "ok";
+    case SMGEMM_ERR_INVALID_ARG: return "invalid argument";
+    case SMGEMM_ERR_UNSUPPORTED: return "unsupported combination";
+    case SMGEMM_ERR_ALIGNMENT: return "misaligned pointer or leading dimension (TMA needs 16 bytes)";
+    case SMGEMM_ERR_WORKSPACE: return "workspace missing or too small";
+    case SMGEMM_ERR_CUDA: return "CUDA error or no sm_100 device";
+    case SMGEMM_ERR_TIMEOUT: return "kernel abandoned a barrier wait";
+  }
+  return "unknown status";
+}
+
+const char* smgemm_last_config(void) { return g_last_config; }
+
+size_t smgemm_workspace_size(int64_t M, int64_t N, int64_t K, int kind) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  DevInfo d;
+  if (current_device(d) != SMGEMM_OK) return 0;
+  if (kind == 1) return plan_fp8(M, N, K, d.sms).ws_bytes();
+  // enough for either path (the skinny path is only taken for a row-major A)
+  return std::max(plan_gemm16(M, N, K, SMGEMM_ROW_MAJOR, d.sms).pl.ws_bytes(),
+                  plan_gemm16(M, N, K, SMGEMM_COL_MAJOR, d.sms).pl.ws_bytes());
+}
+
+smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_dtype ab_dtype,
+                        smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b, int64_t ldb,
+                        const void* bias, smgemm_dtype bias_dtype, smgemm_act act, void* C, smgemm_dtype c_dtype,
+                        int64_t ldc, void* workspace, size_t workspace_bytes, smgemm_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!fits_int(M) || !fits_int(N) || !fits_int(K)) return SMGEMM_ERR_INVALID_ARG;
+  if (ab_dtype != SMGEMM_BF16 && ab_dtype != SMGEMM_F16) return SMGEMM_ERR_UNSUPPORTED;
+  if (!valid_layout(layout_a) || !valid_layout(layout_b)) return SMGEMM_ERR_INVALID_ARG;
+  if (!valid_out_dtype(c_dtype) || !valid_act(act)) return SMGEMM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return SMGEMM_OK;
+  smgemm_status st = check_output(M, N, C, c_dtype, ldc, bias, bias_dtype, act);
+  if (st != SMGEMM_OK) return st;
+  if (K > 0) {
+    if (A == nullptr || B == nullptr) return SMGEMM_ERR_INVALID_ARG;
+    if (lda < (layout_a == SMGEMM_ROW_MAJOR ? K : M) || ldb < (layout_b == SMGEMM_ROW_MAJOR ? N : K))
+      return SMGEMM_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || (lda * 2) % 16 != 0 || (ldb * 2) % 16 != 0) return SMGEMM_ERR_ALIGNMENT;
+  }
+  DevInfo d;
+  if (current_device(d) != SMGEMM_OK) return SMGEMM_ERR_CUDA;
+  if (K == 0) {
+    std::snprintf(g_last_config, sizeof(g_last_config), "path=fill");
+    return launch_status(launch_fill_epilogue(static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C,
+                                              c_dtype, ldc, stream));
+  }
+  const Gemm16Plan g = plan_gemm16(M, N, K, layout_a, d.sms);
+  const CUtensorMapDataType dt =
+      ab_dtype == SMGEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const uint32_t fmt = ab_dtype == SMGEMM_BF16 ? 1u : 0u;
+  CUtensorMap tm_a, tm_b;
+  Tc16Params p{};
+  bool ok;
+  if (g.skinny) {
+    // MMA "A" = the weight B (128 output columns per tile), MMA "B" = the tokens A.
+    const bool w_mn = (layout_b == SMGEMM_ROW_MAJOR);
+    if (w_mn) ok = encode_2d(&tm_a, dt, B, N, K, ldb * 2, 64, g.bk);
+    else ok = encode_2d(&tm_a, dt, B, K, N, ldb * 2, 64, 128);
+    ok = ok && encode_2d(&tm_b, dt, A, K, M, lda * 2, 64, g.mma_n);
+    p.a_mn_major = w_mn ? 1 : 0;
+    p.b_mn_major = 0;
+    p.idesc = idesc_f32acc(fmt, fmt, w_mn ? 1u : 0u, 0u, 128, g.mma_n);
+  } else {
+    const bool a_mn = (layout_a == SMGEMM_COL_MAJOR);
+    const bool b_mn = (layout_b == SMGEMM_ROW_MAJOR);
+    if (a_mn) ok = encode_2d(&tm_a, dt, A, M, K, lda * 2, 64, g.bk);
+    else ok = encode_2d(&tm_a, dt, A, K, M, lda * 2, 64, 128);
+    if (b_mn) ok = ok && encode_2d(&tm_b, dt, B, N, K, ldb * 2, 64, g.bk);
+    else ok = ok && encode_2d(&tm_b, dt, B, K, N, ldb * 2, 64, 256);
+    p.a_mn_major = a_mn ? 1 : 0;
+    p.b_mn_major = b_mn ? 1 : 0;
+    p.idesc = idesc_f32acc(fmt, fmt, a_mn ? 1u : 0u, b_mn ? 1u : 0u, 128, 256);
+  }
+  if (!ok) return SMGEMM_ERR_CUDA;
+  p.s = g.pl.s;
+  p.e = EpiArgs{static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C, c_dtype, ldc};
+  p.wait_limit_ns = wait_limit();
+  st = prepare_workspace(g.pl, workspace, workspace_bytes, stream, &p.slots, &p.counters);
+  if (st != SMGEMM_OK) return st;
+  note_config(g.skinny ? "skinny" : "large", g.pl, g.mma_n);
+  return launch_status(launch_gemm_tc16(tm_a, tm_b, p, g.v, g.pl.grid, stream));
+}
+
+smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_t* Aq, const float* sa,
+                                   const uint8_t* Bq, const float* sb, const void* bias, smgemm_dtype bias_dtype,
+                                   smgemm_act act, void* C, smgemm_dtype c_dtype, int64_t ldc, void* workspace,
+                                   size_t workspace_bytes, smgemm_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!fits_int(M) || !fits_int(N) || !fits_int(K)) return SMGEMM_ERR_INVALID_ARG;
+  if (!valid_out_dtype(c_dtype) || !valid_act(act)) return SMGEMM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return SMGEMM_OK;
+  smgemm_status st = check_output(M, N, C, c_dtype, ldc, bias, bias_dtype, act);
+  if (st != SMGEMM_OK) return st;
+  if (K > 0) {
+    if (Aq == nullptr || Bq == nullptr || sa == nullptr || sb == nullptr) return SMGEMM_ERR_INVALID_ARG;
+    if (!aligned16(Aq) || !aligned16(Bq) || K % 16 != 0) return SMGEMM_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(sa) & 3u) || (reinterpret_cast<uintptr_t>(sb) & 3u)) return SMGEMM_ERR_ALIGNMENT;
+  }
+  DevInfo d;
+  if (current_device(d) != SMGEMM_OK) return SMGEMM_ERR_CUDA;
+  if (K == 0) {
+    std::snprintf(g_last_config, sizeof(g_last_config), "path=fill");
+    return launch_status(launch_fill_epilogue(static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C,
+                                              c_dtype, ldc, stream));
+  }
+  const Plan pl = plan_fp8(M, N, K, d.sms);
+  CUtensorMap tm_a, tm_b;
+  bool ok = encode_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, Aq, K, M, K, 128, 128);
+  ok = ok && encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, Bq, K, N, K, 128, 128);
+  if (!ok) return SMGEMM_ERR_CUDA;
+  Fp8Params p{};
+  p.s = pl.s;
+  p.e = EpiArgs{static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C, c_dtype, ldc};
+  p.K = static_cast<int>(K);
+  p.idesc = idesc_f32acc(0u, 0u, 0u, 0u, 128, 128);
+  p.sa = sa;
+  p.sb = sb;
+  p.nb_count = static_cast<int>((N + 127) / 128);
+  p.wait_limit_ns = wait_limit();
+  st = prepare_workspace(pl, workspace, workspace_bytes, stream, &p.slots, &p.counters);
+  if (st != SMGEMM_OK) return st;
+  note_config("fp8", pl, 128);
+  return launch_status(launch_gemm_fp8(tm_a, tm_b, p, pl.grid, stream));
+}
+
+smgemm_status quantize_fp8_blockwise(const float* X, int64_t rows, int64_t cols, smgemm_layout layout_x,
+                                     int64_t ldx, int group_rows, uint8_t* Q, float* scales,
+                                     smgemm_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (rows < 0 || cols < 0 || !valid_layout(layout_x)) return SMGEMM_ERR_INVALID_ARG;
+  if (group_rows != 1 && group_rows != 128) return SMGEMM_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return SMGEMM_OK;
+  if (X == nullptr || Q == nullptr || scales == nullptr) return SMGEMM_ERR_INVALID_ARG;
+  if (ldx < (layout_x == SMGEMM_ROW_MAJOR ? cols : rows)) return SMGEMM_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Q) || (ldx * 4) % 16 != 0 || (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return SMGEMM_ERR_ALIGNMENT;
+  DevInfo d;
+  if (current_device(d) != SMGEMM_OK) return SMGEMM_ERR_CUDA;
+  const long long rs = layout_x == SMGEMM_ROW_MAJOR ? ldx : 1;
+  const long long cs = layout_x == SMGEMM_ROW_MAJOR ? 1 : ldx;
+  cudaError_t e = group_rows == 1 ? launch_quant_1x128(X, rows, cols, rs, cs, Q, scales, stream)
+                                  : launch_quant_128x128(X, rows, cols, rs, cs, Q, scales, stream);
+  return launch_status(e);
+}
+
+smgemm_status smgemm_check(smgemm_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) {
+    cudaGetLastError();
+    return SMGEMM_ERR_CUDA;
+  }
+  const unsigned e = take_error_word_tc16() | take_error_word_fp8() | take_error_word_misc();
+  return (e & kErrTimeout) ? SMGEMM_ERR_TIMEOUT : SMGEMM_OK;
+}
+
+smgemm_status smgemm_selftest_wait_timeout(uint32_t limit_us, smgemm_stream_t stream_) {
+  DevInfo d;
+  if (current_device(d) != SMGEMM_OK) return SMGEMM_ERR_CUDA;
+  if (limit_us == 0 || limit_us > 10000000u) return SMGEMM_ERR_INVALID_ARG;
+  return launch_status(
+      launch_wait_selftest(static_cast<unsigned long long>(limit_us) * 1000ull, reinterpret_cast<cudaStream_t>(stream_)));
+}
+
+int64_t smgemm_schedule_dump(int64_t M, int64_t N, int64_t K, int kind, smgemm_layout layout_a, int num_sms,
+                             int32_t* out, int64_t cap) {
+  if (M <= 0 || N <= 0 || K <= 0 || num_sms <= 0) return 0;
+  const Plan pl = kind == 1 ? plan_fp8(M, N, K, num_sms) : plan_gemm16(M, N, K, layout_a, num_sms).pl;
+  int64_t n = 0;
+  for (int c = 0; c < pl.grid; ++c) {
+    WorkIter it;
+    it.init(pl.s, c);
+    Seg seg;
+    while (it.next(pl.s, seg)) {
+      if (out != nullptr && n < cap) {
+        int mt, nt;
+        tile_coords(pl.s, seg.tile, mt, nt);
+        int32_t* r = out + 7 * n;
+        r[0] = c; r[1] = seg.tile; r[2] = mt; r[3] = nt; r[4] = seg.kb0; r[5] = seg.kb1;
+        r[6] = seg.tile < pl.s.dp_tiles ? -1 : seg.slot;
+      }
+      ++n;
+    }
+  }
+  return n;
+}
+
+}  // extern "C"

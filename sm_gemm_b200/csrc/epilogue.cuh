@@ -1,0 +1,100 @@
+// Fused GEMM epilogue: FP32 accumulator + bias[n] -> activation -> one round-to-
+// nearest-even cast to the output type -> store. The bias add and activation run in
+// registers before the single write-back, as the DeepGEMM kernel-library walkthrough
+// (zwxr.cn), section 5.1 recommends; "为什么我们要死磕GEMM" (kwkr.cn), section 2.1
+// defines the linear layer as GEMM + bias add.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace smg {
+
+struct EpiArgs {
+  int M, N;            // output C is M x N, row-major
+  const void* bias;    // nullable, N entries
+  int bias_dtype;      // kF32 / kBF16 / kF16
+  int act;             // kActNone / kActGeluTanh / kActSilu
+  void* C;
+  int c_dtype;         // kF32 / kBF16 / kF16
+  long long ldc;
+};
+
+__device__ __forceinline__ float act_apply(float x, int act) {
+  if (act == 1) {  // GeLU, tanh form
+    const float c = 0.7978845608028654f;  // sqrt(2/pi)
+    return 0.5f * x * (1.0f + tanhf(c * (x + 0.044715f * x * x * x)));
+  }
+  if (act == 2) return x / (1.0f + expf(-x));  // SiLU
+  return x;
+}
+
+__device__ __forceinline__ float load_bias(const void* bias, int dtype, int idx) {
+  if (dtype == 0) return static_cast<const float*>(bias)[idx];
+  if (dtype == 1) return __bfloat162float(static_cast<const __nv_bfloat16*>(bias)[idx]);
+  return __half2float(static_cast<const __half*>(bias)[idx]);
+}
+
+__device__ __forceinline__ void store_one(void* C, int dtype, long long off, float x) {
+  if (dtype == 0) static_cast<float*>(C)[off] = x;
+  else if (dtype == 1) static_cast<__nv_bfloat16*>(C)[off] = __float2bfloat16_rn(x);
+  else static_cast<__half*>(C)[off] = __float2half_rn(x);
+}
+
+// 32 consecutive columns col0.. of one output row. The caller guarantees that C and
+// ldc*elem_size are 16-byte aligned (checked by the host), so whole chunks use 16-byte
+// vector stores.
+__device__ __forceinline__ void epi_row32(const EpiArgs& e, int row, int col0, float (&v)[32]) {
+  const bool full = col0 + 32 <= e.N;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    float x = v[j];
+    if (e.bias != nullptr && (full || col0 + j < e.N)) x += load_bias(e.bias, e.bias_dtype, col0 + j);
+    v[j] = act_apply(x, e.act);
+  }
+  if (row >= e.M) return;
+  const long long base = static_cast<long long>(row) * e.ldc + col0;
+  if (full) {
+    if (e.c_dtype == 0) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(e.C) + base);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(e.C) + base);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          if (e.c_dtype == 1) {
+            __nv_bfloat162 t = __floats2bfloat162_rn(v[8 * j + 2 * h], v[8 * j + 2 * h + 1]);
+            w[h] = *reinterpret_cast<uint32_t*>(&t);
+          } else {
+            __half2 t = __floats2half2_rn(v[8 * j + 2 * h], v[8 * j + 2 * h + 1]);
+            w[h] = *reinterpret_cast<uint32_t*>(&t);
+          }
+        }
+        dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j < e.N) store_one(e.C, e.c_dtype, base + j, v[j]);
+  }
+}
+
+// CNT consecutive output rows row0.. of one column (transposed accumulator tiles).
+template <int CNT>
+__device__ __forceinline__ void epi_col(const EpiArgs& e, int col, int row0, const float* v) {
+  if (col >= e.N) return;
+  const float b = e.bias != nullptr ? load_bias(e.bias, e.bias_dtype, col) : 0.0f;
+#pragma unroll
+  for (int j = 0; j < CNT; ++j) {
+    const int row = row0 + j;
+    if (row < e.M) store_one(e.C, e.c_dtype, static_cast<long long>(row) * e.ldc + col, act_apply(v[j] + b, e.act));
+  }
+}
+
+}  // namespace smg

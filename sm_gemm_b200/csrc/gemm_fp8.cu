@@ -1,0 +1,273 @@
+// Block-scaled FP8 (E4M3) GEMM with per-K-block scale promotion into FP32.
+//
+// The DeepGEMM kernel-library walkthrough (zwxr.cn), section 2.4 quantises with one
+// FP32 scale per 1x128 group of the activations and per 128x128 block of the
+// weights, and accumulates the low-precision products in FP32 before rescaling. Here
+// each 128-wide K-block kb of a 128x128 output tile is multiplied on the tensor core
+// into an FP32 TMEM partial P_kb (kind::f8f6f4, four K=32 steps), and promotion warps
+// fold it into a register accumulator: acc += (sa[kb,m] * sb[kb,nb]) * P_kb. The
+// scales are arbitrary FP32 values (amax/448), not powers of two, so the hardware
+// block-scaled MMA (UE8M0 / UE4M3 scale factors) cannot apply them exactly; the
+// promotion is done in software. Two TMEM partial buffers let the MMA of kb+1 run
+// while kb is promoted.
+//
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM
+// allocator, warp 3 idle, warps 4..11 promotion + epilogue: warp w reads TMEM lanes
+// 32*(w%4).. (tile rows) and columns 64*((w-4)/4).. (64 of the 128 tile columns).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace smg {
+
+namespace {
+constexpr int kThreads = 384;
+constexpr int kPromoWarp0 = 4;
+constexpr int kPromoThreads = 256;
+constexpr int BM = kFp8BM, BN = kFp8BN, BKB = kFp8BK;  // BK in bytes = elements
+constexpr int A_BYTES = BM * BKB;                       // 16 KB
+constexpr int B_BYTES = BN * BKB;                       // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int STAGES = 6;
+constexpr int TCOLS = 256;  // two 128-column FP32 partial buffers
+
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int i) {
+  // K-major tile of 128 rows x 128 bytes, 128-byte swizzle; K step i = 32 bytes.
+  return sdesc_sw128(base + i * 32, 16, 1024);
+}
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_fp8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                    const Fp8Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
+  const uint32_t bar_base = smem_base + STAGES * STAGE_BYTES;
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto pfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
+  auto pempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
+  uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  volatile int* reduce_flag = reinterpret_cast<volatile int*>(misc + 8);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(pfull_bar(b), 1);
+      mbar_init(pempty_bar(b), 8);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), TCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const TileSched& s = p.s;
+  const uint64_t limit = p.wait_limit_ns;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    long long issued = 0;
+    WorkIter it;
+    it.init(s, blockIdx.x);
+    Seg seg;
+    bool ok = true;
+    while (ok && it.next(s, seg)) {
+      int mt, nt;
+      tile_coords(s, seg.tile, mt, nt);
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit)) { ok = false; break; }
+        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
+        tma_load_2d(sa, &tm_a, full_bar(stage), kb * BKB, mt * BM);
+        tma_load_2d(sa + A_BYTES, &tm_b, full_bar(stage), kb * BKB, nt * BN);
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok) {
+      int st = stage;
+      uint32_t ph = phase;
+      volatile int no_abort = 0;
+      for (long long i = 0; i < issued && i < STAGES; ++i) {
+        if (--st < 0) { st = STAGES - 1; ph ^= 1u; }
+        mbar_wait(full_bar(st), ph, &no_abort, limit);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    long long kcount = 0;  // K-blocks issued by this CTA: selects the partial buffer
+    WorkIter it;
+    it.init(s, blockIdx.x);
+    Seg seg;
+    bool ok = true;
+    while (ok && it.next(s, seg)) {
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++kcount) {
+        const int buf = static_cast<int>(kcount & 1);
+        const uint32_t bphase = static_cast<uint32_t>((kcount >> 1) & 1);
+        if (!mbar_wait(pempty_bar(buf), bphase ^ 1u, abort_flag, limit)) { ok = false; break; }
+        if (!mbar_wait(full_bar(stage), phase, abort_flag, limit)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        const uint32_t d_tmem = tmem_base + buf * BN;
+#pragma unroll
+        for (int k = 0; k < BKB / 32; ++k)
+          umma_f8(d_tmem, kmajor_desc(sa, k), kmajor_desc(sa + A_BYTES, k), p.idesc, k > 0 ? 1u : 0u);
+        umma_commit(empty_bar(stage));
+        umma_commit(pfull_bar(buf));
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    umma_commit(drain_bar);
+    volatile int no_abort = 0;
+    mbar_wait(drain_bar, 0, &no_abort, limit);
+  } else if (warp >= kPromoWarp0) {
+    // ---------------------------------------------------------------- promotion + epilogue
+    const int q = warp & 3;
+    const int half = (warp - kPromoWarp0) >> 2;
+    const int r_local = q * 32 + lane;
+    const int c_local0 = half * 64;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const int ptid = threadIdx.x - kPromoWarp0 * 32;
+    const int M = p.e.M;
+    long long kcount = 0;
+    WorkIter it;
+    it.init(s, blockIdx.x);
+    Seg seg;
+    // `dead` is warp-uniform. After an abandoned wait the loop keeps walking the
+    // (deterministic) segment list without touching TMEM or memory, so every named
+    // barrier below is still reached by all 256 promotion threads.
+    bool dead = false;
+    while (it.next(s, seg)) {
+      int mt, nt;
+      tile_coords(s, seg.tile, mt, nt);
+      const int row = mt * BM + r_local;
+      const bool row_ok = row < M;
+      float acc[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++kcount) {
+        const int buf = static_cast<int>(kcount & 1);
+        const uint32_t bphase = static_cast<uint32_t>((kcount >> 1) & 1);
+        // scale of this row and K-block; issued before the wait so its latency hides
+        const float sa = row_ok ? __ldg(p.sa + static_cast<long long>(kb) * M + row) : 0.0f;
+        const float sb = __ldg(p.sb + static_cast<long long>(kb) * p.nb_count + nt);
+        if (!dead) dead = !mbar_wait(pfull_bar(buf), bphase, abort_flag, limit);
+        dead = __any_sync(0xffffffffu, dead);
+        if (dead) continue;
+        tc_fence_after();
+        const float sc = sa * sb;
+        const uint32_t taddr = tmem_base + lane_addr + buf * BN + c_local0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + h * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[h * 32 + j] = fmaf(sc, __uint_as_float(r[j]), acc[h * 32 + j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pempty_bar(buf));
+      }
+
+      const bool whole = (seg.kb0 == 0 && seg.kb1 == s.kb_total);
+      const int col0 = nt * BN + c_local0;
+      if (whole) {
+        if (!dead) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = acc[h * 32 + j];
+            epi_row32(p.e, row, col0 + h * 32, v);
+          }
+        }
+      } else {
+        // Stream-K partial: store, then the last contributor reduces in CTA order.
+        float* my_slot = p.slots + (static_cast<size_t>(blockIdx.x) * 2 + seg.slot) * (BM * BN);
+        if (!dead) {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) my_slot[(c_local0 + j) * BM + r_local] = acc[j];
+        }
+        const long long t_sk = seg.tile - s.dp_tiles;
+        __threadfence();
+        named_barrier_sync(1, kPromoThreads);
+        if (ptid == 0) {
+          const int c_lo = sk_owner(s, t_sk * s.kb_total);
+          const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
+          int n = 0;
+          for (int c = c_lo; c <= c_hi; ++c) n += sk_bound(s, c) < sk_bound(s, c + 1);
+          const bool any_dead = *abort_flag != 0;
+          const int old = any_dead ? -1 : atomicAdd(p.counters + t_sk, 1);
+          *reduce_flag = (!any_dead && old == n - 1);
+        }
+        named_barrier_sync(1, kPromoThreads);
+        if (*reduce_flag) {
+          __threadfence();
+          const int c_lo = sk_owner(s, t_sk * s.kb_total);
+          const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+#pragma unroll 1
+            for (int cc = c_lo; cc <= c_hi; ++cc) {
+              if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
+              const float* src = p.slots + (static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * (BM * BN);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] += __ldcg(src + (c_local0 + h * 32 + j) * BM + r_local);
+            }
+            epi_row32(p.e, row, col0 + h * 32, v);
+          }
+        }
+        named_barrier_sync(1, kPromoThreads);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem_base, TCOLS);
+}
+
+cudaError_t launch_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Fp8Params& p,
+                            int grid, cudaStream_t stream) {
+  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5) + 16;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(gemm_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return e;
+  gemm_fp8_kernel<<<grid, kThreads, SMEM, stream>>>(tm_a, tm_b, p);
+  return cudaGetLastError();
+}
+
+unsigned take_error_word_fp8() { return take_error_word(); }
+
+}  // namespace smg

@@ -1,0 +1,327 @@
+// Persistent warp-specialised tcgen05 GEMM for 16-bit inputs (bf16 / f16), FP32
+// accumulation in TMEM, fused bias + activation + cast epilogue.
+//
+// One kernel template serves both paths of gemm_bf16:
+//  - large tiles: MMA tile 128 x 256 (MMA "A" = A rows, MMA "B" = B columns), BK = 64;
+//  - skinny M (the thin-and-tall LM-head / decode shape of "为什么我们要死磕GEMM",
+//    kwkr.cn, sections 2.2 and 7.2): swap-AB, the weight supplies the 128 MMA rows
+//    and the few tokens are the MMA N (16..64), so the tensor core streams the
+//    weight once; the epilogue writes the transposed accumulator.
+//
+// Warp roles (256 threads): warp 0 = TMA producer, warp 1 = MMA issuer, warp 2 =
+// TMEM allocator, warp 3 idle, warps 4..7 = epilogue (warp w reads TMEM lanes
+// 32*(w%4) .. +31). Shared memory holds an S-stage ring of operand tiles with
+// full/empty mbarriers; TMEM holds two accumulators so the epilogue of one tile
+// overlaps the MMAs of the next (DeepGEMM kernel-library walkthrough, zwxr.cn,
+// section 2.3: keep the copy running ahead of the math). The fused epilogue is that
+// page's section 5.1; the FP32 accumulator its section 2.4.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace smg {
+
+namespace {
+
+constexpr int kEpiWarp0 = 4;
+constexpr int kThreads = 256;
+
+template <int R, int BK>
+__device__ __forceinline__ void load_operand(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                             int mn_major, int r0, int k0) {
+  if (!mn_major) {
+    // K-major: boxes of {64 (K), R (rows)}, BK/64 of them along K, R*128 bytes apart.
+#pragma unroll
+    for (int j = 0; j < BK / 64; ++j) tma_load_2d(dst + j * R * 128, map, bar, k0 + 64 * j, r0);
+  } else {
+    // MN-major: boxes of {64 (rows), BK (K)}, R/64 of them along the rows, BK*128 bytes apart.
+#pragma unroll
+    for (int j = 0; j < R / 64; ++j) tma_load_2d(dst + j * BK * 128, map, bar, r0 + 64 * j, k0);
+  }
+}
+
+// Descriptor of the i-th 16-element K slice of an operand tile laid out by load_operand.
+template <int R, int BK>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int mn_major, int i) {
+  if (!mn_major) return sdesc_sw128(base + (i >> 2) * (R * 128) + (i & 3) * 32, 16, 1024);
+  return sdesc_sw128(base + i * 2048, BK * 128, 1024);
+}
+
+template <int MMA_N>
+struct TmemCols {
+  static constexpr int v = (2 * MMA_N <= 32) ? 32 : (2 * MMA_N <= 64) ? 64 : (2 * MMA_N <= 128) ? 128
+                          : (2 * MMA_N <= 256) ? 256 : 512;
+};
+
+}  // namespace
+
+template <int MMA_N, int BK, int STAGES, bool SWAP>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                     const Tc16Params p) {
+  constexpr int A_BYTES = 128 * BK * 2;
+  constexpr int B_BYTES = MMA_N * BK * 2;
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr int KSTEPS = BK / 16;
+  constexpr int TCOLS = TmemCols<MMA_N>::v;
+  constexpr int CH = MMA_N < 32 ? MMA_N : 32;  // epilogue chunk (TMEM columns per load)
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
+  const uint32_t bar_base = smem_base + STAGES * STAGE_BYTES;
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
+  uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  volatile int* reduce_flag = reinterpret_cast<volatile int*>(misc + 8);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), TCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const TileSched& s = p.s;
+  const uint64_t limit = p.wait_limit_ns;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    long long issued = 0;
+    WorkIter it;
+    it.init(s, blockIdx.x);
+    Seg seg;
+    bool ok = true;
+    while (ok && it.next(s, seg)) {
+      int mt, nt;
+      tile_coords(s, seg.tile, mt, nt);
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit)) { ok = false; break; }
+        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
+        load_operand<128, BK>(sa, &tm_a, full_bar(stage), p.a_mn_major, mt * 128, kb * BK);
+        load_operand<MMA_N, BK>(sa + A_BYTES, &tm_b, full_bar(stage), p.b_mn_major, nt * MMA_N, kb * BK);
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok) {
+      // Wait (bounded, independent of the abort flag) for copies still in flight.
+      int st = stage;
+      uint32_t ph = phase;
+      volatile int no_abort = 0;
+      for (long long i = 0; i < issued && i < STAGES; ++i) {
+        if (--st < 0) { st = STAGES - 1; ph ^= 1u; }
+        mbar_wait(full_bar(st), ph, &no_abort, limit);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int local = 0;
+    WorkIter it;
+    it.init(s, blockIdx.x);
+    Seg seg;
+    bool ok = true;
+    while (ok && it.next(s, seg)) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, limit)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * MMA_N;
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb) {
+        if (!mbar_wait(full_bar(stage), phase, abort_flag, limit)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+        for (int k = 0; k < KSTEPS; ++k) {
+          umma_f16(d_tmem, operand_desc<128, BK>(sa, p.a_mn_major, k),
+                   operand_desc<MMA_N, BK>(sb, p.b_mn_major, k), p.idesc,
+                   (kb > seg.kb0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(empty_bar(stage));
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      umma_commit(tfull_bar(acc));
+      ++local;
+    }
+    // Drain: every MMA issued above completes before TMEM is released.
+    umma_commit(drain_bar);
+    volatile int no_abort = 0;
+    mbar_wait(drain_bar, 0, &no_abort, limit);
+  } else if (warp >= kEpiWarp0) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int r_local = q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const int epi_tid = threadIdx.x - kEpiWarp0 * 32;
+    int local = 0;
+    WorkIter it;
+    it.init(s, blockIdx.x);
+    Seg seg;
+    // `dead` is warp-uniform; after an abandoned wait the loop keeps walking the
+    // segment list without touching TMEM or memory so that all 128 epilogue threads
+    // still reach every named barrier.
+    bool dead = false;
+    while (it.next(s, seg)) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!dead) dead = !mbar_wait(tfull_bar(acc), acc_phase, abort_flag, limit);
+      dead = __any_sync(0xffffffffu, dead);
+      int mt, nt;
+      tile_coords(s, seg.tile, mt, nt);
+      const uint32_t tacc = tmem_base + lane_addr + acc * MMA_N;
+      const bool whole = (seg.kb0 == 0 && seg.kb1 == s.kb_total);
+      float* my_slot = p.slots + (static_cast<size_t>(blockIdx.x) * 2 + seg.slot) * (128 * MMA_N);
+      if (!dead) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < MMA_N / CH; ++c) {
+          uint32_t r[32];
+          if constexpr (CH == 32) {
+            tmem_ld_32x32b_x32(tacc + c * 32, r);
+          } else {
+            uint32_t r16[16];
+            tmem_ld_32x32b_x16(tacc + c * 16, r16);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) r[j] = r16[j];
+          }
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          if (whole) {
+            if constexpr (SWAP) epi_col<CH>(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
+            else epi_row32(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
+          } else {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) my_slot[(c * CH + j) * 128 + r_local] = v[j];
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(acc));
+      }
+
+      if (!whole) {
+        // Stream-K fix-up: the last contributor of the tile sums every contributor's
+        // partial in CTA order (= K order) and runs the epilogue.
+        const long long t_sk = seg.tile - s.dp_tiles;
+        __threadfence();
+        named_barrier_sync(1, 128);
+        if (epi_tid == 0) {
+          const int c_lo = sk_owner(s, t_sk * s.kb_total);
+          const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
+          int n = 0;
+          for (int c = c_lo; c <= c_hi; ++c) n += sk_bound(s, c) < sk_bound(s, c + 1);
+          const bool any_dead = *abort_flag != 0;
+          const int old = any_dead ? -1 : atomicAdd(p.counters + t_sk, 1);
+          *reduce_flag = (!any_dead && old == n - 1);
+        }
+        named_barrier_sync(1, 128);
+        if (*reduce_flag) {
+          __threadfence();
+          const int c_lo = sk_owner(s, t_sk * s.kb_total);
+          const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
+#pragma unroll 1
+          for (int c = 0; c < MMA_N / CH; ++c) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+#pragma unroll 1
+            for (int cc = c_lo; cc <= c_hi; ++cc) {
+              if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
+              const float* src = p.slots + (static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * (128 * MMA_N);
+#pragma unroll
+              for (int j = 0; j < CH; ++j) v[j] += __ldcg(src + (c * CH + j) * 128 + r_local);
+            }
+            if constexpr (SWAP) epi_col<CH>(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
+            else epi_row32(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
+          }
+        }
+        named_barrier_sync(1, 128);
+      }
+      ++local;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem_base, TCOLS);
+}
+
+// ------------------------------------------------------------------ host launchers
+
+template <int MMA_N, int BK, int STAGES, bool SWAP>
+static cudaError_t launch_tc16(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Tc16Params& p,
+                               int grid, cudaStream_t stream) {
+  constexpr int STAGE_BYTES = 128 * BK * 2 + MMA_N * BK * 2;
+  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5) + 16;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  auto kern = gemm_tc16_kernel<MMA_N, BK, STAGES, SWAP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, SMEM, stream>>>(tm_a, tm_b, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc16(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Tc16Params& p,
+                             Tc16Variant v, int grid, cudaStream_t stream) {
+  switch (v) {
+    case Tc16Variant::kLarge: return launch_tc16<256, 64, 4, false>(tm_a, tm_b, p, grid, stream);
+    case Tc16Variant::kSkinny16: return launch_tc16<16, 128, 6, true>(tm_a, tm_b, p, grid, stream);
+    case Tc16Variant::kSkinny32: return launch_tc16<32, 128, 5, true>(tm_a, tm_b, p, grid, stream);
+    case Tc16Variant::kSkinny64: return launch_tc16<64, 128, 4, true>(tm_a, tm_b, p, grid, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+int tc16_mma_n(Tc16Variant v) {
+  switch (v) {
+    case Tc16Variant::kLarge: return 256;
+    case Tc16Variant::kSkinny16: return 16;
+    case Tc16Variant::kSkinny32: return 32;
+    case Tc16Variant::kSkinny64: return 64;
+  }
+  return 0;
+}
+
+int tc16_bk(Tc16Variant v) { return v == Tc16Variant::kLarge ? 64 : 128; }
+
+unsigned take_error_word_tc16() { return take_error_word(); }
+
+}  // namespace smg

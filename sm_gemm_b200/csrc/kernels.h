@@ -1,0 +1,71 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernels. Not installed.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "epilogue.cuh"
+#include "sm100.cuh"
+
+namespace smg {
+
+// Element types and activations, numerically equal to the public smgemm_* enums.
+constexpr int kF32 = 0, kBF16 = 1, kF16 = 2, kE4M3 = 3;
+constexpr int kActNone = 0, kActGeluTanh = 1, kActSilu = 2;
+
+// Default limit of every bounded barrier wait inside the kernels.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+struct Tc16Params {
+  TileSched s;
+  EpiArgs e;                // output, bias, activation
+  uint32_t idesc;           // tcgen05 instruction descriptor
+  int a_mn_major;           // MMA "A" operand tile is MN-major (else K-major)
+  int b_mn_major;           // MMA "B" operand tile is MN-major (else K-major)
+  float* slots;             // stream-K partial tiles: [num_ctas][2][MMA_N][128] floats
+  int* counters;            // stream-K arrival counters, one per stream-K tile, zeroed per call
+  unsigned long long wait_limit_ns;
+};
+
+enum class Tc16Variant { kLarge, kSkinny16, kSkinny32, kSkinny64 };
+
+cudaError_t launch_gemm_tc16(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Tc16Params& p,
+                             Tc16Variant v, int grid, cudaStream_t stream);
+int tc16_mma_n(Tc16Variant v);
+int tc16_bk(Tc16Variant v);
+
+struct Fp8Params {
+  TileSched s;
+  EpiArgs e;
+  int K;
+  uint32_t idesc;
+  const float* sa;          // [KB][M]
+  const float* sb;          // [KB][NB]
+  int nb_count;             // NB = ceil(N/128)
+  float* slots;             // [num_ctas][2][128][128] floats
+  int* counters;
+  unsigned long long wait_limit_ns;
+};
+
+cudaError_t launch_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Fp8Params& p,
+                            int grid, cudaStream_t stream);
+constexpr int kFp8BM = 128, kFp8BN = 128, kFp8BK = 128;
+
+// C[m, n] = act(bias[n]) (or act(0)) for the K == 0 degenerate GEMM.
+cudaError_t launch_fill_epilogue(int M, int N, const void* bias, int bias_dtype, int act, void* C,
+                                 int c_dtype, long long ldc, cudaStream_t stream);
+
+cudaError_t launch_quant_1x128(const float* X, long long rows, long long cols, long long rs,
+                               long long cs, uint8_t* Q, float* S, cudaStream_t stream);
+cudaError_t launch_quant_128x128(const float* X, long long K, long long N, long long rs,
+                                 long long cs, uint8_t* Q, float* S, cudaStream_t stream);
+
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
+
+// Per-translation-unit device error words (see sm100.cuh).
+unsigned take_error_word_tc16();
+unsigned take_error_word_fp8();
+unsigned take_error_word_misc();
+
+}  // namespace smg

@@ -1,0 +1,229 @@
+// FP32 -> FP8 E4M3 group quantiser (1x128 row groups for activations, 128x128 blocks
+// for weights), the memory-bound producer of the operands of the block-scaled GEMM.
+//
+// Per group, following the DeepGEMM kernel-library walkthrough (zwxr.cn),
+// section 2.4: amax = max|x| over the group's elements, scale s = amax / 448 (FP32,
+// correctly rounded division; 1.0 for an all-zero group), code = E4M3(x / s) with a
+// correctly rounded division and the hardware's round-to-nearest-even, saturating
+// conversion (cvt.rn.satfinite.e4m3x2.f32). The result is bit-exact with a plain
+// sequential implementation: the max is order-independent and every other step is
+// a single correctly rounded operation.
+//
+// Plus two small kernels: the K == 0 epilogue fill, and the bounded-wait self-test.
+#include <cuda_fp8.h>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace smg {
+
+namespace {
+
+__device__ __forceinline__ float group_scale(float amax) {
+  return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+}
+
+// Two codes packed little-endian: x0 -> low byte, x1 -> high byte.
+__device__ __forceinline__ uint32_t e4m3x2(float x0, float x1) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// One warp per 1x128 group of a row-major X (element (r, c) at r*ldx + c).
+__global__ void __launch_bounds__(256) quant_1x128_rows_kernel(const float* __restrict__ X, long long rows,
+                                                               long long cols, long long ldx,
+                                                               uint8_t* __restrict__ Q, float* __restrict__ S) {
+  const long long kbn = (cols + 127) / 128;
+  const long long g = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (g >= rows * kbn) return;
+  const int lane = threadIdx.x & 31;
+  const long long r = g / kbn, kb = g - r * kbn;
+  const long long c0 = kb * 128 + lane * 4;
+  const float* src = X + r * ldx;
+  float v[4];
+  const bool vec = (kb * 128 + 128 <= cols) && ((ldx & 3) == 0);
+  if (vec) {
+    const float4 t = __ldcs(reinterpret_cast<const float4*>(src + c0));
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = (c0 + j < cols) ? src[c0 + j] : 0.0f;
+  }
+  float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+  amax = warp_max(amax);
+  const float s = group_scale(amax);
+  const uint32_t lo = e4m3x2(__fdiv_rn(v[0], s), __fdiv_rn(v[1], s));
+  const uint32_t hi = e4m3x2(__fdiv_rn(v[2], s), __fdiv_rn(v[3], s));
+  uint8_t* dst = Q + r * cols + c0;
+  if (vec && (cols & 3) == 0) {
+    *reinterpret_cast<uint32_t*>(dst) = lo | (hi << 16);
+  } else {
+    const uint32_t w = lo | (hi << 16);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (c0 + j < cols) dst[j] = static_cast<uint8_t>(w >> (8 * j));
+  }
+  if (lane == 0) S[kb * rows + r] = s;
+}
+
+// One thread per (row, group) of a column-major X (element (r, c) at c*ldx + r):
+// consecutive threads read consecutive rows, so every load of the warp is coalesced.
+__global__ void __launch_bounds__(256) quant_1x128_cols_kernel(const float* __restrict__ X, long long rows,
+                                                               long long cols, long long ldx,
+                                                               uint8_t* __restrict__ Q, float* __restrict__ S) {
+  const long long kbn = (cols + 127) / 128;
+  const long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long kb = blockIdx.y;
+  if (r >= rows || kb >= kbn) return;
+  const long long c0 = kb * 128;
+  const long long c1 = (c0 + 128 < cols) ? c0 + 128 : cols;
+  float amax = 0.0f;
+  for (long long c = c0; c < c1; ++c) amax = fmaxf(amax, fabsf(X[c * ldx + r]));
+  const float s = group_scale(amax);
+  uint8_t* dst = Q + r * cols;
+  for (long long c = c0; c < c1; c += 2) {
+    const float x0 = X[c * ldx + r];
+    const float x1 = (c + 1 < c1) ? X[(c + 1) * ldx + r] : 0.0f;
+    const uint32_t w = e4m3x2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
+    dst[c] = static_cast<uint8_t>(w);
+    if (c + 1 < c1) dst[c + 1] = static_cast<uint8_t>(w >> 8);
+  }
+  S[kb * rows + r] = s;
+}
+
+// One CTA per 128x128 block of the weight X[K, N] (element (k, n) at k*rs + n*cs).
+// The block is staged transposed in shared memory ([n][k], padded row of 129) so the
+// codes can be written as Q[n][k] rows of up to 128 contiguous bytes.
+constexpr int kQPitch = 129;
+__global__ void __launch_bounds__(256) quant_128x128_kernel(const float* __restrict__ X, long long K, long long N,
+                                                            long long rs, long long cs, uint8_t* __restrict__ Q,
+                                                            float* __restrict__ S) {
+  extern __shared__ float tile[];  // [128][kQPitch]
+  __shared__ float warp_amax[8];
+  const long long kb = blockIdx.y, nb = blockIdx.x;
+  const long long k0 = kb * 128, n0 = nb * 128;
+  const long long nbn = (N + 127) / 128;
+  const int t = threadIdx.x;
+  const bool n_contig = (cs == 1);
+  float amax = 0.0f;
+#pragma unroll 4
+  for (int i = 0; i < 64; ++i) {
+    const int idx = i * 256 + t;
+    const int kk = n_contig ? (idx >> 7) : (idx & 127);
+    const int nn = n_contig ? (idx & 127) : (idx >> 7);
+    const long long k = k0 + kk, n = n0 + nn;
+    const float x = (k < K && n < N) ? __ldcs(X + k * rs + n * cs) : 0.0f;
+    amax = fmaxf(amax, fabsf(x));
+    tile[nn * kQPitch + kk] = x;
+  }
+  amax = warp_max(amax);
+  if ((t & 31) == 0) warp_amax[t >> 5] = amax;
+  __syncthreads();
+  float m = warp_amax[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = fmaxf(m, warp_amax[w]);
+  const float s = group_scale(m);
+  if (t == 0) S[kb * nbn + nb] = s;
+
+  // Thread t: output row n = n0 + t/2, k range [64*(t&1), +64).
+  const int nn = t >> 1;
+  const int kh = (t & 1) * 64;
+  const long long n = n0 + nn;
+  if (n >= N) return;
+  uint8_t* dst = Q + n * K + k0 + kh;
+  const bool vec = (k0 + kh + 64 <= K) && ((K & 15) == 0);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float* src = tile + nn * kQPitch + kh + u * 16 + h * 4;
+      const uint32_t lo = e4m3x2(__fdiv_rn(src[0], s), __fdiv_rn(src[1], s));
+      const uint32_t hi = e4m3x2(__fdiv_rn(src[2], s), __fdiv_rn(src[3], s));
+      w[h] = lo | (hi << 16);
+    }
+    if (vec) {
+      *reinterpret_cast<uint4*>(dst + u * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (k0 + kh + u * 16 + j < K) dst[u * 16 + j] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
+    }
+  }
+}
+
+__global__ void fill_epilogue_kernel(int M, int N, const void* bias, int bias_dtype, int act, void* C,
+                                     int c_dtype, long long ldc) {
+  const long long total = static_cast<long long>(M) * N;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / N, c = i - r * N;
+    const float b = bias != nullptr ? load_bias(bias, bias_dtype, static_cast<int>(c)) : 0.0f;
+    store_one(C, c_dtype, r * ldc + c, act_apply(b, act));
+  }
+}
+
+// Waits on an mbarrier that nothing arrives on; the bounded wait gives up after
+// `limit_ns`, records kErrTimeout and the kernel returns normally.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);
+  __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_quant_1x128(const float* X, long long rows, long long cols, long long rs,
+                               long long cs, uint8_t* Q, float* S, cudaStream_t stream) {
+  const long long kbn = (cols + 127) / 128;
+  if (cs == 1) {
+    const long long groups = rows * kbn;
+    const long long blocks = (groups + 7) / 8;
+    quant_1x128_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(X, rows, cols, rs, Q, S);
+  } else {
+    dim3 grid(static_cast<unsigned>((rows + 255) / 256), static_cast<unsigned>(kbn));
+    quant_1x128_cols_kernel<<<grid, 256, 0, stream>>>(X, rows, cols, cs, Q, S);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_128x128(const float* X, long long K, long long N, long long rs, long long cs,
+                                 uint8_t* Q, float* S, cudaStream_t stream) {
+  const int smem = 128 * kQPitch * static_cast<int>(sizeof(float));
+  cudaError_t e = cudaFuncSetAttribute(quant_128x128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((K + 127) / 128));
+  quant_128x128_kernel<<<grid, 256, smem, stream>>>(X, K, N, rs, cs, Q, S);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_epilogue(int M, int N, const void* bias, int bias_dtype, int act, void* C,
+                                 int c_dtype, long long ldc, cudaStream_t stream) {
+  const long long total = static_cast<long long>(M) * N;
+  const long long blocks = (total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096;
+  fill_epilogue_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(M, N, bias, bias_dtype, act, C,
+                                                                          c_dtype, ldc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+  return cudaGetLastError();
+}
+
+unsigned take_error_word_misc() { return take_error_word(); }
+
+}  // namespace smg

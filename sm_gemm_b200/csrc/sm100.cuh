@@ -1,0 +1,322 @@
+// Blackwell (sm_100a) building blocks shared by the GEMM kernels: mbarriers with a
+// bounded wait, TMA tile loads, tcgen05 (TMEM allocation, MMA, commit, loads), the
+// UMMA shared-memory and instruction descriptors, and the persistent tile scheduler
+// (grouped rasterisation, data-parallel tiles followed by a stream-K range).
+//
+// The pipeline is the "copy the next tile while the current one is multiplied"
+// scheme of the DeepGEMM kernel-library walkthrough (zwxr.cn), section 2.3, built
+// from TMA + an S-stage mbarrier ring instead of thread copies and a 2-buffer swap.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace smg {
+
+// ------------------------------------------------------------------ error word
+
+// Bit set in the device error word when a bounded wait gives up. The host reads and
+// clears it in smgemm_check(). Each translation unit has its own word (internal
+// linkage, no relocatable device code needed) and exports a take_error_word_* hook.
+constexpr unsigned kErrTimeout = 1u;
+
+namespace {
+__device__ unsigned int g_error_word = 0;
+
+// Returns and clears this translation unit's device error word (current device).
+inline unsigned take_error_word() {
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(v)) != cudaSuccess) return 0;
+  if (v != 0) {
+    const unsigned z = 0;
+    cudaMemcpyToSymbol(g_error_word, &z, sizeof(z));
+  }
+  return v;
+}
+}  // namespace
+
+// ------------------------------------------------------------------ small helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
+__device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
+
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ------------------------------------------------------------------ mbarrier
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait until the phase with the given parity of barrier `bar` has completed, for at
+// most `limit_ns` nanoseconds. On expiry: record kErrTimeout in the device error word,
+// raise the CTA-wide abort flag and return false. Every later wait of the CTA returns
+// false at once when the abort flag is up, so a stalled pipeline drains in about one
+// limit instead of one per wait.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (*abort_flag) return false;
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(&g_error_word, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ TMA
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// 2-D tiled bulk tensor copy global -> shared; completion is counted in bytes on `bar`.
+// c0 is the innermost (contiguous) coordinate. No multicast.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int32_t c0, int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// ------------------------------------------------------------------ tcgen05 / TMEM
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], 16-bit inputs (bf16 or f16), FP32 accumulate.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// D[tmem] (+)= A * B with 8-bit float inputs (E4M3 here), FP32 accumulate.
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// Arrive once on `bar` when every tcgen05.mma issued so far by this thread has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets lane (base + t),
+// columns col .. col+31 of `taddr`.
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ UMMA descriptors
+
+// Shared-memory matrix descriptor (sm_100 format): start address, leading and stride
+// byte offsets (all >> 4), descriptor version 1, base offset 0, 128-byte swizzle.
+//  - K-major tiles (rows of 128 B along K, 8-row swizzle atoms of 1 KB): SBO = 1024,
+//    LBO unused (16).
+//  - MN-major tiles (rows of 128 B along M/N, one row per k): SBO = 1024 (8 k-rows),
+//    LBO = byte distance between consecutive 64-element M/N atoms.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Instruction descriptor for kind::f16 / kind::f8f6f4 with FP32 accumulation.
+// fmt: kind::f16 -> 0 = F16, 1 = BF16; kind::f8f6f4 -> 0 = E4M3.
+__host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t a_fmt, uint32_t b_fmt, uint32_t a_mn,
+                                                    uint32_t b_mn, uint32_t M, uint32_t N) {
+  return (1u << 4) | (a_fmt << 7) | (b_fmt << 10) | (a_mn << 15) | (b_mn << 16) |
+         ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ tile scheduler
+
+// Work of one launch: an (m_tiles x n_tiles) grid of output tiles, each needing
+// kb_total K-blocks. Tiles [0, dp_tiles) (in rasterised order) go round-robin to the
+// CTAs with their full K range; the remaining tiles form a flat space of
+// sk_iters = (tiles - dp_tiles) * kb_total K-block iterations cut into num_ctas
+// contiguous ranges (stream-K). A tile whose K range is cut is summed in fixed CTA
+// order by whichever contributor finishes last, so results are deterministic.
+struct TileSched {
+  int m_tiles, n_tiles, kb_total;
+  int dp_tiles;
+  int num_ctas;
+  int group_m;
+  long long sk_iters;
+};
+
+struct Seg {
+  int tile;      // rasterised tile index
+  int kb0, kb1;  // K-block range [kb0, kb1)
+  int slot;      // 0 / 1: which workspace slot a partial result of this CTA goes to
+};
+
+__host__ __device__ inline long long sk_bound(const TileSched& s, int c) {
+  return (s.sk_iters * c) / s.num_ctas;
+}
+
+// CTA owning stream-K iteration i.
+__host__ __device__ inline int sk_owner(const TileSched& s, long long i) {
+  int c = static_cast<int>((i * s.num_ctas) / (s.sk_iters > 0 ? s.sk_iters : 1));
+  if (c >= s.num_ctas) c = s.num_ctas - 1;
+  while (c + 1 < s.num_ctas && sk_bound(s, c + 1) <= i) ++c;
+  while (c > 0 && sk_bound(s, c) > i) --c;
+  return c;
+}
+
+// Rasterised tile index -> (m tile, n tile): groups of group_m tile-rows, walked down
+// the rows of a group first, then across the columns, so CTAs running together share
+// B columns and a small band of A rows in L2.
+__host__ __device__ inline void tile_coords(const TileSched& s, int t, int& mt, int& nt) {
+  const int per_group = s.group_m * s.n_tiles;
+  const int g = t / per_group;
+  const int first_m = g * s.group_m;
+  int gm = s.m_tiles - first_m;
+  if (gm > s.group_m) gm = s.group_m;
+  const int r = t - g * per_group;
+  mt = first_m + r % gm;
+  nt = r / gm;
+}
+
+struct WorkIter {
+  int dp_next;
+  long long sk_begin, sk_pos, sk_end;
+
+  __host__ __device__ void init(const TileSched& s, int cta) {
+    dp_next = cta;
+    sk_begin = sk_pos = sk_bound(s, cta);
+    sk_end = sk_bound(s, cta + 1);
+  }
+  __host__ __device__ bool next(const TileSched& s, Seg& out) {
+    if (dp_next < s.dp_tiles) {
+      out.tile = dp_next;
+      out.kb0 = 0;
+      out.kb1 = s.kb_total;
+      out.slot = 0;
+      dp_next += s.num_ctas;
+      return true;
+    }
+    if (sk_pos < sk_end) {
+      const long long t = sk_pos / s.kb_total;
+      const int kb0 = static_cast<int>(sk_pos - t * s.kb_total);
+      long long rem = sk_end - sk_pos;
+      int kb1 = s.kb_total;
+      if (rem < kb1 - kb0) kb1 = kb0 + static_cast<int>(rem);
+      out.tile = s.dp_tiles + static_cast<int>(t);
+      out.kb0 = kb0;
+      out.kb1 = kb1;
+      out.slot = (sk_pos == sk_begin) ? 0 : 1;
+      sk_pos += kb1 - kb0;
+      return true;
+    }
+    return false;
+  }
+};
+
+// The slot a contributor CTA `c` used for stream-K tile `t_sk` (index among the
+// stream-K tiles): 0 if the tile holds the start of c's range, else 1.
+__host__ __device__ inline int sk_slot_of(const TileSched& s, int c, long long t_sk) {
+  const long long begin = sk_bound(s, c);
+  return (begin / s.kb_total == t_sk) ? 0 : 1;
+}
+
+}  // namespace smg

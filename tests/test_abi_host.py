@@ -1,0 +1,208 @@
+"""Host-side tests of the C-ABI library (no GPU needed).
+
+The library must load without a GPU driver and export every function that
+include/smgemm.h declares. Argument errors are reported before any CUDA call, so
+they are exercised here with fake device addresses. The persistent schedule
+(data-parallel tiles + stream-K ranges) is checked through smgemm_schedule_dump:
+every (tile, K-block) pair is computed exactly once, segments of one tile are
+contiguous in K, and partial tiles use the slots the kernels' fix-up expects.
+"""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+import sm_gemm_b200 as sg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "smgemm.h")
+
+# A fake, 16-byte aligned device address: these tests only reach host-side validation.
+FAKE = 0x7F0000001000
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)) - {"if"})
+
+
+def test_header_declares_the_abi():
+    names = _declared_functions()
+    for want in ("gemm_bf16", "gemm_fp8_blockscaled", "quantize_fp8_blockwise", "smgemm_workspace_size",
+                 "smgemm_status_string", "smgemm_check"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", sg.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    missing = [n for n in _declared_functions() if n not in exported]
+    assert not missing, missing
+    L = sg.lib()
+    for n in _declared_functions():
+        assert hasattr(L, n)
+
+
+def test_library_has_no_driver_dependency():
+    out = subprocess.run(["ldd", sg.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out
+
+
+def test_status_strings():
+    for s in range(7):
+        assert len(sg.status_string(s)) > 0
+    assert sg.status_string(99) == "unknown status"
+
+
+needs_cpu = pytest.mark.skipif(torch.cuda.is_available(),
+                               reason="fake-pointer validation tests run only where no GPU can be reached")
+
+
+def _gemm(M=256, N=256, K=256, A=FAKE, ab=sg.BF16, la=sg.ROW_MAJOR, lda=None, B=FAKE, lb=sg.COL_MAJOR,
+          ldb=None, bias=None, bias_dt=sg.F32, act=0, Cp=FAKE, c_dt=sg.BF16, ldc=None, ws=None, wsb=0):
+    lda = lda if lda is not None else (K if la == sg.ROW_MAJOR else M)
+    ldb = ldb if ldb is not None else (N if lb == sg.ROW_MAJOR else K)
+    ldc = ldc if ldc is not None else N
+    return sg.lib().gemm_bf16(M, N, K, A, ab, la, lda, B, lb, ldb, bias, bias_dt, act, Cp, c_dt, ldc, ws, wsb,
+                              None)
+
+
+@needs_cpu
+def test_gemm_bf16_argument_errors():
+    assert _gemm(M=-1) == sg.ERR_INVALID_ARG
+    assert _gemm(K=1 << 31) == sg.ERR_INVALID_ARG
+    assert _gemm(ab=sg.F32) == sg.ERR_UNSUPPORTED
+    assert _gemm(ab=sg.E4M3) == sg.ERR_UNSUPPORTED
+    assert _gemm(la=7) == sg.ERR_INVALID_ARG
+    assert _gemm(act=9) == sg.ERR_INVALID_ARG
+    assert _gemm(c_dt=sg.E4M3) == sg.ERR_INVALID_ARG
+    assert _gemm(A=None) == sg.ERR_INVALID_ARG
+    assert _gemm(Cp=None) == sg.ERR_INVALID_ARG
+    assert _gemm(lda=100) == sg.ERR_INVALID_ARG              # lda < K
+    assert _gemm(ldc=100) == sg.ERR_INVALID_ARG              # ldc < N
+    assert _gemm(A=FAKE + 2) == sg.ERR_ALIGNMENT
+    assert _gemm(lda=260) == sg.ERR_ALIGNMENT                # 520 bytes: not a multiple of 16
+    assert _gemm(Cp=FAKE + 8) == sg.ERR_ALIGNMENT
+    assert _gemm(N=250, ldc=250) == sg.ERR_ALIGNMENT         # 500 bytes
+    assert _gemm(bias=FAKE + 2, bias_dt=sg.F32) == sg.ERR_ALIGNMENT
+    assert _gemm(bias=FAKE, bias_dt=9) == sg.ERR_INVALID_ARG
+
+
+@needs_cpu
+def test_empty_shapes_are_noops_and_valid_calls_need_a_device():
+    assert _gemm(M=0) == sg.OK
+    assert _gemm(N=0, Cp=None) == sg.OK
+    # a valid call with no reachable sm_100 device fails cleanly
+    assert _gemm() == sg.ERR_CUDA
+    assert _gemm(K=0) == sg.ERR_CUDA
+    assert sg.lib().smgemm_check(None) == sg.ERR_CUDA
+    assert sg.lib().smgemm_selftest_wait_timeout(1000, None) == sg.ERR_CUDA
+    assert sg.workspace_size(4096, 4096, 4096) == 0          # unknown device -> 0
+
+
+@needs_cpu
+def test_fp8_and_quant_argument_errors():
+    L = sg.lib()
+    def fp8(M=256, N=256, K=256, Aq=FAKE, sa=FAKE, Bq=FAKE, sb=FAKE, Cp=FAKE, ldc=256, c_dt=sg.BF16):
+        return L.gemm_fp8_blockscaled(M, N, K, Aq, sa, Bq, sb, None, 0, 0, Cp, c_dt, ldc, None, 0, None)
+    assert fp8(K=200) == sg.ERR_ALIGNMENT                     # K must be a multiple of 16
+    assert fp8(sa=None) == sg.ERR_INVALID_ARG
+    assert fp8(Aq=FAKE + 1) == sg.ERR_ALIGNMENT
+    assert fp8(sb=FAKE + 2) == sg.ERR_ALIGNMENT
+    assert fp8(M=0) == sg.OK
+    assert fp8() == sg.ERR_CUDA
+    def q(rows=256, cols=256, layout=sg.ROW_MAJOR, ldx=256, g=1, X=FAKE, Q=FAKE, S=FAKE):
+        return L.quantize_fp8_blockwise(X, rows, cols, layout, ldx, g, Q, S, None)
+    assert q(g=64) == sg.ERR_INVALID_ARG
+    assert q(ldx=100) == sg.ERR_INVALID_ARG
+    assert q(ldx=258) == sg.ERR_ALIGNMENT
+    assert q(X=FAKE + 4) == sg.ERR_ALIGNMENT
+    assert q(Q=FAKE + 1) == sg.ERR_ALIGNMENT
+    assert q(rows=0) == sg.OK
+    assert q() == sg.ERR_CUDA
+
+
+# ------------------------------------------------------------------ persistent schedule
+
+def _check_schedule(M, N, K, kind=0, layout_a=sg.ROW_MAJOR, sms=148, bk=None):
+    d = sg.schedule_dump(M, N, K, kind, layout_a, sms)
+    assert d.shape[0] > 0
+    ctas = d[:, 0]
+    assert ctas.min() == 0 and ctas.max() < sms
+    # every (tile, K-block) exactly once
+    if bk is None:
+        bk = 128 if kind == 1 else (128 if (M <= 64 and layout_a == sg.ROW_MAJOR) else 64)
+    kb_total = -(-K // bk)
+    seen = {}
+    for c, t, mt, nt, k0, k1, slot in d:
+        assert 0 <= k0 < k1 <= kb_total
+        for kb in range(k0, k1):
+            assert (t, kb) not in seen
+            seen[(t, kb)] = c
+    tiles = sorted({int(t) for t in d[:, 1]})
+    assert tiles == list(range(len(tiles)))
+    assert len(seen) == len(tiles) * kb_total
+    # tile -> (mt, nt) is a bijection onto the tile grid
+    coords = {(int(t), int(mt), int(nt)) for _, t, mt, nt, *_ in d}
+    assert len({(m, n) for _, m, n in coords}) == len(tiles)
+    # a split tile's contributors are consecutive CTAs in K order, and each partial
+    # segment's slot is 0 iff it is the first segment of that CTA
+    first_seg = {}
+    for i, (c, t, mt, nt, k0, k1, slot) in enumerate(d):
+        if slot >= 0:
+            first_seg.setdefault(int(c), i)
+        else:
+            assert k0 == 0 and k1 == kb_total and int(c) not in first_seg   # DP tiles come first
+    by_tile = {}
+    for i, (c, t, mt, nt, k0, k1, slot) in enumerate(d):
+        by_tile.setdefault(int(t), []).append((int(k0), int(c), int(slot), i))
+    for t, segs in by_tile.items():
+        segs.sort()
+        if len(segs) > 1:
+            cs = [c for _, c, _, _ in segs]
+            assert cs == sorted(cs) and len(set(cs)) == len(cs)
+            for k0, c, slot, i in segs:
+                assert slot == (0 if first_seg[c] == i else 1)
+    # stream-K work is balanced: per-CTA K-block counts differ by at most one
+    sk = d[d[:, 6] >= 0]
+    if sk.size:
+        per = np.bincount(sk[:, 0], weights=sk[:, 5] - sk[:, 4])
+        per = per[per > 0]
+        assert per.max() - per.min() <= 1
+    return d
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 4096, 4096), (1024, 16384, 4096), (1024, 4096, 16384),
+                                   (300, 600, 500), (64, 64, 64), (128, 256, 4096), (67, 50, 33)])
+def test_schedule_large_covers_each_kblock_once(M, N, K):
+    _check_schedule(M, N, K, layout_a=sg.COL_MAJOR if M <= 64 else sg.ROW_MAJOR)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16, 64])
+def test_schedule_skinny_lm_head(M):
+    d = _check_schedule(M, 128256, 4096)
+    # all 148 SMs get work and the K-blocks are shared within 1 of each other
+    per_cta = np.bincount(d[:, 0], weights=d[:, 5] - d[:, 4], minlength=148)
+    assert per_cta.min() > 0 and per_cta.max() - per_cta.min() <= 1
+
+
+@pytest.mark.parametrize("M,N,K", [(2048, 16384, 4096), (256, 384, 1024), (130, 260, 128)])
+def test_schedule_fp8(M, N, K):
+    _check_schedule(M, N, K, kind=1)
+
+
+def test_schedule_small_grid_override(monkeypatch):
+    monkeypatch.setenv("SMGEMM_GRID", "3")
+    d = _check_schedule(1000, 1000, 1000)
+    assert d[:, 0].max() == 2
+    monkeypatch.setenv("SMGEMM_SCHED", "sk")
+    _check_schedule(300, 300, 3000)
+    monkeypatch.setenv("SMGEMM_SCHED", "dp")
+    d = _check_schedule(300, 300, 3000)
+    assert (d[:, 4] == 0).all()

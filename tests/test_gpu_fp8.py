@@ -1,0 +1,153 @@
+"""GPU parity of quantize_fp8_blockwise (bit-exact) and gemm_fp8_blockscaled
+(tolerance; exact on integer codes) against the CPU oracle, through the C-ABI.
+
+Group scaling follows the DeepGEMM kernel-library walkthrough (zwxr.cn), section 2.4.
+The quantiser must reproduce the oracle's scales and codes bit for bit, including
+ragged groups, all-zero groups, signed zeros and saturation; the GEMM must meet the
+contract computed from the same quantised operands.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sm_gemm_b200 as sg
+import synth
+from _parity import check_tolerance
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_quant(X: np.ndarray, group_rows: int, layout: str = "row"):
+    t = torch.from_numpy(np.ascontiguousarray(X))
+    if layout == "row":
+        R, Cn = X.shape
+        ld = -(-Cn // 4) * 4
+        buf = torch.zeros((R, ld), dtype=torch.float32, device="cuda")
+        buf[:, :Cn] = t.cuda()
+        Xd = buf[:, :Cn]
+    else:
+        R, Cn = X.shape
+        ld = -(-R // 4) * 4
+        buf = torch.zeros((Cn, ld), dtype=torch.float32, device="cuda")
+        buf[:, :R] = t.t().cuda()
+        Xd = buf[:, :R].t()
+    Q, S = sg.quantize_fp8_blockwise(Xd, group_rows)
+    assert sg.check() == sg.OK
+    return Q.cpu().numpy(), S.cpu().numpy()
+
+
+@pytest.mark.parametrize("shape", [(37, 300), (128, 128), (1, 1), (5, 1000), (2048, 4096)])
+@pytest.mark.parametrize("layout", ["row", "col"])
+def test_quant_1x128_bit_exact(cuda_device, shape, layout):
+    X = synth.normal_with_outliers(70, 0, shape)
+    Q, S = _gpu_quant(X, 1, layout)
+    Qr, Sr = oracle.quant_1x128(X)
+    assert np.array_equal(S.view(np.uint32), Sr.view(np.uint32))
+    assert np.array_equal(Q, Qr)
+
+
+@pytest.mark.parametrize("shape", [(300, 200), (128, 128), (1, 1), (4096, 1024), (257, 130)])
+@pytest.mark.parametrize("layout", ["row", "col"])
+def test_quant_128x128_bit_exact(cuda_device, shape, layout):
+    X = synth.normal_with_outliers(71, 0, shape)
+    Q, S = _gpu_quant(X, 128, layout)
+    Qr, Sr = oracle.quant_128x128(X)
+    assert np.array_equal(S.view(np.uint32), Sr.view(np.uint32))
+    assert np.array_equal(Q, Qr)
+
+
+def test_quant_special_values(cuda_device):
+    """Signed zeros, tiny values that round to zero, all-zero groups, a constant group,
+    exact ties and values at the saturation edge."""
+    X = np.zeros((4, 256), dtype=np.float32)
+    X[0, :8] = [-0.0, 0.0, -1e-30, 1e-30, 448.0, -448.0, 1.0, -1.0]
+    X[1, :128] = -3.0
+    X[2, :128] = np.float32(1.0) + np.arange(128, dtype=np.float32) * np.float32(2.0 ** -7)
+    X[3, 128:] = 2.0 ** (np.arange(128) % 20 - 10)
+    for g in (1, 128):
+        Q, S = _gpu_quant(X if g == 1 else np.ascontiguousarray(X.T), g)
+        Qr, Sr = (oracle.quant_1x128(X) if g == 1 else oracle.quant_128x128(np.ascontiguousarray(X.T)))
+        assert np.array_equal(S.view(np.uint32), Sr.view(np.uint32))
+        assert np.array_equal(Q, Qr)
+
+
+def _quantised_problem(M, N, K, seed):
+    A = synth.normal_with_outliers(seed, 0, (M, K))
+    B = synth.normal_with_outliers(seed, 1, (K, N))
+    qa, sa = oracle.quant_1x128(A)
+    qb, sb = oracle.quant_128x128(B)
+    return qa, sa, qb, sb
+
+
+def _run_fp8(qa, sa, qb, sb, out_dt=torch.bfloat16, bias=None, act="none"):
+    M, N = qa.shape[0], qb.shape[0]
+    out = torch.empty((M, -(-N // 8) * 8), dtype=out_dt, device="cuda")[:, :N]
+    sg.gemm_fp8_blockscaled(torch.from_numpy(qa).cuda(), torch.from_numpy(sa).cuda(),
+                            torch.from_numpy(qb).cuda(), torch.from_numpy(sb).cuda(),
+                            bias=None if bias is None else bias.cuda(), act=act, out=out)
+    assert sg.check() == sg.OK
+    return out.float().cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (300, 260, 384), (64, 1000, 1024), (257, 129, 2048)])
+def test_fp8_gemm_within_tolerance(cuda_device, M, N, K):
+    qa, sa, qb, sb = _quantised_problem(M, N, K, seed=M + N + K)
+    got = _run_fp8(qa, sa, qb, sb)
+    ref, acc = oracle.gemm_fp8(qa, sa, qb, sb, out_dtype=oracle.BF16, want_absacc=True)
+    check_tolerance(got, ref, acc, torch.bfloat16, what=f"fp8 {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("sched", ["dp", "sk", "auto"])
+def test_fp8_gemm_integer_codes_unit_scales_exact(cuda_device, monkeypatch, sched):
+    monkeypatch.setenv("SMGEMM_SCHED", sched)
+    rs = np.random.RandomState(5)
+    M, N, K = 300, 400, 1024
+    qa = oracle.e4m3_encode(rs.randint(-8, 9, (M, K)).astype(np.float32))
+    qb = oracle.e4m3_encode(rs.randint(-8, 9, (N, K)).astype(np.float32))
+    sa = np.ones((K // 128, M), np.float32)
+    sb = np.ones((K // 128, -(-N // 128)), np.float32)
+    got = _run_fp8(qa, sa, qb, sb, out_dt=torch.float32)
+    ref = oracle.gemm_fp8(qa, sa, qb, sb, out_dtype=oracle.F32)
+    assert np.array_equal(got, ref)
+
+
+def test_fp8_gemm_power_of_two_scales_exact(cuda_device):
+    rs = np.random.RandomState(6)
+    M, N, K = 200, 300, 512
+    qa = oracle.e4m3_encode(rs.randint(-8, 9, (M, K)).astype(np.float32))
+    qb = oracle.e4m3_encode(rs.randint(-8, 9, (N, K)).astype(np.float32))
+    # scale products in 2^[-4, 4] keep every FP32 partial sum exact (<= 24 significant bits)
+    sa = (2.0 ** rs.randint(-2, 3, (K // 128, M))).astype(np.float32)
+    sb = (2.0 ** rs.randint(-2, 3, (K // 128, 3))).astype(np.float32)
+    got = _run_fp8(qa, sa, qb, sb, out_dt=torch.float32)
+    ref = oracle.gemm_fp8(qa, sa, qb, sb, out_dtype=oracle.F32)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("act", ["gelu_tanh", "silu"])
+def test_fp8_gemm_bias_activation(cuda_device, act):
+    qa, sa, qb, sb = _quantised_problem(200, 300, 256, seed=77)
+    bias = torch.from_numpy(synth.normal(77, 5, (300,), 0.5)).to(torch.bfloat16)
+    got = _run_fp8(qa, sa, qb, sb, bias=bias, act=act)
+    bb = bias.view(torch.int16).numpy().view(np.uint16)
+    ref, acc = oracle.gemm_fp8(qa, sa, qb, sb, bias=bb, bias_dtype=oracle.BF16,
+                               act={"gelu_tanh": oracle.ACT_GELU_TANH, "silu": oracle.ACT_SILU}[act],
+                               out_dtype=oracle.BF16, want_absacc=True)
+    check_tolerance(got, ref, acc, torch.bfloat16, what=f"fp8 {act}")
+
+
+def test_quantise_then_gemm_end_to_end_on_gpu(cuda_device):
+    """Both quantisations and the GEMM on the GPU; codes and scales must equal the
+    oracle's, so the GEMM reference is computed from identical operands."""
+    A = synth.normal_with_outliers(80, 0, (256, 512))
+    B = synth.normal_with_outliers(80, 1, (512, 384))
+    qa, sa = sg.quantize_fp8_blockwise(torch.from_numpy(A).cuda(), 1)
+    qb, sb = sg.quantize_fp8_blockwise(torch.from_numpy(B).cuda(), 128)
+    out = sg.gemm_fp8_blockscaled(qa, sa, qb, sb, out_dtype=torch.bfloat16)
+    assert sg.check() == sg.OK
+    qa_r, sa_r = oracle.quant_1x128(A)
+    qb_r, sb_r = oracle.quant_128x128(B)
+    assert np.array_equal(qa.cpu().numpy(), qa_r) and np.array_equal(qb.cpu().numpy(), qb_r)
+    ref, acc = oracle.gemm_fp8(qa_r, sa_r, qb_r, sb_r, out_dtype=oracle.BF16, want_absacc=True)
+    check_tolerance(out.float().cpu().numpy(), ref, acc, torch.bfloat16, what="quant+gemm")
