@@ -1,0 +1,486 @@
+"""Benchmark of the GEMM library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {smgemm,reference}] [--headline-only]
+
+One step is one call of the hot path on one batch of synthetic input. The headline
+workload is the square BF16 GEMM (A[4096,4096] row-major x B[4096,4096] column-major,
+FP32 accumulation, BF16 out); its throughput in TFLOP/s is ``value``. The other
+workloads (tiny FP16, the FFN pair, FP8 block-scaled GEMM and its quantiser, the
+LM-head GEMM at M in {1,4,16,64}) are timed the same way and reported under
+``configs``. FLOPs are 2*M*N*K; bytes count every operand once.
+
+Timing: W untimed warm-up steps, then K steps between CUDA events on the launching
+stream, bracketed by a barrier and a device synchronise; the maximum over ranks is
+taken. Workloads whose operands fit in L2 rotate over enough copies that the bytes
+touched between two uses of one copy exceed L2. SM clocks and throttle reasons are
+sampled with nvidia-smi during the headline's timed region.
+
+``--impl reference`` times the CPU oracle (plain FP64 triple loop) on a bounded
+sample of the same workload on the host cores, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "GEMM TFLOPS & % of B200 tensor peak (BF16/FP8); GB/s & % HBM for skinny M"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["sm_gemm_b200/csrc/gemm_tc16.cu", "sm_gemm_b200/csrc/sm100.cuh",
+                  "sm_gemm_b200/csrc/epilogue.cuh"]
+
+
+# ----------------------------------------------------------------------------- utilities
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d[kernel][workload]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except (KeyError, ValueError, TypeError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def time_steps(torch, step, warmup: int, steps: int, dist=None):
+    """Device time of `steps` calls of step(i) after `warmup` calls: CUDA events on the
+    current stream, barrier + synchronise on both sides, max over ranks (ms total)."""
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(steps):
+        step(warmup + i)
+    e.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = s.elapsed_time(e)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def n_copies(bytes_per_set: int) -> int:
+    return max(1, -(-2 * L2_BYTES // max(bytes_per_set, 1)) + 1) if bytes_per_set < 2 * L2_BYTES else 1
+
+
+class Ctx:
+    def __init__(self, args, world, dist):
+        import torch
+        import sm_gemm_b200 as sg
+        import synth
+        from sm_gemm_b200 import metrics
+        self.torch, self.sg, self.synth, self.metrics = torch, sg, synth, metrics
+        self.dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+        torch.cuda.set_device(self.dev)
+        self.peaks = load_peaks()
+        self.fp8_peak = 2.0 * self.peaks["bf16_tflops"]   # measured bf16 x nominal fp8/bf16 ratio (2)
+        self.W, self.K = args.warmup, args.steps
+        self.world, self.dist = world, dist
+        self.launches = 0
+        self.results = {}
+
+    def time(self, step, launches_per_step=1, warmup=None, steps=None):
+        w = self.W if warmup is None else warmup
+        k = self.K if steps is None else steps
+        ms = time_steps(self.torch, step, w, k, self.dist)
+        self.launches += launches_per_step * k
+        return ms
+
+    def record(self, name, ms_total, steps, flops=None, nbytes=None, peak_tf=None, extra=None):
+        t = ms_total / steps / 1e3
+        r = {"us_per_call": round(t * 1e6, 2)}
+        if flops is not None:
+            r["tflops"] = round(flops / t / 1e12, 1)
+            if peak_tf:
+                r["frac_tensor_peak"] = round(flops / t / 1e12 / peak_tf, 4)
+        if nbytes is not None:
+            r["gbs"] = round(nbytes / t / 1e9, 1)
+            r["frac_hbm"] = round(nbytes / t / 1e9 / self.peaks["hbm_gbs"], 4)
+        if extra:
+            r.update(extra)
+        self.results[name] = r
+        return r
+
+    def t(self, x, dtype=None):
+        return self.torch.from_numpy(np.ascontiguousarray(x)).to(dtype or self.torch.bfloat16).to(self.dev)
+
+
+def wl_square_bf16(c: Ctx, headline: bool):
+    """Square BF16 4096^3 (the headline): returns the JSON line's core fields."""
+    torch, sg, m = c.torch, c.sg, c.metrics
+    n = 4096
+    d = c.synth.square_bf16(n)
+    A0, Bt0 = c.t(d["A"]), c.t(d["Bt"])
+    set_bytes = m.gemm_bytes(n, n, n, "bf16", "bf16", "bf16")
+    copies = n_copies(set_bytes)
+    As = [A0] + [A0.clone() for _ in range(copies - 1)]
+    Bs = [Bt0] + [Bt0.clone() for _ in range(copies - 1)]
+    Cs = [torch.empty((n, n), dtype=torch.bfloat16, device=c.dev) for _ in range(copies)]
+    ws = torch.empty(max(sg.workspace_size(n, n, n, 0), 16), dtype=torch.uint8, device=c.dev)
+
+    def step(i):
+        j = i % copies
+        sg.gemm_bf16(As[j], Bs[j].t(), out=Cs[j], workspace=ws)
+
+    try:
+        smi_id = "GPU-" + str(torch.cuda.get_device_properties(c.dev).uuid)
+    except Exception:
+        smi_id = str(c.dev.index)
+    with ClockSampler(smi_id) as clk:
+        ms = c.time(step)
+    assert sg.check() == sg.OK
+    flops = m.gemm_flops(n, n, n)
+    plan = sg.last_config()
+    c.record("square_bf16_4096", ms, c.K, flops=flops, peak_tf=c.peaks["bf16_tflops"], extra={"plan": plan})
+    out = {"ms": ms, "flops": flops, "copies": copies, "set_bytes": set_bytes, "plan": plan,
+           "clocks": clk.summary()}
+    if not headline:
+        return out
+    # end to end through the public API from pinned host buffers (H2D inputs, D2H result)
+    Ah = torch.from_numpy(np.ascontiguousarray(d["A"])).to(torch.bfloat16).pin_memory()
+    Bh = torch.from_numpy(np.ascontiguousarray(d["Bt"])).to(torch.bfloat16).pin_memory()
+    Ch = torch.empty((n, n), dtype=torch.bfloat16).pin_memory()
+    Ad, Bd, Cd = torch.empty_like(A0), torch.empty_like(Bt0), torch.empty_like(Cs[0])
+
+    def e2e_step(i):
+        Ad.copy_(Ah, non_blocking=True)
+        Bd.copy_(Bh, non_blocking=True)
+        sg.gemm_bf16(Ad, Bd.t(), out=Cd, workspace=ws)
+        Ch.copy_(Cd, non_blocking=True)
+
+    e2e_steps = max(2, c.K // 4)
+    e2e_ms = c.time(e2e_step, warmup=max(1, c.W // 2), steps=e2e_steps)
+    out["e2e"] = {"value": round(flops * e2e_steps * c.world / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+                  "h2d_bytes_per_step": 2 * n * n * 2, "d2h_bytes_per_step": n * n * 2}
+    return out
+
+
+def wl_tiny_fp16(c: Ctx):
+    torch, sg = c.torch, c.sg
+    t = c.synth.tiny_fp16()
+    A, B = c.t(t["A"], torch.float16), c.t(t["B"], torch.float16)
+    C = torch.empty((64, 64), dtype=torch.float32, device=c.dev)
+    ms = c.time(lambda i: sg.gemm_bf16(A, B, out=C))
+    c.record("tiny_fp16_64", ms, c.K, flops=c.metrics.gemm_flops(64, 64, 64), extra={"plan": sg.last_config()})
+
+
+def wl_ffn(c: Ctx):
+    torch, sg, m = c.torch, c.sg, c.metrics
+    f = c.synth.ffn_pair()
+    X, W1, W2, b1 = c.t(f["X"]), c.t(f["W1"]), c.t(f["W2"]), c.t(f["b1"])
+    H = torch.empty((1024, 16384), dtype=torch.bfloat16, device=c.dev)
+    Y = torch.empty((1024, 4096), dtype=torch.bfloat16, device=c.dev)
+    ws = torch.empty(max(sg.workspace_size(1024, 16384, 4096), sg.workspace_size(1024, 4096, 16384), 16),
+                     dtype=torch.uint8, device=c.dev)
+    ms1 = c.time(lambda i: sg.gemm_bf16(X, W1, bias=b1, act="gelu_tanh", out=H, workspace=ws))
+    p1 = sg.last_config()
+    ms2 = c.time(lambda i: sg.gemm_bf16(H, W2, out=Y, workspace=ws))
+    p2 = sg.last_config()
+    fl = m.gemm_flops(1024, 16384, 4096)
+    pk = c.peaks["bf16_tflops"]
+    c.record("ffn_gemm1_bias_gelu", ms1, c.K, flops=fl, peak_tf=pk, extra={"plan": p1})
+    c.record("ffn_gemm2", ms2, c.K, flops=fl, peak_tf=pk, extra={"plan": p2})
+    c.record("ffn_pair", ms1 + ms2, c.K, flops=2 * fl, peak_tf=pk)
+
+
+def wl_fp8(c: Ctx, quant=True, gemm=True):
+    torch, sg, m = c.torch, c.sg, c.metrics
+    f8 = c.synth.fp8_blockscaled()
+    Af, Bf = c.t(f8["A"], torch.float32), c.t(f8["B"], torch.float32)
+    qa = torch.empty((2048, 4096), dtype=torch.uint8, device=c.dev)
+    sa = torch.empty((32, 2048), dtype=torch.float32, device=c.dev)
+    qb = torch.empty((16384, 4096), dtype=torch.uint8, device=c.dev)
+    sb = torch.empty((32, 128), dtype=torch.float32, device=c.dev)
+    if quant:
+        msa = c.time(lambda i: sg.quantize_fp8_blockwise(Af, 1, Q=qa, scales=sa))
+        msb = c.time(lambda i: sg.quantize_fp8_blockwise(Bf, 128, Q=qb, scales=sb))
+        c.record("quant_1x128_A_2048x4096", msa, c.K, nbytes=m.quant_bytes(2048, 4096, 1))
+        c.record("quant_128x128_B_4096x16384", msb, c.K, nbytes=m.quant_bytes(4096, 16384, 128))
+    else:
+        sg.quantize_fp8_blockwise(Af, 1, Q=qa, scales=sa)
+        sg.quantize_fp8_blockwise(Bf, 128, Q=qb, scales=sb)
+    del Af, Bf
+    if not gemm:
+        return
+    set8 = m.fp8_gemm_bytes(2048, 16384, 4096, "bf16")
+    n8 = n_copies(set8)
+    qas = [qa] + [qa.clone() for _ in range(n8 - 1)]
+    qbs = [qb] + [qb.clone() for _ in range(n8 - 1)]
+    C8 = [torch.empty((2048, 16384), dtype=torch.bfloat16, device=c.dev) for _ in range(n8)]
+    ws = torch.empty(max(sg.workspace_size(2048, 16384, 4096, 1), 16), dtype=torch.uint8, device=c.dev)
+    ms = c.time(lambda i: sg.gemm_fp8_blockscaled(qas[i % n8], sa, qbs[i % n8], sb, out=C8[i % n8], workspace=ws))
+    c.record("fp8_blockscaled_2048x16384x4096", ms, c.K, flops=m.gemm_flops(2048, 16384, 4096), peak_tf=c.fp8_peak,
+             extra={"plan": sg.last_config(), "peak_note": "fp8 peak = 2 x measured bf16 (nominal ratio)"})
+
+
+def wl_lm_head(c: Ctx, ms_list=(1, 4, 16, 64)):
+    torch, sg, m = c.torch, c.sg, c.metrics
+    Wl = c.t(c.synth.lm_head(m=1)["W"])
+    ws = torch.empty(max(max(sg.workspace_size(mm, 128256, 4096) for mm in ms_list), 16), dtype=torch.uint8,
+                     device=c.dev)
+    for mm in ms_list:
+        Xl = c.t(c.synth.lm_head(m=mm, vocab=8)["X"])
+        Cl = torch.empty((mm, 128256), dtype=torch.float32, device=c.dev)
+        ms = c.time(lambda i: sg.gemm_bf16(Xl, Wl, out=Cl, workspace=ws))
+        c.record(f"lm_head_m{mm}", ms, c.K, flops=m.gemm_flops(mm, 128256, 4096),
+                 nbytes=m.gemm_bytes(mm, 128256, 4096, "bf16", "bf16", "f32"), extra={"plan": sg.last_config()})
+
+
+def run_gpu(args, rank: int, world: int, dist):
+    c = Ctx(args, world, dist)
+    if args.only is not None and args.only != "square_bf16":
+        {"tiny_fp16": lambda: wl_tiny_fp16(c), "ffn": lambda: wl_ffn(c),
+         "fp8": lambda: wl_fp8(c, quant=False), "quant": lambda: wl_fp8(c, gemm=False),
+         "lm_head": lambda: wl_lm_head(c)}[args.only]()
+        assert c.sg.check() == c.sg.OK
+        return {"only": args.only, "steps": c.K, "warmup": c.W, "gpu_launches": c.launches, "configs": c.results}
+
+    h = wl_square_bf16(c, headline=args.only is None)
+    if args.only is None and not args.headline_only:
+        wl_tiny_fp16(c)
+        wl_ffn(c)
+        wl_fp8(c)
+        wl_lm_head(c)
+    assert c.sg.check() == c.sg.OK
+    peaks = c.peaks
+    per_launch_s = h["ms"] / c.K / 1e3
+    achieved = h["flops"] / per_launch_s / 1e12
+    line = {
+        "metric": METRIC, "value": round(h["flops"] * c.K * world / (h["ms"] / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": c.K, "warmup": c.W, "ms_per_step": round(h["ms"] / c.K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "square_bf16_4096", "M": 4096, "N": 4096, "K": 4096,
+                   "layout": "A row-major, B column-major (W^T stored K-contiguous)", "out": "bf16",
+                   "accumulate": "fp32",
+                   "l2": f"rotating {h['copies']} input/output sets ({h['copies'] * h['set_bytes'] / 2**20:.0f} MiB) "
+                         f"so reuse distance exceeds L2",
+                   "parallelism": f"replicas{world}" if world > 1 else "single-gpu", "plan": h["plan"]},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "peak_kind": f"{peaks['source']} bf16 burst",
+                     "traffic": recorded_traffic("gemm_tc16_large", "square_bf16_4096"),
+                     "algorithmic_bytes": h["set_bytes"], "kernel": "gemm_tc16_kernel<256,64,4,false>"},
+        "gpu_launches": c.launches,
+        "clocks": h["clocks"],
+        "configs": c.results,
+    }
+    if "e2e" in h:
+        line["e2e"] = h["e2e"]
+    return line
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_cores() -> int:
+    if os.environ.get("OMP_NUM_THREADS"):
+        return int(os.environ["OMP_NUM_THREADS"])
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+_SQUARE_BITS = {}
+
+
+def _square_bits():
+    """The square BF16 workload as raw bf16 bits (generated once per process)."""
+    if not _SQUARE_BITS:
+        import torch
+        import synth
+        d = synth.square_bf16(4096)
+        for k in ("A", "Bt"):
+            _SQUARE_BITS[k] = torch.from_numpy(d[k]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    return _SQUARE_BITS["A"], _SQUARE_BITS["Bt"]
+
+
+def oracle_sample(rows: int):
+    """Oracle (FP64 triple loop) on `rows` full rows of the square BF16 workload.
+    Returns (seconds, flops)."""
+    import oracle
+    n = 4096
+    Afull, Bt = _square_bits()
+    A = Afull[:rows]
+    t0 = time.perf_counter()
+    oracle.gemm(A, Bt.T, a_dtype=oracle.BF16, b_dtype=oracle.BF16, out_dtype=oracle.BF16)
+    return time.perf_counter() - t0, 2 * rows * n * n
+
+
+def cpu_baseline(target_s: float = 10.0):
+    t, _ = oracle_sample(16)
+    rows = int(min(4096, max(16, 16 * target_s / max(t, 1e-3))))
+    t, fl = oracle_sample(rows)
+    return {"value": round(fl / t / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{rows} of 4096 output rows of the square BF16 4096^3 GEMM (FP64 accumulation), "
+                      f"{t:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, as it stands, timed on bounded samples."""
+    t, _ = oracle_sample(8)
+    rows = int(min(4096, max(8, 8 * 4.0 / max(t, 1e-3))))          # ~4 s per step
+    for _ in range(args.warmup):
+        oracle_sample(max(8, rows // 8))
+    total, fl_total = 0.0, 0
+    for _ in range(args.steps):
+        t, fl = oracle_sample(rows)
+        total += t
+        fl_total += fl
+    v = fl_total / total / 1e12
+    cb = {"value": round(v, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+          "sample": f"{rows} of 4096 output rows of the square BF16 4096^3 GEMM per step"}
+    return {"metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "square_bf16_4096", "M": 4096, "N": 4096, "K": 4096,
+                       "sample_rows_per_step": rows},
+            "cpu_baseline": cb,
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="smgemm", choices=["smgemm", "reference"])
+    ap.add_argument("--headline-only", action="store_true")
+    ap.add_argument("--only", default=None,
+                    choices=["square_bf16", "tiny_fp16", "ffn", "fp8", "quant", "lm_head"],
+                    help="time one workload and print its line (profiling runs)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    line = run_gpu(args, rank, world, dist)
+    if rank == 0 and not args.no_cpu_baseline and args.only is None:
+        line["cpu_baseline"] = cpu_baseline()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
