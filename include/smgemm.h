@@ -81,6 +81,29 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K,
                         void* workspace, size_t workspace_bytes, smgemm_stream_t stream);
 
 /*
+ * gemm_bf16_noalloc: gemm_bf16 without a workspace argument, for callers that cannot
+ * allocate device memory - e.g. a plugin or custom-op host that is handed only its
+ * input and output buffers, or a latency-critical decode loop that must not call
+ * cudaMalloc (which can synchronise the device). The GEMM sources have no counterpart
+ * for this entry point; it only changes where the scratch comes from.
+ *   Arguments, results and errors are those of gemm_bf16 (same kernels, same schedule).
+ *   Scratch is a fixed SMGEMM_NOALLOC_SCRATCH_BYTES (16 MiB) array inside the library's
+ *   device image; every GPU that loads the library holds it until the process exits.
+ *   A call whose schedule needs more scratch than that (at most smgemm_workspace_size)
+ *   returns SMGEMM_ERR_WORKSPACE before enqueueing anything. The library allocates nothing.
+ *   All calls share the array and it keeps the previous call's contents (each call
+ *   clears what must start at zero); calls that can overlap on the GPU race on it.
+ *   The first call on each device resolves the array's device address; make that
+ *   first call before any stream capture.
+ */
+#define SMGEMM_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+smgemm_status gemm_bf16_noalloc(int64_t M, int64_t N, int64_t K,
+                                const void* A, smgemm_dtype ab_dtype, smgemm_layout layout_a, int64_t lda,
+                                const void* B, smgemm_layout layout_b, int64_t ldb,
+                                const void* bias, smgemm_dtype bias_dtype, smgemm_act act,
+                                void* C, smgemm_dtype c_dtype, int64_t ldc, smgemm_stream_t stream);
+
+/*
  * gemm_fp8_blockscaled: C[i,j] = cast_c( act( sum_kb sa[kb,i] * sb[kb, j/128] *
  *                                         sum_{k in kb} dec(Aq[i,k]) * dec(Bq[j,k]) + bias[j] ) )
  *
