@@ -108,7 +108,8 @@ struct Plan {
   size_t ws_bytes() const { return counter_bytes + slot_bytes; }
 };
 
-Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, size_t slot_floats) {
+Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, size_t slot_floats,
+               int counters_per_tile = 1) {
   Plan pl;
   const long long T = static_cast<long long>(m_tiles) * n_tiles;
   long long max_ctas = env_ll("SMGEMM_GRID", sms);
@@ -147,7 +148,7 @@ Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, siz
   pl.s.sk_iters = sk_iters;
   pl.grid = static_cast<int>(grid);
   if (sk_iters > 0) {
-    pl.counter_bytes = ((static_cast<size_t>(T - dp) * sizeof(int)) + 255) / 256 * 256;
+    pl.counter_bytes = ((static_cast<size_t>(T - dp) * counters_per_tile * sizeof(int)) + 255) / 256 * 256;
     pl.slot_bytes = static_cast<size_t>(grid) * 2 * slot_floats * sizeof(float);
   }
   return pl;
@@ -202,19 +203,30 @@ smgemm_status launch_status(cudaError_t e) {
 struct Gemm16Plan {
   Tc16Variant v;
   bool skinny;
+  bool pair;  // large tiles on CTA pairs (256 x 256 per cluster)
   Plan pl;
   int mma_n, bk;
 };
 
-Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms) {
+// Large tiles run on CTA pairs unless SMGEMM_PAIR=0 or the device reports no
+// co-resident pair clusters; `sms` is then the SM count and `pair_clusters` the number
+// of co-resident clusters of two.
+Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms, int pair_clusters) {
   Gemm16Plan g;
   const bool force_large = env_ll("SMGEMM_FORCE_LARGE", 0) != 0;
   g.skinny = (M <= 64 && layout_a == SMGEMM_ROW_MAJOR && !force_large);
+  g.pair = !g.skinny && pair_clusters > 0 && env_ll("SMGEMM_PAIR", 1) != 0;
   if (g.skinny) g.v = M <= 16 ? Tc16Variant::kSkinny16 : (M <= 32 ? Tc16Variant::kSkinny32 : Tc16Variant::kSkinny64);
   else g.v = Tc16Variant::kLarge;
   g.mma_n = tc16_mma_n(g.v);
-  g.bk = tc16_bk(g.v);
+  g.bk = g.pair ? tc16_pair_bk() : tc16_bk(g.v);
   const int kb = static_cast<int>((K + g.bk - 1) / g.bk);
+  const int group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", 8));
+  if (g.pair) {
+    g.pl = make_plan(static_cast<int>((M + 255) / 256), static_cast<int>((N + 255) / 256), std::max(kb, 1),
+                     pair_clusters, group_m, static_cast<size_t>(2) * 128 * 256, 2);
+    return g;
+  }
   int m_tiles, n_tiles;
   if (g.skinny) {
     m_tiles = static_cast<int>((N + 127) / 128);  // MMA rows run over the output columns
@@ -223,8 +235,7 @@ Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms) {
     m_tiles = static_cast<int>((M + 127) / 128);
     n_tiles = static_cast<int>((N + g.mma_n - 1) / g.mma_n);
   }
-  g.pl = make_plan(m_tiles, n_tiles, std::max(kb, 1), sms, static_cast<int>(env_ll("SMGEMM_GROUP_M", 8)),
-                   static_cast<size_t>(128) * g.mma_n);
+  g.pl = make_plan(m_tiles, n_tiles, std::max(kb, 1), sms, group_m, static_cast<size_t>(128) * g.mma_n);
   return g;
 }
 
@@ -254,8 +265,10 @@ void note_config(const char* path, const Plan& pl, int mma_n) {
   if (env_ll("SMGEMM_LOG", 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
 }
 
+// Limit of the kernels' bounded barrier waits, in SM cycles.
 unsigned long long wait_limit() {
-  return static_cast<unsigned long long>(env_ll("SMGEMM_WAIT_LIMIT_NS", static_cast<long long>(kWaitLimitNs)));
+  return kCyclesPerNs *
+         static_cast<unsigned long long>(env_ll("SMGEMM_WAIT_LIMIT_NS", static_cast<long long>(kWaitLimitNs)));
 }
 
 }  // namespace
@@ -283,8 +296,9 @@ size_t smgemm_workspace_size(int64_t M, int64_t N, int64_t K, int kind) {
   if (current_device(d) != SMGEMM_OK) return 0;
   if (kind == 1) return plan_fp8(M, N, K, d.sms).ws_bytes();
   // enough for either path (the skinny path is only taken for a row-major A)
-  return std::max(plan_gemm16(M, N, K, SMGEMM_ROW_MAJOR, d.sms).pl.ws_bytes(),
-                  plan_gemm16(M, N, K, SMGEMM_COL_MAJOR, d.sms).pl.ws_bytes());
+  const int pc = tc16_pair_max_clusters();
+  return std::max(plan_gemm16(M, N, K, SMGEMM_ROW_MAJOR, d.sms, pc).pl.ws_bytes(),
+                  plan_gemm16(M, N, K, SMGEMM_COL_MAJOR, d.sms, pc).pl.ws_bytes());
 }
 
 smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_dtype ab_dtype,
@@ -312,7 +326,7 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_d
     return launch_status(launch_fill_epilogue(static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C,
                                               c_dtype, ldc, stream));
   }
-  const Gemm16Plan g = plan_gemm16(M, N, K, layout_a, d.sms);
+  const Gemm16Plan g = plan_gemm16(M, N, K, layout_a, d.sms, tc16_pair_max_clusters());
   const CUtensorMapDataType dt =
       ab_dtype == SMGEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const uint32_t fmt = ab_dtype == SMGEMM_BF16 ? 1u : 0u;
@@ -331,20 +345,27 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_d
   } else {
     const bool a_mn = (layout_a == SMGEMM_COL_MAJOR);
     const bool b_mn = (layout_b == SMGEMM_ROW_MAJOR);
+    // Each CTA loads 128 rows of A; B tiles are 256 columns (one-SM kernel) or 128 (each
+    // CTA of a pair).
+    const uint32_t b_rows = g.pair ? 128 : 256;
     if (a_mn) ok = encode_2d(&tm_a, dt, A, M, K, lda * 2, 64, g.bk);
     else ok = encode_2d(&tm_a, dt, A, K, M, lda * 2, 64, 128);
     if (b_mn) ok = ok && encode_2d(&tm_b, dt, B, N, K, ldb * 2, 64, g.bk);
-    else ok = ok && encode_2d(&tm_b, dt, B, K, N, ldb * 2, 64, 256);
+    else ok = ok && encode_2d(&tm_b, dt, B, K, N, ldb * 2, 64, b_rows);
     p.a_mn_major = a_mn ? 1 : 0;
     p.b_mn_major = b_mn ? 1 : 0;
-    p.idesc = idesc_f32acc(fmt, fmt, a_mn ? 1u : 0u, b_mn ? 1u : 0u, 128, 256);
+    p.idesc = idesc_f32acc(fmt, fmt, a_mn ? 1u : 0u, b_mn ? 1u : 0u, g.pair ? 256 : 128, 256);
   }
   if (!ok) return SMGEMM_ERR_CUDA;
   p.s = g.pl.s;
   p.e = EpiArgs{static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C, c_dtype, ldc};
-  p.wait_limit_ns = wait_limit();
+  p.wait_limit_cycles = wait_limit();
   st = prepare_workspace(g.pl, workspace, workspace_bytes, stream, &p.slots, &p.counters);
   if (st != SMGEMM_OK) return st;
+  if (g.pair) {
+    note_config("pair", g.pl, 256);
+    return launch_status(launch_gemm_tc16_pair(tm_a, tm_b, p, g.pl.grid, stream));
+  }
   note_config(g.skinny ? "skinny" : "large", g.pl, g.mma_n);
   return launch_status(launch_gemm_tc16(tm_a, tm_b, p, g.v, g.pl.grid, stream));
 }
@@ -384,7 +405,7 @@ smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_
   p.sa = sa;
   p.sb = sb;
   p.nb_count = static_cast<int>((N + 127) / 128);
-  p.wait_limit_ns = wait_limit();
+  p.wait_limit_cycles = wait_limit();
   st = prepare_workspace(pl, workspace, workspace_bytes, stream, &p.slots, &p.counters);
   if (st != SMGEMM_OK) return st;
   note_config("fp8", pl, 128);
@@ -417,7 +438,7 @@ smgemm_status smgemm_check(smgemm_stream_t stream_) {
     cudaGetLastError();
     return SMGEMM_ERR_CUDA;
   }
-  const unsigned e = take_error_word_tc16() | take_error_word_fp8() | take_error_word_misc();
+  const unsigned e = take_error_word_tc16() | take_error_word_fp8() | take_error_word_misc() | take_error_word_pair();
   return (e & kErrTimeout) ? SMGEMM_ERR_TIMEOUT : SMGEMM_OK;
 }
 
@@ -432,7 +453,7 @@ smgemm_status smgemm_selftest_wait_timeout(uint32_t limit_us, smgemm_stream_t st
 int64_t smgemm_schedule_dump(int64_t M, int64_t N, int64_t K, int kind, smgemm_layout layout_a, int num_sms,
                              int32_t* out, int64_t cap) {
   if (M <= 0 || N <= 0 || K <= 0 || num_sms <= 0) return 0;
-  const Plan pl = kind == 1 ? plan_fp8(M, N, K, num_sms) : plan_gemm16(M, N, K, layout_a, num_sms).pl;
+  const Plan pl = kind == 1 ? plan_fp8(M, N, K, num_sms) : plan_gemm16(M, N, K, layout_a, num_sms, num_sms / 2).pl;
   int64_t n = 0;
   for (int c = 0; c < pl.grid; ++c) {
     WorkIter it;

@@ -42,38 +42,67 @@ __device__ __forceinline__ void store_one(void* C, int dtype, long long off, flo
   else static_cast<__half*>(C)[off] = __float2half_rn(x);
 }
 
-// 32 consecutive columns col0.. of one output row. The caller guarantees that C and
-// ldc*elem_size are 16-byte aligned (checked by the host), so whole chunks use 16-byte
-// vector stores.
-__device__ __forceinline__ void epi_row32(const EpiArgs& e, int row, int col0, float (&v)[32]) {
-  const bool full = col0 + 32 <= e.N;
+// In-place bias add and activation over 32 values. Every branch is taken once per
+// chunk, outside the per-element loops, so the common plain path jumps over these
+// blocks in one step and stays a short, straight run of instructions (the epilogue
+// warps share instruction caches with the producer and MMA-issuer warps).
+__device__ __forceinline__ void epi_bias_act32(const EpiArgs& e, int col0, float (&v)[32]) {
+  if (e.bias != nullptr) {
+    if (col0 + 32 <= e.N) {
+      if (e.bias_dtype == 0) {
+        const float* b = static_cast<const float*>(e.bias) + col0;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    float x = v[j];
-    if (e.bias != nullptr && (full || col0 + j < e.N)) x += load_bias(e.bias, e.bias_dtype, col0 + j);
-    v[j] = act_apply(x, e.act);
+        for (int j = 0; j < 32; ++j) v[j] += b[j];
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += load_bias(e.bias, e.bias_dtype, col0 + j);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < e.N) v[j] += load_bias(e.bias, e.bias_dtype, col0 + j);
+    }
   }
+  if (e.act == 1) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], 1);
+  } else if (e.act == 2) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], 2);
+  }
+}
+
+// Stores 32 finished values of one output row (vector stores when the chunk is whole;
+// the host guarantees 16-byte aligned C and ldc*elem_size).
+__device__ __forceinline__ void epi_store_row32(const EpiArgs& e, int row, int col0, const float (&v)[32]) {
   if (row >= e.M) return;
   const long long base = static_cast<long long>(row) * e.ldc + col0;
-  if (full) {
-    if (e.c_dtype == 0) {
-      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(e.C) + base);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-    } else {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(e.C) + base);
+  if (col0 + 32 <= e.N) {
+    if (e.c_dtype == 1) {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(e.C) + base);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t w[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          if (e.c_dtype == 1) {
-            __nv_bfloat162 t = __floats2bfloat162_rn(v[8 * j + 2 * h], v[8 * j + 2 * h + 1]);
-            w[h] = *reinterpret_cast<uint32_t*>(&t);
-          } else {
-            __half2 t = __floats2half2_rn(v[8 * j + 2 * h], v[8 * j + 2 * h + 1]);
-            w[h] = *reinterpret_cast<uint32_t*>(&t);
-          }
+          __nv_bfloat162 t = __floats2bfloat162_rn(v[8 * j + 2 * h], v[8 * j + 2 * h + 1]);
+          w[h] = *reinterpret_cast<uint32_t*>(&t);
+        }
+        dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    } else if (e.c_dtype == 0) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(e.C) + base);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(e.C) + base);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          __half2 t = __floats2half2_rn(v[8 * j + 2 * h], v[8 * j + 2 * h + 1]);
+          w[h] = *reinterpret_cast<uint32_t*>(&t);
         }
         dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
       }
@@ -83,6 +112,12 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int row, int col0, f
     for (int j = 0; j < 32; ++j)
       if (col0 + j < e.N) store_one(e.C, e.c_dtype, base + j, v[j]);
   }
+}
+
+// 32 consecutive columns col0.. of one output row: bias, activation, cast, store.
+__device__ __forceinline__ void epi_row32(const EpiArgs& e, int row, int col0, float (&v)[32]) {
+  if (e.bias != nullptr || e.act != 0) epi_bias_act32(e, col0, v);
+  epi_store_row32(e, row, col0, v);
 }
 
 // CNT consecutive output rows row0.. of one column (transposed accumulator tiles).

@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const TileSched& s = p.s;
-  const uint64_t limit = p.wait_limit_ns;
+  const uint64_t limit = p.wait_limit_cycles;
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -212,8 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Stream-K partial: store, then the last contributor reduces in CTA order.
         float* my_slot = p.slots + (static_cast<size_t>(blockIdx.x) * 2 + seg.slot) * (BM * BN);
         if (!dead) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) my_slot[(c_local0 + j) * BM + r_local] = acc[j];
+          slot_store<64>(my_slot, r_local, c_local0, acc);
         }
         const long long t_sk = seg.tile - s.dp_tiles;
         __threadfence();
@@ -241,8 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int cc = c_lo; cc <= c_hi; ++cc) {
               if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
               const float* src = p.slots + (static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * (BM * BN);
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] += __ldcg(src + (c_local0 + h * 32 + j) * BM + r_local);
+              slot_accumulate<32>(src, r_local, c_local0 + h * 32, v);
             }
             epi_row32(p.e, row, col0 + h * 32, v);
           }

@@ -20,6 +20,7 @@
 
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "operands.cuh"
 #include "sm100.cuh"
 
 namespace smg {
@@ -28,33 +29,6 @@ namespace {
 
 constexpr int kEpiWarp0 = 4;
 constexpr int kThreads = 256;
-
-template <int R, int BK>
-__device__ __forceinline__ void load_operand(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                             int mn_major, int r0, int k0) {
-  if (!mn_major) {
-    // K-major: boxes of {64 (K), R (rows)}, BK/64 of them along K, R*128 bytes apart.
-#pragma unroll
-    for (int j = 0; j < BK / 64; ++j) tma_load_2d(dst + j * R * 128, map, bar, k0 + 64 * j, r0);
-  } else {
-    // MN-major: boxes of {64 (rows), BK (K)}, R/64 of them along the rows, BK*128 bytes apart.
-#pragma unroll
-    for (int j = 0; j < R / 64; ++j) tma_load_2d(dst + j * BK * 128, map, bar, r0 + 64 * j, k0);
-  }
-}
-
-// Descriptor of the i-th 16-element K slice of an operand tile laid out by load_operand.
-template <int R, int BK>
-__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int mn_major, int i) {
-  if (!mn_major) return sdesc_sw128(base + (i >> 2) * (R * 128) + (i & 3) * 32, 16, 1024);
-  return sdesc_sw128(base + i * 2048, BK * 128, 1024);
-}
-
-template <int MMA_N>
-struct TmemCols {
-  static constexpr int v = (2 * MMA_N <= 32) ? 32 : (2 * MMA_N <= 64) ? 64 : (2 * MMA_N <= 128) ? 128
-                          : (2 * MMA_N <= 256) ? 256 : 512;
-};
 
 }  // namespace
 
@@ -111,7 +85,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const TileSched& s = p.s;
-  const uint64_t limit = p.wait_limit_ns;
+  const uint64_t limit = p.wait_limit_cycles;
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -227,8 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (SWAP) epi_col<CH>(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
             else epi_row32(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
           } else {
-#pragma unroll
-            for (int j = 0; j < CH; ++j) my_slot[(c * CH + j) * 128 + r_local] = v[j];
+            slot_store<CH>(my_slot, r_local, c * CH, v);
           }
         }
         tc_fence_before();
@@ -265,8 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int cc = c_lo; cc <= c_hi; ++cc) {
               if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
               const float* src = p.slots + (static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * (128 * MMA_N);
-#pragma unroll
-              for (int j = 0; j < CH; ++j) v[j] += __ldcg(src + (c * CH + j) * 128 + r_local);
+              slot_accumulate<CH>(src, r_local, c * CH, v);
             }
             if constexpr (SWAP) epi_col<CH>(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
             else epi_row32(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);

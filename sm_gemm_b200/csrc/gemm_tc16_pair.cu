@@ -1,0 +1,313 @@
+// Large-tile 16-bit GEMM on CTA pairs (tcgen05.mma.cta_group::2): one 256 x 256 output
+// tile per pair of SMs, FP32 accumulators in both SMs' TMEM, fused epilogue.
+//
+// Against the one-SM 128 x 256 kernel (gemm_tc16.cu) each SM now stages only its own
+// 128 rows of A and its own 128 columns of B per K-block (32 KB instead of 48 KB for the
+// same 128 x 256 share of the output), which halves the B traffic from L2 per FLOP and
+// leaves room for 6 pipeline stages. The pipeline is still the copy-ahead-of-the-math
+// scheme of the DeepGEMM kernel-library walkthrough (zwxr.cn), section 2.3; the fused
+// epilogue is its section 5.1.
+//
+// Roles (256 threads per CTA, both CTAs of the cluster):
+//  warp 0   TMA producer: loads this CTA's A rows and B columns; the byte count of
+//           both CTAs' copies completes on the rank-0 CTA's "full" barrier.
+//  warp 1   MMA issuer (rank 0 only): 4 x K=16 MMAs of 256 x 256 per stage; commits
+//           free the stage in both CTAs and signal both CTAs' accumulators.
+//  warp 2   TMEM allocator (cta_group::2, 512 columns = two 256-column accumulators).
+//  warps 4-7 epilogue: each CTA drains its own 128 rows; they release the accumulator
+//           to the rank-0 MMA issuer with a cluster-scope arrive.
+// Stream-K partial tiles are kept per (cluster, slot, rank) and reduced per rank.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "operands.cuh"
+#include "sm100.cuh"
+
+namespace smg {
+
+namespace {
+constexpr int kThreads = 256;
+constexpr int kEpiWarp0 = 4;
+constexpr int kTileN = 256;  // columns of the pair tile (128 per CTA for B, all 256 in each TMEM)
+constexpr int kTcols = 512;
+}  // namespace
+
+template <int BK, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc16_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                          const Tc16Params p) {
+  constexpr int A_BYTES = 128 * BK * 2;
+  constexpr int B_BYTES = 128 * BK * 2;
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr int KSTEPS = BK / 16;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
+  const uint32_t bar_base = smem_base + STAGES * STAGE_BYTES;
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
+  uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  volatile int* reduce_flag = reinterpret_cast<volatile int*>(misc + 8);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();
+  const int cluster = blockIdx.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 8);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTcols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive or copy targets them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const TileSched& s = p.s;
+  const uint64_t limit = p.wait_limit_cycles;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    long long issued = 0;
+    WorkIter it;
+    it.init(s, cluster);
+    Seg seg;
+    bool ok = true;
+    while (ok && it.next(s, seg)) {
+      int mt, nt;
+      tile_coords(s, seg.tile, mt, nt);
+      const int a_row = mt * 256 + static_cast<int>(rank) * 128;
+      const int b_row = nt * kTileN + static_cast<int>(rank) * 128;
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit)) { ok = false; break; }
+        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
+        if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+        load_operand_pair<128, BK>(sa, &tm_a, leader_full, p.a_mn_major, a_row, kb * BK);
+        load_operand_pair<128, BK>(sa + A_BYTES, &tm_b, leader_full, p.b_mn_major, b_row, kb * BK);
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok && rank == 0) {
+      // Wait (bounded, independent of the abort flag) for copies still in flight.
+      int st = stage;
+      uint32_t ph = phase;
+      volatile int no_abort = 0;
+      for (long long i = 0; i < issued && i < STAGES; ++i) {
+        if (--st < 0) { st = STAGES - 1; ph ^= 1u; }
+        mbar_wait(full_bar(st), ph, &no_abort, limit);
+      }
+    }
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int local = 0;
+    WorkIter it;
+    it.init(s, cluster);
+    Seg seg;
+    bool ok = true;
+    while (ok && it.next(s, seg)) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, limit)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * kTileN;
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb) {
+        if (!mbar_wait(full_bar(stage), phase, abort_flag, limit)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+        for (int k = 0; k < KSTEPS; ++k) {
+          umma_f16_pair(d_tmem, operand_desc<128, BK>(sa, p.a_mn_major, k),
+                        operand_desc<128, BK>(sb, p.b_mn_major, k), p.idesc, (kb > seg.kb0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit_pair(empty_bar(stage), 0x3);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      umma_commit_pair(tfull_bar(acc), 0x3);
+      ++local;
+    }
+    umma_commit_pair(drain_bar, 0x1);
+    volatile int no_abort = 0;
+    mbar_wait(drain_bar, 0, &no_abort, limit);
+  } else if (warp >= kEpiWarp0) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int r_local = q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const int epi_tid = threadIdx.x - kEpiWarp0 * 32;
+    constexpr int SLOT = 128 * kTileN;
+    int local = 0;
+    WorkIter it;
+    it.init(s, cluster);
+    Seg seg;
+    bool dead = false;
+    while (it.next(s, seg)) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!dead) dead = !mbar_wait(tfull_bar(acc), acc_phase, abort_flag, limit);
+      dead = __any_sync(0xffffffffu, dead);
+      int mt, nt;
+      tile_coords(s, seg.tile, mt, nt);
+      const int row = mt * 256 + static_cast<int>(rank) * 128 + r_local;
+      const uint32_t tacc = tmem_base + lane_addr + acc * kTileN;
+      const bool whole = (seg.kb0 == 0 && seg.kb1 == s.kb_total);
+      float* my_slot = p.slots + ((static_cast<size_t>(cluster) * 2 + seg.slot) * 2 + rank) * SLOT;
+      if (!dead) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < kTileN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tacc + c * 32, r);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          if (whole) {
+            epi_row32(p.e, row, nt * kTileN + c * 32, v);
+          } else {
+            slot_store<32>(my_slot, r_local, c * 32, v);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+      }
+
+      if (!whole) {
+        const long long t_sk = seg.tile - s.dp_tiles;
+        __threadfence();
+        named_barrier_sync(1, 128);
+        if (epi_tid == 0) {
+          const int c_lo = sk_owner(s, t_sk * s.kb_total);
+          const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
+          int n = 0;
+          for (int c = c_lo; c <= c_hi; ++c) n += sk_bound(s, c) < sk_bound(s, c + 1);
+          const bool any_dead = *abort_flag != 0;
+          const int old = any_dead ? -1 : atomicAdd(p.counters + t_sk * 2 + rank, 1);
+          *reduce_flag = (!any_dead && old == n - 1);
+        }
+        named_barrier_sync(1, 128);
+        if (*reduce_flag) {
+          __threadfence();
+          const int c_lo = sk_owner(s, t_sk * s.kb_total);
+          const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
+#pragma unroll 1
+          for (int c = 0; c < kTileN / 32; ++c) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+#pragma unroll 1
+            for (int cc = c_lo; cc <= c_hi; ++cc) {
+              if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
+              const float* src = p.slots + ((static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * 2 + rank) * SLOT;
+              slot_accumulate<32>(src, r_local, c * 32, v);
+            }
+            epi_row32(p.e, row, nt * kTileN + c * 32, v);
+          }
+        }
+        named_barrier_sync(1, 128);
+      }
+      ++local;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer stays resident until the rank-0 MMA issuer has drained
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc_pair(tmem_base, kTcols);
+}
+
+namespace {
+constexpr int kPairBK = 64, kPairStages = 6;
+constexpr int kPairSmem = 1024 + kPairStages * (2 * 128 * kPairBK * 2) + 8 * (2 * kPairStages + 5) + 16;
+static_assert(kPairSmem <= 232448, "shared memory budget");
+
+cudaError_t prepare_pair_kernel() {
+  static cudaError_t st = cudaFuncSetAttribute(gemm_tc16_pair_kernel<kPairBK, kPairStages>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+  return st;
+}
+}  // namespace
+
+int tc16_pair_max_clusters() {
+  static int cached = -1;
+  if (cached >= 0) return cached;
+  if (prepare_pair_kernel() != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPairSmem;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc16_pair_kernel<kPairBK, kPairStages>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cached = n;
+  return n;
+}
+
+cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Tc16Params& p,
+                                  int clusters, cudaStream_t stream) {
+  cudaError_t e = prepare_pair_kernel();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPairSmem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages>, tm_a, tm_b, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+int tc16_pair_bk() { return kPairBK; }
+
+unsigned take_error_word_pair() { return take_error_word(); }
+
+}  // namespace smg

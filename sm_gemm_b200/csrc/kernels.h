@@ -14,8 +14,11 @@ namespace smg {
 constexpr int kF32 = 0, kBF16 = 1, kF16 = 2, kE4M3 = 3;
 constexpr int kActNone = 0, kActGeluTanh = 1, kActSilu = 2;
 
-// Default limit of every bounded barrier wait inside the kernels.
+// Default limit of every bounded barrier wait inside the kernels, and the SM clock
+// used to turn it into cycles (an upper bound of the B200 SM clock, so the real limit
+// is at least the stated time).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr unsigned long long kCyclesPerNs = 2;
 
 struct Tc16Params {
   TileSched s;
@@ -25,7 +28,7 @@ struct Tc16Params {
   int b_mn_major;           // MMA "B" operand tile is MN-major (else K-major)
   float* slots;             // stream-K partial tiles: [num_ctas][2][MMA_N][128] floats
   int* counters;            // stream-K arrival counters, one per stream-K tile, zeroed per call
-  unsigned long long wait_limit_ns;
+  unsigned long long wait_limit_cycles;
 };
 
 enum class Tc16Variant { kLarge, kSkinny16, kSkinny32, kSkinny64 };
@@ -34,6 +37,13 @@ cudaError_t launch_gemm_tc16(const CUtensorMap& tm_a, const CUtensorMap& tm_b, c
                              Tc16Variant v, int grid, cudaStream_t stream);
 int tc16_mma_n(Tc16Variant v);
 int tc16_bk(Tc16Variant v);
+
+// CTA-pair large-tile kernel (256 x 256 per cluster of 2). p.s counts clusters;
+// p.slots is [clusters][2][2 ranks][256][128] floats, p.counters [stream-K tiles][2].
+cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Tc16Params& p,
+                                  int clusters, cudaStream_t stream);
+int tc16_pair_max_clusters();   // co-resident clusters of 2 on the current device (0 if unknown)
+int tc16_pair_bk();
 
 struct Fp8Params {
   TileSched s;
@@ -45,7 +55,7 @@ struct Fp8Params {
   int nb_count;             // NB = ceil(N/128)
   float* slots;             // [num_ctas][2][128][128] floats
   int* counters;
-  unsigned long long wait_limit_ns;
+  unsigned long long wait_limit_cycles;
 };
 
 cudaError_t launch_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Fp8Params& p,
@@ -67,5 +77,6 @@ cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t strea
 unsigned take_error_word_tc16();
 unsigned take_error_word_fp8();
 unsigned take_error_word_misc();
+unsigned take_error_word_pair();
 
 }  // namespace smg

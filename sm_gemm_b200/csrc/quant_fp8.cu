@@ -170,8 +170,8 @@ __global__ void fill_epilogue_kernel(int M, int N, const void* bias, int bias_dt
 }
 
 // Waits on an mbarrier that nothing arrives on; the bounded wait gives up after
-// `limit_ns`, records kErrTimeout and the kernel returns normally.
-__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+// `limit_cycles` SM cycles, records kErrTimeout and the kernel returns normally.
+__global__ void wait_selftest_kernel(unsigned long long limit_cycles) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -180,7 +180,7 @@ __global__ void wait_selftest_kernel(unsigned long long limit_ns) {
     fence_barrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_cycles);
   __syncthreads();
 }
 
@@ -220,7 +220,7 @@ cudaError_t launch_fill_epilogue(int M, int N, const void* bias, int bias_dtype,
 }
 
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t stream) {
-  wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns * kCyclesPerNs);
   return cudaGetLastError();
 }
 

@@ -42,12 +42,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t global_timer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 
@@ -86,26 +80,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait until the phase with the given parity of barrier `bar` has completed, for at
-// most `limit_ns` nanoseconds. On expiry: record kErrTimeout in the device error word,
-// raise the CTA-wide abort flag and return false. Every later wait of the CTA returns
-// false at once when the abort flag is up, so a stalled pipeline drains in about one
-// limit instead of one per wait.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+// Slow path of mbar_wait: spin on try_wait, checking the CTA abort flag and the SM cycle
+// counter (clock64, cheap) every 64 polls; give up after `limit_cycles` cycles.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            uint64_t limit_cycles) {
+  const long long t0 = clock64();
   while (true) {
-    if (*abort_flag) return false;
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
+    for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > limit_ns) {
+    if (*abort_flag) return false;
+    if (static_cast<uint64_t>(clock64() - t0) > limit_cycles) {
       *abort_flag = 1;
       atomicOr(&g_error_word, kErrTimeout);
       return false;
     }
   }
+}
+
+// Wait until the phase with the given parity of barrier `bar` has completed, for at
+// most `limit_cycles` SM cycles. On expiry: record kErrTimeout in the device error
+// word, raise the CTA-wide abort flag and return false. Every later wait of the CTA
+// returns false soon after when the abort flag is up, so a stalled pipeline drains in
+// about one limit instead of one per wait. The common case (phase already complete,
+// or completing during the first poll) stays inline and never reads a timer.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_cycles) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, limit_cycles);
 }
 
 // ------------------------------------------------------------------ TMA
@@ -202,6 +204,76 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ CTA pairs (cta_group::2)
+//
+// Two CTAs of a cluster (ranks 0 and 1, on the two SMs of one TPC) share one MMA: the
+// rank-0 CTA issues tcgen05.mma.cta_group::2 over both CTAs' shared-memory operand
+// tiles and the result lands in both CTAs' TMEM (rows 0..127 in rank 0, 128..255 in
+// rank 1). No load here uses TMA multicast: each CTA loads only its own tiles.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on an mbarrier of any CTA of the cluster (address from mapa_shared).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA tile load into this CTA's shared memory whose byte count completes on an
+// mbarrier of either CTA of the pair (here: always the rank-0 CTA's).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t c0, int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// Arrive once on the barrier at offset `bar` in every CTA of `cta_mask` when all
+// tcgen05.mma issued so far by this thread (over the pair) have completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          bar),
+      "h"(cta_mask)
+      : "memory");
+}
+
 // ------------------------------------------------------------------ UMMA descriptors
 
 // Shared-memory matrix descriptor (sm_100 format): start address, leading and stride
@@ -236,6 +308,8 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t a_fmt, uint32_t b_f
 // sk_iters = (tiles - dp_tiles) * kb_total K-block iterations cut into num_ctas
 // contiguous ranges (stream-K). A tile whose K range is cut is summed in fixed CTA
 // order by whichever contributor finishes last, so results are deterministic.
+// Partial tiles are stored as float4 units [col/4][row] (the TMEM lane is the row), so
+// the 32 lanes of a warp write and read 512 contiguous bytes per instruction.
 struct TileSched {
   int m_tiles, n_tiles, kb_total;
   int dp_tiles;
@@ -286,15 +360,10 @@ struct WorkIter {
     sk_begin = sk_pos = sk_bound(s, cta);
     sk_end = sk_bound(s, cta + 1);
   }
+  // Stream-K range first, then the data-parallel tiles: the fix-up of a split tile
+  // (done by its last contributor's epilogue warps) then overlaps the MMAs of that
+  // CTA's remaining tiles instead of landing in the kernel's tail.
   __host__ __device__ bool next(const TileSched& s, Seg& out) {
-    if (dp_next < s.dp_tiles) {
-      out.tile = dp_next;
-      out.kb0 = 0;
-      out.kb1 = s.kb_total;
-      out.slot = 0;
-      dp_next += s.num_ctas;
-      return true;
-    }
     if (sk_pos < sk_end) {
       const long long t = sk_pos / s.kb_total;
       const int kb0 = static_cast<int>(sk_pos - t * s.kb_total);
@@ -308,9 +377,41 @@ struct WorkIter {
       sk_pos += kb1 - kb0;
       return true;
     }
+    if (dp_next < s.dp_tiles) {
+      out.tile = dp_next;
+      out.kb0 = 0;
+      out.kb1 = s.kb_total;
+      out.slot = 0;
+      dp_next += s.num_ctas;
+      return true;
+    }
     return false;
   }
 };
+
+// Partial-tile slot access for the TMEM lane `r` (tile row) and N consecutive columns
+// starting at col0 (N and col0 multiples of 4): float4 units at [col/4][r], so a
+// warp's 32 lanes touch 512 contiguous bytes per instruction.
+template <int N>
+__device__ __forceinline__ void slot_store(float* slot, int r, int col0, const float* v) {
+  float4* s4 = reinterpret_cast<float4*>(slot);
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q)
+    s4[((col0 >> 2) + q) * 128 + r] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+template <int N>
+__device__ __forceinline__ void slot_accumulate(const float* slot, int r, int col0, float* v) {
+  const float4* s4 = reinterpret_cast<const float4*>(slot);
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) {
+    const float4 t = __ldcg(s4 + ((col0 >> 2) + q) * 128 + r);
+    v[4 * q] += t.x;
+    v[4 * q + 1] += t.y;
+    v[4 * q + 2] += t.z;
+    v[4 * q + 3] += t.w;
+  }
+}
 
 // The slot a contributor CTA `c` used for stream-K tile `t_sk` (index among the
 // stream-K tiles): 0 if the tile holds the start of c's range, else 1.

@@ -153,12 +153,14 @@ def _check_schedule(M, N, K, kind=0, layout_a=sg.ROW_MAJOR, sms=148, bk=None):
     assert len({(m, n) for _, m, n in coords}) == len(tiles)
     # a split tile's contributors are consecutive CTAs in K order, and each partial
     # segment's slot is 0 iff it is the first segment of that CTA
-    first_seg = {}
+    first_seg, seen_dp = {}, set()
     for i, (c, t, mt, nt, k0, k1, slot) in enumerate(d):
         if slot >= 0:
+            assert int(c) not in seen_dp                   # a CTA's stream-K range comes first
             first_seg.setdefault(int(c), i)
         else:
-            assert k0 == 0 and k1 == kb_total and int(c) not in first_seg   # DP tiles come first
+            assert k0 == 0 and k1 == kb_total
+            seen_dp.add(int(c))
     by_tile = {}
     for i, (c, t, mt, nt, k0, k1, slot) in enumerate(d):
         by_tile.setdefault(int(t), []).append((int(k0), int(c), int(slot), i))

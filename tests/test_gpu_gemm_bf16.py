@@ -104,9 +104,13 @@ def test_tiny_fp16_64cube_fp32_out(cuda_device):
 @pytest.mark.parametrize("la", ["row", "col"])
 @pytest.mark.parametrize("lb", ["row", "col"])
 @pytest.mark.parametrize("sched", ["auto", "dp", "sk"])
-def test_integer_inputs_bit_exact_all_layouts(cuda_device, monkeypatch, la, lb, sched):
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_integer_inputs_bit_exact_all_layouts(cuda_device, monkeypatch, la, lb, sched, pair):
+    """pair=1: 256x256 tiles on CTA pairs (cta_group::2); pair=0: 128x256 one-SM tiles."""
     monkeypatch.setenv("SMGEMM_SCHED", sched)
+    monkeypatch.setenv("SMGEMM_PAIR", pair)
     got, ref, _ = run_case(300, 600, 520, la=la, lb=lb, out_dt=torch.float32, integer=True, seed=3)
+    assert ("path=pair" in sg.last_config()) == (pair == "1")
     assert np.array_equal(got, ref)
 
 
@@ -145,7 +149,9 @@ def test_identity_and_permutation(cuda_device):
 @pytest.mark.parametrize("M,N,K", [(32, 32, 32), (64, 64, 64), (67, 50, 33), (300, 700, 1000),
                                    (129, 257, 4096)])
 @pytest.mark.parametrize("la,lb", [("row", "col"), ("row", "row"), ("col", "col")])
-def test_random_within_tolerance(cuda_device, M, N, K, la, lb):
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_random_within_tolerance(cuda_device, monkeypatch, M, N, K, la, lb, pair):
+    monkeypatch.setenv("SMGEMM_PAIR", pair)
     got, ref, acc = run_case(M, N, K, la=la, lb=lb, seed=M + N + K)
     check_tolerance(got, ref, acc, torch.bfloat16, what=f"{M}x{N}x{K} {la}/{lb}")
 
@@ -229,9 +235,22 @@ def test_stream_k_split_across_many_ctas(cuda_device, monkeypatch):
     check_tolerance(got, ref, acc, torch.float32, what="stream-K")
 
 
-def test_persistent_multi_tile_per_cta(cuda_device, monkeypatch):
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_persistent_multi_tile_per_cta(cuda_device, monkeypatch, pair):
     monkeypatch.setenv("SMGEMM_GRID", "3")
+    monkeypatch.setenv("SMGEMM_PAIR", pair)
     got, ref, _ = run_case(700, 1100, 300, integer=True, out_dt=torch.float32, seed=51)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_stream_k_hybrid_many_tiles(cuda_device, monkeypatch, pair):
+    """More tiles than CTAs, not a multiple: data-parallel waves + a stream-K tail."""
+    monkeypatch.setenv("SMGEMM_PAIR", pair)
+    monkeypatch.setenv("SMGEMM_GRID", "5")
+    got, ref, _ = run_case(1500, 1300, 1024, integer=True, out_dt=torch.float32, seed=52)
+    cfg = sg.last_config()
+    assert "sk_iters=0" not in cfg and "dp_tiles=0" not in cfg, cfg
     assert np.array_equal(got, ref)
 
 
