@@ -96,10 +96,17 @@ SchedMode sched_mode() {
   return SchedMode::kAuto;
 }
 
-// Tile-grid plan. Large tile counts run data-parallel waves with the ragged last
-// wave(s) handed to stream-K; small tile counts with a long K are split by stream-K
-// so every SM streams an equal share of the K-blocks (the page's concern that small
-// shapes leave SMs idle: "为什么我们要死磕GEMM", kwkr.cn, section 3.3).
+// Tile-grid plan over T output tiles and P persistent CTAs (or CTA pairs).
+//  - auto: whole waves of tiles run data-parallel; the R = T mod P tiles of a ragged
+//    last wave are split along K into s = min(P / R, KB / 8) equal pieces that run
+//    side by side (one piece per CTA), so the last wave takes 1/s of a tile instead of
+//    a whole one. Pieces of tiles that share operands start at the same K offsets, so
+//    L2 reuse is kept (a free-running stream-K range would scatter the CTAs that share
+//    a B column block across K and re-stream it from HBM). The pages' concern this
+//    addresses: small or ragged shapes leave SMs idle ("为什么我们要死磕GEMM",
+//    kwkr.cn, section 3.3).
+//  - SMGEMM_SCHED=dp: data-parallel only; SMGEMM_SCHED=sk: every tile in one stream-K
+//    range over all CTAs (kept for tests).
 struct Plan {
   TileSched s;
   int grid = 0;
@@ -116,27 +123,21 @@ Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, siz
   if (max_ctas < 1) max_ctas = 1;
   if (max_ctas > sms) max_ctas = sms;
   const SchedMode mode = sched_mode();
-  constexpr int kMinItersPerCta = 8;
+  constexpr int kMinItersPerPiece = 8;
 
-  long long dp = T, sk_iters = 0, grid = std::min<long long>(T, max_ctas);
+  long long dp = T, sk_iters = 0, sk_ctas = 0, grid = std::min<long long>(T, max_ctas);
   if (mode == SchedMode::kSK) {
     dp = 0;
     sk_iters = T * kb_total;
-    grid = std::min<long long>(max_ctas, sk_iters);
+    grid = sk_ctas = std::min<long long>(max_ctas, sk_iters);
   } else if (mode == SchedMode::kAuto) {
-    if (T >= max_ctas) {
-      if (T % max_ctas != 0 && kb_total >= kMinItersPerCta) {
-        dp = (T / max_ctas - 1) * max_ctas;
-        sk_iters = (T - dp) * kb_total;
-        grid = max_ctas;
-      }
-    } else {
-      const long long want = std::min<long long>(max_ctas, T * kb_total / kMinItersPerCta);
-      if (want > T) {
-        dp = 0;
-        sk_iters = T * kb_total;
-        grid = want;
-      }
+    const long long waves = T / max_ctas, R = T % max_ctas;
+    long long split = R > 0 ? std::min<long long>(max_ctas / R, kb_total / kMinItersPerPiece) : 1;
+    if (split >= 2) {
+      dp = waves * max_ctas;
+      sk_iters = R * kb_total;
+      sk_ctas = R * split;
+      grid = waves > 0 ? max_ctas : sk_ctas;
     }
   }
   pl.s.m_tiles = m_tiles;
@@ -146,10 +147,11 @@ Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, siz
   pl.s.num_ctas = static_cast<int>(grid);
   pl.s.group_m = std::max(1, std::min(group_m, m_tiles));
   pl.s.sk_iters = sk_iters;
+  pl.s.sk_ctas = static_cast<int>(sk_iters > 0 ? sk_ctas : grid);
   pl.grid = static_cast<int>(grid);
   if (sk_iters > 0) {
     pl.counter_bytes = ((static_cast<size_t>(T - dp) * counters_per_tile * sizeof(int)) + 255) / 256 * 256;
-    pl.slot_bytes = static_cast<size_t>(grid) * 2 * slot_floats * sizeof(float);
+    pl.slot_bytes = static_cast<size_t>(sk_ctas) * 2 * slot_floats * sizeof(float);
   }
   return pl;
 }
@@ -260,8 +262,9 @@ smgemm_status prepare_workspace(const Plan& pl, void* ws, size_t ws_bytes, cudaS
 
 void note_config(const char* path, const Plan& pl, int mma_n) {
   std::snprintf(g_last_config, sizeof(g_last_config),
-                "path=%s tile=128x%d tiles=%dx%d kb=%d grid=%d dp_tiles=%d sk_iters=%lld ws=%zu", path, mma_n,
-                pl.s.m_tiles, pl.s.n_tiles, pl.s.kb_total, pl.grid, pl.s.dp_tiles, pl.s.sk_iters, pl.ws_bytes());
+                "path=%s tile=128x%d tiles=%dx%d kb=%d grid=%d dp_tiles=%d sk_iters=%lld sk_ctas=%d ws=%zu", path,
+                mma_n, pl.s.m_tiles, pl.s.n_tiles, pl.s.kb_total, pl.grid, pl.s.dp_tiles, pl.s.sk_iters, pl.s.sk_ctas,
+                pl.ws_bytes());
   if (env_ll("SMGEMM_LOG", 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
 }
 

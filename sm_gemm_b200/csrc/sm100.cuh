@@ -316,6 +316,7 @@ struct TileSched {
   int num_ctas;
   int group_m;
   long long sk_iters;
+  int sk_ctas;  // CTAs 0 .. sk_ctas-1 share the stream-K range (<= num_ctas)
 };
 
 struct Seg {
@@ -325,14 +326,14 @@ struct Seg {
 };
 
 __host__ __device__ inline long long sk_bound(const TileSched& s, int c) {
-  return (s.sk_iters * c) / s.num_ctas;
+  return c >= s.sk_ctas ? s.sk_iters : (s.sk_iters * c) / s.sk_ctas;
 }
 
 // CTA owning stream-K iteration i.
 __host__ __device__ inline int sk_owner(const TileSched& s, long long i) {
-  int c = static_cast<int>((i * s.num_ctas) / (s.sk_iters > 0 ? s.sk_iters : 1));
-  if (c >= s.num_ctas) c = s.num_ctas - 1;
-  while (c + 1 < s.num_ctas && sk_bound(s, c + 1) <= i) ++c;
+  int c = static_cast<int>((i * s.sk_ctas) / (s.sk_iters > 0 ? s.sk_iters : 1));
+  if (c >= s.sk_ctas) c = s.sk_ctas - 1;
+  while (c + 1 < s.sk_ctas && sk_bound(s, c + 1) <= i) ++c;
   while (c > 0 && sk_bound(s, c) > i) --c;
   return c;
 }

@@ -171,13 +171,24 @@ def _check_schedule(M, N, K, kind=0, layout_a=sg.ROW_MAJOR, sms=148, bk=None):
             assert cs == sorted(cs) and len(set(cs)) == len(cs)
             for k0, c, slot, i in segs:
                 assert slot == (0 if first_seg[c] == i else 1)
-    # stream-K work is balanced: per-CTA K-block counts differ by at most one
+    # stream-K / split work is balanced: per-CTA K-block counts differ by at most one
     sk = d[d[:, 6] >= 0]
     if sk.size:
         per = np.bincount(sk[:, 0], weights=sk[:, 5] - sk[:, 4])
         per = per[per > 0]
         assert per.max() - per.min() <= 1
     return d
+
+
+def test_split_tail_plan_square():
+    """4096^3 on 74 CTA pairs: 3 whole waves of 256x256 tiles, the 34 tiles of the
+    ragged fourth wave split in two K halves over 68 pairs."""
+    d = sg.schedule_dump(4096, 4096, 4096, 0, sg.ROW_MAJOR, 148)
+    dp = d[d[:, 6] < 0]
+    sk = d[d[:, 6] >= 0]
+    assert len(dp) == 3 * 74 and len(sk) == 68
+    assert set((sk[:, 5] - sk[:, 4]).tolist()) == {32}
+    assert sorted(set(sk[:, 4].tolist())) == [0, 32]
 
 
 @pytest.mark.parametrize("M,N,K", [(4096, 4096, 4096), (1024, 16384, 4096), (1024, 4096, 16384),
@@ -189,9 +200,9 @@ def test_schedule_large_covers_each_kblock_once(M, N, K):
 @pytest.mark.parametrize("M", [1, 4, 16, 64])
 def test_schedule_skinny_lm_head(M):
     d = _check_schedule(M, 128256, 4096)
-    # all 148 SMs get work and the K-blocks are shared within 1 of each other
+    # all 148 SMs get work and no SM has more than one tile (32 K-blocks) above another
     per_cta = np.bincount(d[:, 0], weights=d[:, 5] - d[:, 4], minlength=148)
-    assert per_cta.min() > 0 and per_cta.max() - per_cta.min() <= 1
+    assert per_cta.min() > 0 and per_cta.max() - per_cta.min() <= 32
 
 
 @pytest.mark.parametrize("M,N,K", [(2048, 16384, 4096), (256, 384, 1024), (130, 260, 128)])
