@@ -1,19 +1,24 @@
-// Block-scaled FP8 (E4M3) GEMM with per-K-block scale promotion into FP32.
+// Block-scaled FP8 (E4M3) GEMM with per-K-block scale promotion into FP32, one SM per
+// 128 x 128 output tile.
 //
 // The DeepGEMM kernel-library walkthrough (zwxr.cn), section 2.4 quantises with one
 // FP32 scale per 1x128 group of the activations and per 128x128 block of the
 // weights, and accumulates the low-precision products in FP32 before rescaling. Here
-// each 128-wide K-block kb of a 128x128 output tile is multiplied on the tensor core
-// into an FP32 TMEM partial P_kb (kind::f8f6f4, four K=32 steps), and promotion warps
-// fold it into a register accumulator: acc += (sa[kb,m] * sb[kb,nb]) * P_kb. The
-// scales are arbitrary FP32 values (amax/448), not powers of two, so the hardware
-// block-scaled MMA (UE8M0 / UE4M3 scale factors) cannot apply them exactly; the
-// promotion is done in software. Two TMEM partial buffers let the MMA of kb+1 run
-// while kb is promoted.
+// each 128-wide K-block kb of a tile is multiplied on the tensor core into an FP32 TMEM
+// partial P_kb (kind::f8f6f4, four K=32 steps), and promotion warps fold it into a
+// register accumulator: acc += (sa[kb,m] * sb[kb,nb]) * P_kb. The scales are arbitrary
+// FP32 values (amax/448), not powers of two, so the hardware block-scaled MMA (UE8M0 /
+// UE4M3 scale factors) cannot apply them exactly; the promotion is done in software.
+// Two TMEM partial buffers let the MMA of kb+1 run while kb is promoted.
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM
-// allocator, warp 3 idle, warps 4..11 promotion + epilogue: warp w reads TMEM lanes
-// 32*(w%4).. (tile rows) and columns 64*((w-4)/4).. (64 of the 128 tile columns).
+// allocator, warp 3 scale loader, warps 4..11 promotion + epilogue: warp w reads TMEM
+// lanes 32*(w%4).. (tile rows) and columns 64*((w-4)/4).. (64 of the 128 columns).
+//
+// The scale loader stages each K-block's 128 row scales and its block scale in a
+// 4-slot shared-memory ring. Promotion warps then never have a global load in flight
+// when they release a TMEM buffer (an mbarrier arrive has release semantics and
+// would wait for such loads), and read their scales from shared memory.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -25,14 +30,18 @@ namespace smg {
 
 namespace {
 constexpr int kThreads = 384;
+constexpr int kLoaderWarp = 3;
 constexpr int kPromoWarp0 = 4;
-constexpr int kPromoThreads = 256;
+constexpr int kPromoWarps = 8;
+constexpr int kPromoThreads = kPromoWarps * 32;
 constexpr int BM = kFp8BM, BN = kFp8BN, BKB = kFp8BK;  // BK in bytes = elements
 constexpr int A_BYTES = BM * BKB;                       // 16 KB
 constexpr int B_BYTES = BN * BKB;                       // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int STAGES = 6;
-constexpr int TCOLS = 256;  // two 128-column FP32 partial buffers
+constexpr int TCOLS = 256;       // two 128-column FP32 partial buffers
+constexpr int kRing = 4;         // scale ring slots
+constexpr int kSlotFloats = 132; // 128 row scales + block scale, padded to 16 bytes
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int i) {
   // K-major tile of 128 rows x 128 bytes, 128-byte swizzle; K step i = 32 bytes.
@@ -46,13 +55,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
-  const uint32_t bar_base = smem_base + STAGES * STAGE_BYTES;
+  float* ring = reinterpret_cast<float*>(smem_gen + STAGES * STAGE_BYTES);
+  const uint32_t bar_base = smem_base + STAGES * STAGE_BYTES + kRing * kSlotFloats * 4;
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
   auto pfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
   auto pempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
-  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
-  uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5);
+  auto sfull_bar = [&](int r) { return bar_base + 8u * (2 * STAGES + 4 + r); };
+  auto sempty_bar = [&](int r) { return bar_base + 8u * (2 * STAGES + 4 + kRing + r); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4 + 2 * kRing);
+  uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + kRing * kSlotFloats * 4 + 8 * (2 * STAGES + 5 + 2 * kRing);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   volatile int* reduce_flag = reinterpret_cast<volatile int*>(misc + 8);
@@ -65,7 +77,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(pfull_bar(b), 1);
-      mbar_init(pempty_bar(b), 8);
+      mbar_init(pempty_bar(b), kPromoWarps);
+    }
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(sfull_bar(r), 32);
+      mbar_init(sempty_bar(r), kPromoWarps);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -85,6 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const TileSched& s = p.s;
   const uint64_t limit = p.wait_limit_cycles;
+  const int M = p.e.M;
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -121,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- MMA issuer
     int stage = 0;
     uint32_t phase = 0;
-    long long kcount = 0;  // K-blocks issued by this CTA: selects the partial buffer
+    uint32_t kcount = 0;  // K-blocks issued by this CTA: selects the partial buffer
     WorkIter it;
     it.init(s, blockIdx.x);
     Seg seg;
@@ -129,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (ok && it.next(s, seg)) {
       for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++kcount) {
         const int buf = static_cast<int>(kcount & 1);
-        const uint32_t bphase = static_cast<uint32_t>((kcount >> 1) & 1);
+        const uint32_t bphase = (kcount >> 1) & 1;
         if (!mbar_wait(pempty_bar(buf), bphase ^ 1u, abort_flag, limit)) { ok = false; break; }
         if (!mbar_wait(full_bar(stage), phase, abort_flag, limit)) { ok = false; break; }
         tc_fence_after();
@@ -146,6 +163,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     umma_commit(drain_bar);
     volatile int no_abort = 0;
     mbar_wait(drain_bar, 0, &no_abort, limit);
+  } else if (warp == kLoaderWarp) {
+    // ---------------------------------------------------------------- scale loader
+    // Slot layout: [0, 128) row scales sa[kb, m0 + r]; [128] block scale sb[kb, nt].
+    uint32_t kc = 0;
+    WorkIter it;
+    it.init(s, blockIdx.x);
+    Seg seg;
+    bool dead = false;
+    const bool vec = (M & 3) == 0;
+    while (it.next(s, seg)) {
+      int mt, nt;
+      tile_coords(s, seg.tile, mt, nt);
+      const int m0 = mt * BM + 4 * static_cast<int>(lane);
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++kc) {
+        const int slot = static_cast<int>(kc % kRing);
+        const uint32_t ph = (kc / kRing) & 1;
+        if (!dead) dead = !mbar_wait(sempty_bar(slot), ph ^ 1u, abort_flag, limit);
+        dead = __any_sync(0xffffffffu, dead);
+        if (!dead) {
+          const float* src = p.sa + static_cast<long long>(kb) * M + m0;
+          float4 v;
+          if (vec && m0 + 4 <= M) {
+            v = __ldg(reinterpret_cast<const float4*>(src));
+          } else {
+            v.x = m0 < M ? src[0] : 0.0f;
+            v.y = m0 + 1 < M ? src[1] : 0.0f;
+            v.z = m0 + 2 < M ? src[2] : 0.0f;
+            v.w = m0 + 3 < M ? src[3] : 0.0f;
+          }
+          float* dst = ring + slot * kSlotFloats;
+          reinterpret_cast<float4*>(dst)[lane] = v;
+          if (lane == 0) dst[128] = __ldg(p.sb + static_cast<long long>(kb) * p.nb_count + nt);
+        }
+        mbar_arrive(sfull_bar(slot));
+      }
+    }
   } else if (warp >= kPromoWarp0) {
     // ---------------------------------------------------------------- promotion + epilogue
     const int q = warp & 3;
@@ -154,66 +207,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c_local0 = half * 64;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     const int ptid = threadIdx.x - kPromoWarp0 * 32;
-    const int M = p.e.M;
-    long long kcount = 0;
+    uint32_t kcount = 0;
     WorkIter it;
     it.init(s, blockIdx.x);
     Seg seg;
     // `dead` is warp-uniform. After an abandoned wait the loop keeps walking the
     // (deterministic) segment list without touching TMEM or memory, so every named
-    // barrier below is still reached by all 256 promotion threads.
+    // barrier below is still reached by all promotion threads.
     bool dead = false;
     while (it.next(s, seg)) {
       int mt, nt;
       tile_coords(s, seg.tile, mt, nt);
       const int row = mt * BM + r_local;
-      const bool row_ok = row < M;
       float acc[64];
 #pragma unroll
       for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
       for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++kcount) {
         const int buf = static_cast<int>(kcount & 1);
-        const uint32_t bphase = static_cast<uint32_t>((kcount >> 1) & 1);
-        // scale of this row and K-block; issued before the wait so its latency hides
-        const float sa = row_ok ? __ldg(p.sa + static_cast<long long>(kb) * M + row) : 0.0f;
-        const float sb = __ldg(p.sb + static_cast<long long>(kb) * p.nb_count + nt);
+        const uint32_t bphase = (kcount >> 1) & 1;
+        const int slot = static_cast<int>(kcount % kRing);
+        const uint32_t sph = (kcount / kRing) & 1;
+        if (!dead) dead = !mbar_wait(sfull_bar(slot), sph, abort_flag, limit);
         if (!dead) dead = !mbar_wait(pfull_bar(buf), bphase, abort_flag, limit);
         dead = __any_sync(0xffffffffu, dead);
         if (dead) continue;
+        const float* sl = ring + slot * kSlotFloats;
+        const float sc = sl[r_local] * sl[128];
         tc_fence_after();
-        const float sc = sa * sb;
         const uint32_t taddr = tmem_base + lane_addr + buf * BN + c_local0;
+        // Both 32-column loads are issued before one wait: one TMEM round trip per K-block.
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(taddr, r0);
+        tmem_ld_32x32b_x32(taddr + 32, r1);
+        tmem_ld_wait();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + h * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc[h * 32 + j] = fmaf(sc, __uint_as_float(r[j]), acc[h * 32 + j]);
+        for (int j = 0; j < 32; ++j) {
+          acc[j] = fmaf(sc, __uint_as_float(r0[j]), acc[j]);
+          acc[32 + j] = fmaf(sc, __uint_as_float(r1[j]), acc[32 + j]);
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(pempty_bar(buf));
+        if (lane == 0) {
+          mbar_arrive(pempty_bar(buf));
+          mbar_arrive(sempty_bar(slot));
+        }
       }
 
       const bool whole = (seg.kb0 == 0 && seg.kb1 == s.kb_total);
       const int col0 = nt * BN + c_local0;
       if (whole) {
         if (!dead) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            float v[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = acc[h * 32 + j];
-            epi_row32(p.e, row, col0 + h * 32, v);
-          }
+          epi_row32(p.e, row, col0, *reinterpret_cast<float(*)[32]>(acc));
+          epi_row32(p.e, row, col0 + 32, *reinterpret_cast<float(*)[32]>(acc + 32));
         }
       } else {
         // Stream-K partial: store, then the last contributor reduces in CTA order.
         float* my_slot = p.slots + (static_cast<size_t>(blockIdx.x) * 2 + seg.slot) * (BM * BN);
-        if (!dead) {
-          slot_store<64>(my_slot, r_local, c_local0, acc);
-        }
+        if (!dead) slot_store<64>(my_slot, r_local, c_local0, acc);
         const long long t_sk = seg.tile - s.dp_tiles;
         __threadfence();
         named_barrier_sync(1, kPromoThreads);
@@ -231,19 +281,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           __threadfence();
           const int c_lo = sk_owner(s, t_sk * s.kb_total);
           const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
-#pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
-            float v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+          for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
 #pragma unroll 1
-            for (int cc = c_lo; cc <= c_hi; ++cc) {
-              if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
-              const float* src = p.slots + (static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * (BM * BN);
-              slot_accumulate<32>(src, r_local, c_local0 + h * 32, v);
-            }
-            epi_row32(p.e, row, col0 + h * 32, v);
+          for (int cc = c_lo; cc <= c_hi; ++cc) {
+            if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
+            const float* src = p.slots + (static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * (BM * BN);
+            slot_accumulate<64>(src, r_local, c_local0, acc);
           }
+          epi_row32(p.e, row, col0, *reinterpret_cast<float(*)[32]>(acc));
+          epi_row32(p.e, row, col0 + 32, *reinterpret_cast<float(*)[32]>(acc + 32));
         }
         named_barrier_sync(1, kPromoThreads);
       }
@@ -258,10 +305,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Fp8Params& p,
                             int grid, cudaStream_t stream) {
-  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5) + 16;
+  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + kRing * kSlotFloats * 4 + 8 * (2 * STAGES + 5 + 2 * kRing) + 16;
   static_assert(SMEM <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(gemm_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-  if (e != cudaSuccess) return e;
+  static const cudaError_t attr =
+      cudaFuncSetAttribute(gemm_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (attr != cudaSuccess) return attr;
   gemm_fp8_kernel<<<grid, kThreads, SMEM, stream>>>(tm_a, tm_b, p);
   return cudaGetLastError();
 }

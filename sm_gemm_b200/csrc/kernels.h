@@ -62,6 +62,12 @@ cudaError_t launch_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& tm_b, co
                             int grid, cudaStream_t stream);
 constexpr int kFp8BM = 128, kFp8BN = 128, kFp8BK = 128;
 
+// CTA-pair FP8 kernel (256 x 256 per cluster of 2); p.s counts clusters, p.slots is
+// [clusters][2][2 ranks][256][128] floats, p.counters [stream-K tiles][2].
+cudaError_t launch_gemm_fp8_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Fp8Params& p,
+                                 int clusters, cudaStream_t stream);
+int fp8_pair_max_clusters();
+
 // C[m, n] = act(bias[n]) (or act(0)) for the K == 0 degenerate GEMM.
 cudaError_t launch_fill_epilogue(int M, int N, const void* bias, int bias_dtype, int act, void* C,
                                  int c_dtype, long long ldc, cudaStream_t stream);
@@ -78,5 +84,6 @@ unsigned take_error_word_tc16();
 unsigned take_error_word_fp8();
 unsigned take_error_word_misc();
 unsigned take_error_word_pair();
+unsigned take_error_word_fp8_pair();
 
 }  // namespace smg

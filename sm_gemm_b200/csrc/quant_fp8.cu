@@ -35,41 +35,55 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// One warp per 1x128 group of a row-major X (element (r, c) at r*ldx + c).
+// Row-major X (element (r, c) at r*ldx + c): each warp quantises kGroupsPerWarp
+// consecutive 1x128 groups; every lane issues all of its 16-byte loads before using
+// any, so enough bytes are in flight to keep HBM busy.
+constexpr int kGroupsPerWarp = 4;
 __global__ void __launch_bounds__(256) quant_1x128_rows_kernel(const float* __restrict__ X, long long rows,
                                                                long long cols, long long ldx,
                                                                uint8_t* __restrict__ Q, float* __restrict__ S) {
   const long long kbn = (cols + 127) / 128;
-  const long long g = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (g >= rows * kbn) return;
+  const long long total = rows * kbn;
+  const long long g0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kGroupsPerWarp;
+  if (g0 >= total) return;
   const int lane = threadIdx.x & 31;
-  const long long r = g / kbn, kb = g - r * kbn;
-  const long long c0 = kb * 128 + lane * 4;
-  const float* src = X + r * ldx;
-  float v[4];
-  const bool vec = (kb * 128 + 128 <= cols) && ((ldx & 3) == 0);
-  if (vec) {
-    const float4 t = __ldcs(reinterpret_cast<const float4*>(src + c0));
-    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-  } else {
+  const bool vec_ld = (ldx & 3) == 0;
+  float v[kGroupsPerWarp][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = (c0 + j < cols) ? src[c0 + j] : 0.0f;
-  }
-  float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-  amax = warp_max(amax);
-  const float s = group_scale(amax);
-  const uint32_t lo = e4m3x2(__fdiv_rn(v[0], s), __fdiv_rn(v[1], s));
-  const uint32_t hi = e4m3x2(__fdiv_rn(v[2], s), __fdiv_rn(v[3], s));
-  uint8_t* dst = Q + r * cols + c0;
-  if (vec && (cols & 3) == 0) {
-    *reinterpret_cast<uint32_t*>(dst) = lo | (hi << 16);
-  } else {
-    const uint32_t w = lo | (hi << 16);
+  for (int i = 0; i < kGroupsPerWarp; ++i) {
+    const long long g = g0 + i;
+    const long long r = g / kbn, kb = g - r * kbn;
+    const long long c0 = kb * 128 + lane * 4;
+    const float* src = X + r * ldx;
+    if (g < total && vec_ld && kb * 128 + 128 <= cols) {
+      const float4 t = __ldcs(reinterpret_cast<const float4*>(src + c0));
+      v[i][0] = t.x; v[i][1] = t.y; v[i][2] = t.z; v[i][3] = t.w;
+    } else {
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (c0 + j < cols) dst[j] = static_cast<uint8_t>(w >> (8 * j));
+      for (int j = 0; j < 4; ++j) v[i][j] = (g < total && c0 + j < cols) ? src[c0 + j] : 0.0f;
+    }
   }
-  if (lane == 0) S[kb * rows + r] = s;
+#pragma unroll
+  for (int i = 0; i < kGroupsPerWarp; ++i) {
+    const long long g = g0 + i;
+    if (g >= total) break;
+    const long long r = g / kbn, kb = g - r * kbn;
+    const long long c0 = kb * 128 + lane * 4;
+    float amax = fmaxf(fmaxf(fabsf(v[i][0]), fabsf(v[i][1])), fmaxf(fabsf(v[i][2]), fabsf(v[i][3])));
+    amax = warp_max(amax);
+    const float sc = group_scale(amax);
+    const uint32_t w = e4m3x2(__fdiv_rn(v[i][0], sc), __fdiv_rn(v[i][1], sc)) |
+                       (e4m3x2(__fdiv_rn(v[i][2], sc), __fdiv_rn(v[i][3], sc)) << 16);
+    uint8_t* dst = Q + r * cols + c0;
+    if (kb * 128 + 128 <= cols && (cols & 3) == 0) {
+      *reinterpret_cast<uint32_t*>(dst) = w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (c0 + j < cols) dst[j] = static_cast<uint8_t>(w >> (8 * j));
+    }
+    if (lane == 0) S[kb * rows + r] = sc;
+  }
 }
 
 // One thread per (row, group) of a column-major X (element (r, c) at c*ldx + r):
@@ -98,29 +112,80 @@ __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(const float* __re
 }
 
 // One CTA per 128x128 block of the weight X[K, N] (element (k, n) at k*rs + n*cs).
-// The block is staged transposed in shared memory ([n][k], padded row of 129) so the
-// codes can be written as Q[n][k] rows of up to 128 contiguous bytes.
-constexpr int kQPitch = 129;
+// Phase 1 loads the block with 16-byte loads (16 per thread, all issued before use)
+// and stages it transposed in shared memory as [n][k]; phase 2 has each thread encode
+// 64 consecutive k of one n and write them as 16-byte rows of Q[n][k]. The shared tile
+// is XOR-swizzled (column k of row n stored at k ^ g(n), g(n) = ((n >> 2) ^ ((n & 3) << 3)) & 31)
+// so both the transposing stores of phase 1 and the row reads of phase 2 are free of
+// bank conflicts.
+__device__ __forceinline__ int qswz(int n) { return ((n >> 2) ^ ((n & 3) << 3)) & 31; }
+
 __global__ void __launch_bounds__(256) quant_128x128_kernel(const float* __restrict__ X, long long K, long long N,
                                                             long long rs, long long cs, uint8_t* __restrict__ Q,
                                                             float* __restrict__ S) {
-  extern __shared__ float tile[];  // [128][kQPitch]
+  extern __shared__ float tile[];  // [128 n][128 k], swizzled
   __shared__ float warp_amax[8];
   const long long kb = blockIdx.y, nb = blockIdx.x;
   const long long k0 = kb * 128, n0 = nb * 128;
   const long long nbn = (N + 127) / 128;
   const int t = threadIdx.x;
-  const bool n_contig = (cs == 1);
   float amax = 0.0f;
-#pragma unroll 4
-  for (int i = 0; i < 64; ++i) {
-    const int idx = i * 256 + t;
-    const int kk = n_contig ? (idx >> 7) : (idx & 127);
-    const int nn = n_contig ? (idx & 127) : (idx >> 7);
-    const long long k = k0 + kk, n = n0 + nn;
-    const float x = (k < K && n < N) ? __ldcs(X + k * rs + n * cs) : 0.0f;
-    amax = fmaxf(amax, fabsf(x));
-    tile[nn * kQPitch + kk] = x;
+  if (cs == 1) {
+    // N contiguous: float4 = 4 consecutive n of one k. idx -> (kk = idx / 32, n4 = idx % 32).
+    const bool vec = (rs & 3) == 0 && n0 + 128 <= N;
+    float4 r4[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int idx = i * 256 + t, kk = idx >> 5, n4 = idx & 31;
+      const long long k = k0 + kk, n = n0 + 4 * n4;
+      if (k < K && vec) {
+        r4[i] = __ldcs(reinterpret_cast<const float4*>(X + k * rs + n));
+      } else {
+        float e[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) e[q] = (k < K && n + q < N) ? X[k * rs + n + q] : 0.0f;
+        r4[i] = make_float4(e[0], e[1], e[2], e[3]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int idx = i * 256 + t, kk = idx >> 5, n4 = idx & 31;
+      const float e[4] = {r4[i].x, r4[i].y, r4[i].z, r4[i].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int n = 4 * n4 + q;
+        amax = fmaxf(amax, fabsf(e[q]));
+        tile[n * 128 + (kk ^ qswz(n))] = e[q];
+      }
+    }
+  } else {
+    // K contiguous (rs == 1) or general strides: float4 = 4 consecutive k of one n when
+    // possible. idx -> (n = idx / 32, k4 = idx % 32).
+    const bool vec = rs == 1 && (cs & 3) == 0 && k0 + 128 <= K;
+    float4 r4[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int idx = i * 256 + t, nn = idx >> 5, k4 = idx & 31;
+      const long long n = n0 + nn, k = k0 + 4 * k4;
+      if (n < N && vec) {
+        r4[i] = __ldcs(reinterpret_cast<const float4*>(X + n * cs + k));
+      } else {
+        float e[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) e[q] = (n < N && k + q < K) ? X[(k + q) * rs + n * cs] : 0.0f;
+        r4[i] = make_float4(e[0], e[1], e[2], e[3]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int idx = i * 256 + t, nn = idx >> 5, k4 = idx & 31;
+      const float e[4] = {r4[i].x, r4[i].y, r4[i].z, r4[i].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        amax = fmaxf(amax, fabsf(e[q]));
+        tile[nn * 128 + ((4 * k4 + q) ^ qswz(nn))] = e[q];
+      }
+    }
   }
   amax = warp_max(amax);
   if ((t & 31) == 0) warp_amax[t >> 5] = amax;
@@ -128,14 +193,15 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(const float* __restr
   float m = warp_amax[0];
 #pragma unroll
   for (int w = 1; w < 8; ++w) m = fmaxf(m, warp_amax[w]);
-  const float s = group_scale(m);
-  if (t == 0) S[kb * nbn + nb] = s;
+  const float sc = group_scale(m);
+  if (t == 0) S[kb * nbn + nb] = sc;
 
-  // Thread t: output row n = n0 + t/2, k range [64*(t&1), +64).
-  const int nn = t >> 1;
-  const int kh = (t & 1) * 64;
+  // Phase 2: warp w, lane l -> row n = 32*(w & 3) + l, k in [64*(w >> 2), +64).
+  const int nn = 32 * ((t >> 5) & 3) + (t & 31);
+  const int kh = 64 * (t >> 7);
   const long long n = n0 + nn;
   if (n >= N) return;
+  const int g = qswz(nn);
   uint8_t* dst = Q + n * K + k0 + kh;
   const bool vec = (k0 + kh + 64 <= K) && ((K & 15) == 0);
 #pragma unroll
@@ -143,9 +209,10 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(const float* __restr
     uint32_t w[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      const float* src = tile + nn * kQPitch + kh + u * 16 + h * 4;
-      const uint32_t lo = e4m3x2(__fdiv_rn(src[0], s), __fdiv_rn(src[1], s));
-      const uint32_t hi = e4m3x2(__fdiv_rn(src[2], s), __fdiv_rn(src[3], s));
+      const int kk = kh + u * 16 + h * 4;
+      const float* row = tile + nn * 128;
+      const uint32_t lo = e4m3x2(__fdiv_rn(row[(kk + 0) ^ g], sc), __fdiv_rn(row[(kk + 1) ^ g], sc));
+      const uint32_t hi = e4m3x2(__fdiv_rn(row[(kk + 2) ^ g], sc), __fdiv_rn(row[(kk + 3) ^ g], sc));
       w[h] = lo | (hi << 16);
     }
     if (vec) {
@@ -191,7 +258,7 @@ cudaError_t launch_quant_1x128(const float* X, long long rows, long long cols, l
   const long long kbn = (cols + 127) / 128;
   if (cs == 1) {
     const long long groups = rows * kbn;
-    const long long blocks = (groups + 7) / 8;
+    const long long blocks = (groups + 8 * kGroupsPerWarp - 1) / (8 * kGroupsPerWarp);
     quant_1x128_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(X, rows, cols, rs, Q, S);
   } else {
     dim3 grid(static_cast<unsigned>((rows + 255) / 256), static_cast<unsigned>(kbn));
@@ -202,7 +269,7 @@ cudaError_t launch_quant_1x128(const float* X, long long rows, long long cols, l
 
 cudaError_t launch_quant_128x128(const float* X, long long K, long long N, long long rs, long long cs,
                                  uint8_t* Q, float* S, cudaStream_t stream) {
-  const int smem = 128 * kQPitch * static_cast<int>(sizeof(float));
+  const int smem = 128 * 128 * static_cast<int>(sizeof(float));
   cudaError_t e = cudaFuncSetAttribute(quant_128x128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((K + 127) / 128));

@@ -91,7 +91,9 @@ def _run_fp8(qa, sa, qb, sb, out_dt=torch.bfloat16, bias=None, act="none"):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 128, 128), (300, 260, 384), (64, 1000, 1024), (257, 129, 2048)])
-def test_fp8_gemm_within_tolerance(cuda_device, M, N, K):
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_fp8_gemm_within_tolerance(cuda_device, monkeypatch, M, N, K, pair):
+    monkeypatch.setenv("SMGEMM_PAIR", pair)
     qa, sa, qb, sb = _quantised_problem(M, N, K, seed=M + N + K)
     got = _run_fp8(qa, sa, qb, sb)
     ref, acc = oracle.gemm_fp8(qa, sa, qb, sb, out_dtype=oracle.BF16, want_absacc=True)
@@ -99,8 +101,11 @@ def test_fp8_gemm_within_tolerance(cuda_device, M, N, K):
 
 
 @pytest.mark.parametrize("sched", ["dp", "sk", "auto"])
-def test_fp8_gemm_integer_codes_unit_scales_exact(cuda_device, monkeypatch, sched):
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_fp8_gemm_integer_codes_unit_scales_exact(cuda_device, monkeypatch, sched, pair):
+    """pair=1: 256x256 tiles on CTA pairs; pair=0: 128x128 one-SM tiles."""
     monkeypatch.setenv("SMGEMM_SCHED", sched)
+    monkeypatch.setenv("SMGEMM_PAIR", pair)
     rs = np.random.RandomState(5)
     M, N, K = 300, 400, 1024
     qa = oracle.e4m3_encode(rs.randint(-8, 9, (M, K)).astype(np.float32))
