@@ -64,7 +64,8 @@ typedef enum { SMGEMM_ACT_NONE = 0, SMGEMM_ACT_GELU_TANH = 1, SMGEMM_ACT_SILU = 
  *            (row-major: ldb >= N; col-major, i.e. W^T stored [N,K]: ldb >= K).
  *   bias     device, nullable; bias_dtype SMGEMM_BF16 / SMGEMM_F16 / SMGEMM_F32; N entries.
  *   act      SMGEMM_ACT_NONE, SMGEMM_ACT_GELU_TANH (0.5x(1+tanh(sqrt(2/pi)(x+0.044715x^3))))
- *            or SMGEMM_ACT_SILU (x/(1+e^-x)); applied in FP32 after the bias add.
+ *            or SMGEMM_ACT_SILU (x/(1+e^-x)); applied in FP32 after the bias add, with the
+ *            hardware tanh approximation (relative error ~2^-11) and the fast exponential.
  *   C        device, c_dtype SMGEMM_F32 / SMGEMM_BF16 / SMGEMM_F16, row-major, ldc >= N.
  *   workspace  device scratch of at least smgemm_workspace_size(M,N,K,0) bytes,
  *            16-byte aligned (may be NULL when that size is 0). The library uses it

@@ -21,12 +21,32 @@ struct EpiArgs {
   long long ldc;
 };
 
+// Activations in FP32. The GEMM epilogues use the hardware tanh.approx.f32 (maximum
+// relative error about 2^-11, some 16x below half a bf16 ulp) and the fast exponential
+// __expf: the GeLU/SiLU arithmetic then stays a few instructions per element, so the
+// epilogue warps keep pace with the tensor cores. act_apply_precise uses the libm
+// functions (tanhf, expf) for the K == 0 fill, which has no GEMM to hide behind.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float act_apply(float x, int act) {
-  if (act == 1) {  // GeLU, tanh form
+  if (act == 1) {  // GeLU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
     const float c = 0.7978845608028654f;  // sqrt(2/pi)
+    return 0.5f * x * (1.0f + tanh_approx(c * (x + 0.044715f * x * x * x)));
+  }
+  if (act == 2) return x / (1.0f + __expf(-x));  // SiLU: x * sigmoid(x)
+  return x;
+}
+
+__device__ __forceinline__ float act_apply_precise(float x, int act) {
+  if (act == 1) {
+    const float c = 0.7978845608028654f;
     return 0.5f * x * (1.0f + tanhf(c * (x + 0.044715f * x * x * x)));
   }
-  if (act == 2) return x / (1.0f + expf(-x));  // SiLU
+  if (act == 2) return x / (1.0f + expf(-x));
   return x;
 }
 

@@ -232,7 +232,7 @@ __global__ void fill_epilogue_kernel(int M, int N, const void* bias, int bias_dt
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long r = i / N, c = i - r * N;
     const float b = bias != nullptr ? load_bias(bias, bias_dtype, static_cast<int>(c)) : 0.0f;
-    store_one(C, c_dtype, r * ldc + c, act_apply(b, act));
+    store_one(C, c_dtype, r * ldc + c, act_apply_precise(b, act));
   }
 }
 
