@@ -241,20 +241,24 @@ Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms, i
   return g;
 }
 
-// FP8 tiles run on CTA pairs (256 x 256) unless SMGEMM_PAIR=0 or no pair cluster fits.
+// FP8 tiles run on CTA pairs (256 x tn) unless SMGEMM_PAIR=0 or no pair cluster fits.
 struct Fp8Plan {
   bool pair;
+  int tn;  // pair tile width: 256 or 128
   Plan pl;
 };
 
-Fp8Plan plan_fp8(int64_t M, int64_t N, int64_t K, int sms, int pair_clusters) {
+int fp8_tile_n() { return env_ll("SMGEMM_FP8_TN", 256) == 128 ? 128 : 256; }
+
+Fp8Plan plan_fp8(int64_t M, int64_t N, int64_t K, int sms, int tn, int pair_clusters) {
   Fp8Plan f;
   const int kb = static_cast<int>((K + kFp8BK - 1) / kFp8BK);
   const int group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", 8));
   f.pair = pair_clusters > 0 && env_ll("SMGEMM_PAIR", 1) != 0;
+  f.tn = tn;
   if (f.pair) {
-    f.pl = make_plan(static_cast<int>((M + 255) / 256), static_cast<int>((N + 255) / 256), std::max(kb, 1),
-                     pair_clusters, group_m, static_cast<size_t>(2) * 128 * 256, 2);
+    f.pl = make_plan(static_cast<int>((M + 255) / 256), static_cast<int>((N + tn - 1) / tn), std::max(kb, 1),
+                     pair_clusters, group_m, static_cast<size_t>(2) * 128 * tn, 2);
   } else {
     f.pl = make_plan(static_cast<int>((M + kFp8BM - 1) / kFp8BM), static_cast<int>((N + kFp8BN - 1) / kFp8BN),
                      std::max(kb, 1), sms, group_m, static_cast<size_t>(kFp8BM) * kFp8BN);
@@ -311,7 +315,7 @@ size_t smgemm_workspace_size(int64_t M, int64_t N, int64_t K, int kind) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   DevInfo d;
   if (current_device(d) != SMGEMM_OK) return 0;
-  if (kind == 1) return plan_fp8(M, N, K, d.sms, fp8_pair_max_clusters()).pl.ws_bytes();
+  if (kind == 1) return plan_fp8(M, N, K, d.sms, fp8_tile_n(), fp8_pair_max_clusters(fp8_tile_n())).pl.ws_bytes();
   // enough for either path (the skinny path is only taken for a row-major A)
   const int pc = tc16_pair_max_clusters();
   return std::max(plan_gemm16(M, N, K, SMGEMM_ROW_MAJOR, d.sms, pc).pl.ws_bytes(),
@@ -409,17 +413,18 @@ smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_
     return launch_status(launch_fill_epilogue(static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C,
                                               c_dtype, ldc, stream));
   }
-  const Fp8Plan f = plan_fp8(M, N, K, d.sms, fp8_pair_max_clusters());
+  const int tn = fp8_tile_n();
+  const Fp8Plan f = plan_fp8(M, N, K, d.sms, tn, fp8_pair_max_clusters(tn));
   const Plan& pl = f.pl;
   CUtensorMap tm_a, tm_b;
   bool ok = encode_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, Aq, K, M, K, 128, 128);
-  ok = ok && encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, Bq, K, N, K, 128, 128);
+  ok = ok && encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, Bq, K, N, K, 128, f.pair ? f.tn / 2 : 128);
   if (!ok) return SMGEMM_ERR_CUDA;
   Fp8Params p{};
   p.s = pl.s;
   p.e = EpiArgs{static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C, c_dtype, ldc};
   p.K = static_cast<int>(K);
-  p.idesc = f.pair ? idesc_f32acc(0u, 0u, 0u, 0u, 256, 256) : idesc_f32acc(0u, 0u, 0u, 0u, 128, 128);
+  p.idesc = f.pair ? idesc_f32acc(0u, 0u, 0u, 0u, 256, f.tn) : idesc_f32acc(0u, 0u, 0u, 0u, 128, 128);
   p.sa = sa;
   p.sb = sb;
   p.nb_count = static_cast<int>((N + 127) / 128);
@@ -427,8 +432,8 @@ smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_
   st = prepare_workspace(pl, workspace, workspace_bytes, stream, &p.slots, &p.counters);
   if (st != SMGEMM_OK) return st;
   if (f.pair) {
-    note_config("fp8pair", pl, 256);
-    return launch_status(launch_gemm_fp8_pair(tm_a, tm_b, p, pl.grid, stream));
+    note_config("fp8pair", pl, f.tn);
+    return launch_status(launch_gemm_fp8_pair(tm_a, tm_b, p, pl.grid, f.tn, stream));
   }
   note_config("fp8", pl, 128);
   return launch_status(launch_gemm_fp8(tm_a, tm_b, p, pl.grid, stream));
@@ -476,7 +481,7 @@ smgemm_status smgemm_selftest_wait_timeout(uint32_t limit_us, smgemm_stream_t st
 int64_t smgemm_schedule_dump(int64_t M, int64_t N, int64_t K, int kind, smgemm_layout layout_a, int num_sms,
                              int32_t* out, int64_t cap) {
   if (M <= 0 || N <= 0 || K <= 0 || num_sms <= 0) return 0;
-  const Plan pl = kind == 1 ? plan_fp8(M, N, K, num_sms, num_sms / 2).pl
+  const Plan pl = kind == 1 ? plan_fp8(M, N, K, num_sms, fp8_tile_n(), num_sms / 2).pl
                             : plan_gemm16(M, N, K, layout_a, num_sms, num_sms / 2).pl;
   int64_t n = 0;
   for (int c = 0; c < pl.grid; ++c) {

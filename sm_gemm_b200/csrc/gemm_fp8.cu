@@ -15,10 +15,11 @@
 // allocator, warp 3 scale loader, warps 4..11 promotion + epilogue: warp w reads TMEM
 // lanes 32*(w%4).. (tile rows) and columns 64*((w-4)/4).. (64 of the 128 columns).
 //
-// The scale loader stages each K-block's 128 row scales and its block scale in a
-// 4-slot shared-memory ring. Promotion warps then never have a global load in flight
-// when they release a TMEM buffer (an mbarrier arrive has release semantics and
-// would wait for such loads), and read their scales from shared memory.
+// The scale loader stages each K-block's 128 row scales and its block scale in an
+// 8-slot shared-memory ring with asynchronous copies. Promotion warps then never have
+// a global load in flight when they release a TMEM buffer (an mbarrier arrive has
+// release semantics and would wait for such loads), and read their scales from
+// shared memory.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -40,7 +41,7 @@ constexpr int B_BYTES = BN * BKB;                       // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int STAGES = 6;
 constexpr int TCOLS = 256;       // two 128-column FP32 partial buffers
-constexpr int kRing = 4;         // scale ring slots
+constexpr int kRing = 8;         // scale ring slots
 constexpr int kSlotFloats = 132; // 128 row scales + block scale, padded to 16 bytes
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int i) {
@@ -166,12 +167,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kLoaderWarp) {
     // ---------------------------------------------------------------- scale loader
     // Slot layout: [0, 128) row scales sa[kb, m0 + r]; [128] block scale sb[kb, nt].
+    // Asynchronous copies (cp.async, zero fill past the matrix edge) complete on the
+    // slot's full barrier, so up to kRing K-blocks of scales are in flight at once.
     uint32_t kc = 0;
     WorkIter it;
     it.init(s, blockIdx.x);
     Seg seg;
     bool dead = false;
-    const bool vec = (M & 3) == 0;
+    const bool vec = (M & 3) == 0 && (reinterpret_cast<uintptr_t>(p.sa) & 15u) == 0;
+    const uint32_t ring_u32 = smem_u32(ring);
     while (it.next(s, seg)) {
       int mt, nt;
       tile_coords(s, seg.tile, mt, nt);
@@ -181,24 +185,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (kc / kRing) & 1;
         if (!dead) dead = !mbar_wait(sempty_bar(slot), ph ^ 1u, abort_flag, limit);
         dead = __any_sync(0xffffffffu, dead);
-        if (!dead) {
-          const float* src = p.sa + static_cast<long long>(kb) * M + m0;
-          float4 v;
-          if (vec && m0 + 4 <= M) {
-            v = __ldg(reinterpret_cast<const float4*>(src));
-          } else {
-            v.x = m0 < M ? src[0] : 0.0f;
-            v.y = m0 + 1 < M ? src[1] : 0.0f;
-            v.z = m0 + 2 < M ? src[2] : 0.0f;
-            v.w = m0 + 3 < M ? src[3] : 0.0f;
-          }
-          float* dst = ring + slot * kSlotFloats;
-          reinterpret_cast<float4*>(dst)[lane] = v;
-          if (lane == 0) dst[128] = __ldg(p.sb + static_cast<long long>(kb) * p.nb_count + nt);
+        if (dead) {
+          mbar_arrive(sfull_bar(slot));
+          continue;
         }
-        mbar_arrive(sfull_bar(slot));
+        const float* src = p.sa + static_cast<long long>(kb) * M + m0;
+        const uint32_t dst = ring_u32 + static_cast<uint32_t>(slot * kSlotFloats * 4);
+        if (vec) {
+          cp_async_16(dst + 16 * lane, m0 < M ? src : p.sa, m0 < M ? 16u : 0u);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            cp_async_4(dst + 16 * lane + 4 * e, m0 + e < M ? src + e : p.sa, m0 + e < M ? 4u : 0u);
+        }
+        if (lane == 0) cp_async_4(dst + 4 * 128, p.sb + static_cast<long long>(kb) * p.nb_count + nt, 4u);
+        cp_async_mbar_arrive(sfull_bar(slot));
       }
     }
+    cp_async_wait_all();
   } else if (warp >= kPromoWarp0) {
     // ---------------------------------------------------------------- promotion + epilogue
     const int q = warp & 3;
@@ -240,11 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(taddr, r0);
         tmem_ld_32x32b_x32(taddr + 32, r1);
         tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          acc[j] = fmaf(sc, __uint_as_float(r0[j]), acc[j]);
-          acc[32 + j] = fmaf(sc, __uint_as_float(r1[j]), acc[32 + j]);
-        }
+        fma_scaled32(acc, sc, r0);
+        fma_scaled32(acc + 32, sc, r1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {

@@ -1,24 +1,30 @@
-// Block-scaled FP8 (E4M3) GEMM on CTA pairs (tcgen05.mma.cta_group::2), 256 x 256
-// output tile per pair of SMs, with per-K-block scale promotion into FP32 registers.
+// Block-scaled FP8 (E4M3) GEMM on CTA pairs (tcgen05.mma.cta_group::2): a 256 x TN
+// output tile per pair of SMs (TN = 256 or 128), with per-K-block scale promotion into
+// FP32 registers.
 //
 // Same method as gemm_fp8.cu (the DeepGEMM kernel-library walkthrough, zwxr.cn,
 // section 2.4: one FP32 scale per 1x128 activation group and per 128x128 weight block,
 // FP32 accumulation, rescale per group): for each 128-wide K-block kb the pair's
-// tensor cores write the FP32 partial P_kb of the 256 x 256 tile into one of two TMEM
-// buffers (each SM holds its 128 rows x 256 columns), and 16 promotion warps per SM
-// fold it into registers, acc += (sa[kb, m] * sb[kb, n / 128]) * P_kb. The pair tile
-// halves each SM's shared-memory operand traffic against a one-SM 128 x 128 tile (32 KB
-// per 512 MMA cycles instead of per 256), which is what bounds the one-SM kernel.
+// tensor cores write the FP32 partial P_kb of the 256 x TN tile into one of the TMEM
+// buffers (each SM holds its 128 rows x TN columns), and 8 promotion warps per SM
+// fold it into registers, acc += (sa[kb, m] * sb[kb, n / 128]) * P_kb.
+//
+// TMEM holds 512 / TN partial buffers, and the MMA of K-block kb can only start once
+// the promotion of kb - 512/TN has freed its buffer. With TN = 256 (two buffers) the
+// K loop is bound by that round trip (MMA latency + promotion latency over two
+// K-blocks) rather than by the tensor cores; TN = 128 has four buffers and twice the
+// slack, at the price of re-reading A once per 128 instead of 256 output columns.
 //
 // Roles (384 threads per CTA = 3 warpgroups):
 //  warp 0     TMEM allocator (whole warp), then lane 0 is the TMA producer.
 //  warp 1     MMA issuer (rank-0 CTA only).
-//  warp 2     scale loader: stages each K-block's 128 row scales and two block scales of
-//             this CTA in a shared-memory ring, so promotion warps never hold a global
-//             load in flight when they release a TMEM buffer (an mbarrier arrive has
-//             release semantics and would wait for it).
+//  warp 2     scale loader: stages each K-block's 128 row scales and the block scales of
+//             this CTA in a shared-memory ring with asynchronous copies, so promotion
+//             warps never hold a global load in flight when they release a TMEM buffer
+//             (an mbarrier arrive has release semantics and would wait for it).
 //  warps 4-11 promotion + epilogue: warp w reads TMEM lanes 32*(w%4).. (tile rows) and
-//             the 128 columns 128*((w-4)/4).. of the 256; 128 FP32 accumulators per thread.
+//             the TN/2 columns (TN/2)*((w-4)/4).. of the tile; TN/2 FP32 accumulators
+//             per thread.
 // Warpgroup 0 gives up registers (setmaxnreg 40) so the two promotion warpgroups can
 // hold the accumulators (setmaxnreg 232; 384 x 168 registers at launch).
 #include <cuda_bf16.h>
@@ -38,23 +44,37 @@ constexpr int kPromoWarps = 8;
 constexpr int kPromoThreads = kPromoWarps * 32;
 constexpr int BKB = 128;                 // K-block in bytes = elements = one scale group
 constexpr int A_BYTES = 128 * BKB;       // this CTA's 128 rows of A
-constexpr int B_BYTES = 128 * BKB;       // this CTA's 128 columns of B
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int STAGES = 6;
-constexpr int kTileN = 256;
-constexpr int TCOLS = 512;               // two 256-column FP32 partial buffers
-constexpr int kRing = 4;                 // scale ring slots
-constexpr int kSlotFloats = 132;         // 128 row scales + 2 block scales, padded to 16 B
+constexpr int TCOLS = 512;               // all of TMEM: 512 / TN partial buffers
+constexpr int kRing = 8;                 // scale ring slots
+constexpr int kSlotFloats = 132;         // 128 row scales + up to 2 block scales, padded to 16 B
 constexpr int kRoleRegs = 40, kPromoRegs = 232;  // setmaxnreg split (384 x 168 at launch)
+
+// Per-tile-width constants: this CTA's B rows (TN / 2), stage size, pipeline depth and
+// the number of TMEM partial buffers.
+template <int TN>
+struct PairCfg {
+  static constexpr int kBRows = TN / 2;
+  static constexpr int B_BYTES = kBRows * BKB;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = TN == 256 ? 6 : 8;
+  static constexpr int NBUF = TCOLS / TN;
+  static constexpr int CPW = TN / 2;                  // columns per promotion warp
+  static constexpr int kBars = 2 * STAGES + 2 * NBUF + 2 * kRing + 1;
+  static constexpr int kSmem = 1024 + STAGES * STAGE_BYTES + kRing * kSlotFloats * 4 + 8 * kBars + 16;
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int i) {
   return sdesc_sw128(base + i * 32, 16, 1024);
 }
 }  // namespace
 
+template <int TN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                          const Fp8Params p) {
+  using Cfg = PairCfg<TN>;
+  constexpr int STAGES = Cfg::STAGES, STAGE_BYTES = Cfg::STAGE_BYTES, NBUF = Cfg::NBUF, CPW = Cfg::CPW;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
@@ -63,11 +83,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
   auto pfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
-  auto pempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
-  auto sfull_bar = [&](int r) { return bar_base + 8u * (2 * STAGES + 4 + r); };
-  auto sempty_bar = [&](int r) { return bar_base + 8u * (2 * STAGES + 4 + kRing + r); };
-  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4 + 2 * kRing);
-  uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + kRing * kSlotFloats * 4 + 8 * (2 * STAGES + 5 + 2 * kRing);
+  auto pempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + NBUF + b); };
+  auto sfull_bar = [&](int r) { return bar_base + 8u * (2 * STAGES + 2 * NBUF + r); };
+  auto sempty_bar = [&](int r) { return bar_base + 8u * (2 * STAGES + 2 * NBUF + kRing + r); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 2 * NBUF + 2 * kRing);
+  uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + kRing * kSlotFloats * 4 + 8 * Cfg::kBars;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   volatile int* reduce_flag = reinterpret_cast<volatile int*>(misc + 8);
@@ -81,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(pfull_bar(b), 1);
       mbar_init(pempty_bar(b), 2 * kPromoWarps);
     }
@@ -125,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int mt, nt;
         tile_coords(s, seg.tile, mt, nt);
         const int a_row = mt * 256 + static_cast<int>(rank) * 128;
-        const int b_row = nt * kTileN + static_cast<int>(rank) * 128;
+        const int b_row = nt * TN + static_cast<int>(rank) * Cfg::kBRows;
         for (int kb = seg.kb0; kb < seg.kb1; ++kb) {
           if (!mbar_wait_inl(empty_bar(stage), phase ^ 1u, abort_flag, limit)) { ok = false; break; }
           const uint32_t sa_s = smem_base + stage * STAGE_BYTES;
@@ -159,13 +179,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       while (ok && it.next(s, seg)) {
         for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++kcount) {
-          const int buf = static_cast<int>(kcount & 1);
-          const uint32_t bphase = static_cast<uint32_t>((kcount >> 1) & 1);
+          const int buf = static_cast<int>(kcount % NBUF);
+          const uint32_t bphase = static_cast<uint32_t>((kcount / NBUF) & 1);
           if (!mbar_wait_inl(pempty_bar(buf), bphase ^ 1u, abort_flag, limit)) { ok = false; break; }
           if (!mbar_wait_inl(full_bar(stage), phase, abort_flag, limit)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa_s = smem_base + stage * STAGE_BYTES;
-          const uint32_t d_tmem = tmem_base + buf * kTileN;
+          const uint32_t d_tmem = tmem_base + buf * TN;
 #pragma unroll
           for (int k = 0; k < BKB / 32; ++k)
             umma_f8_pair(d_tmem, kmajor_desc(sa_s, k), kmajor_desc(sa_s + A_BYTES, k), p.idesc, k > 0 ? 1u : 0u);
@@ -181,14 +201,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kLoaderWarp) {
     // ---------------------------------------------------------------- scale loader
     // Slot layout: [0, 128) row scales sa[kb, m0 + r]; [128 + h] block scale of the tile's
-    // h-th 128-column half, sb[kb, 2 * nt + h].
+    // h-th 128-column block, sb[kb, (TN / 128) * nt + h]. The copies are asynchronous (cp.async,
+    // zero fill past the matrix edge) and complete on the slot's full barrier, so the
+    // loader keeps up to kRing K-blocks of scales in flight instead of one.
     const int M = p.e.M;
     uint32_t kc = 0;
     WorkIter it;
     it.init(s, cluster);
     Seg seg;
     bool dead = false;
-    const bool vec = (M & 3) == 0;
+    const bool vec = (M & 3) == 0 && (reinterpret_cast<uintptr_t>(p.sa) & 15u) == 0;
+    const uint32_t ring_u32 = smem_u32(ring);
     while (it.next(s, seg)) {
       int mt, nt;
       tile_coords(s, seg.tile, mt, nt);
@@ -198,39 +221,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (kc / kRing) & 1;
         if (!dead) dead = !mbar_wait_inl(sempty_bar(slot), ph ^ 1u, abort_flag, limit);
         dead = __any_sync(0xffffffffu, dead);
-        if (!dead) {
-          const float* src = p.sa + static_cast<long long>(kb) * M + m0;
-          float4 v;
-          if (vec && m0 + 4 <= M) {
-            v = __ldg(reinterpret_cast<const float4*>(src));
-          } else {
-            v.x = m0 < M ? src[0] : 0.0f;
-            v.y = m0 + 1 < M ? src[1] : 0.0f;
-            v.z = m0 + 2 < M ? src[2] : 0.0f;
-            v.w = m0 + 3 < M ? src[3] : 0.0f;
-          }
-          float* dst = ring + slot * kSlotFloats;
-          reinterpret_cast<float4*>(dst)[lane] = v;
-          if (lane < 2) {
-            const int nb = 2 * nt + static_cast<int>(lane);
-            dst[128 + lane] = nb < p.nb_count ? __ldg(p.sb + static_cast<long long>(kb) * p.nb_count + nb) : 0.0f;
-          }
+        if (dead) {
+          mbar_arrive(sfull_bar(slot));
+          continue;
         }
-        mbar_arrive(sfull_bar(slot));
+        const float* src = p.sa + static_cast<long long>(kb) * M + m0;
+        const uint32_t dst = ring_u32 + static_cast<uint32_t>(slot * kSlotFloats * 4);
+        if (vec) {
+          cp_async_16(dst + 16 * lane, m0 < M ? src : p.sa, m0 < M ? 16u : 0u);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            cp_async_4(dst + 16 * lane + 4 * e, m0 + e < M ? src + e : p.sa, m0 + e < M ? 4u : 0u);
+        }
+        if (lane < TN / 128) {
+          const int nb = (TN / 128) * nt + static_cast<int>(lane);
+          const float* sbp = p.sb + static_cast<long long>(kb) * p.nb_count + nb;
+          cp_async_4(dst + 4 * (128 + lane), nb < p.nb_count ? sbp : p.sb, nb < p.nb_count ? 4u : 0u);
+        }
+        cp_async_mbar_arrive(sfull_bar(slot));
       }
     }
+    cp_async_wait_all();
   }
   } else {
-    // Warpgroups 1-4: promotion + epilogue (64 accumulators per thread).
+    // Warpgroups 1-2: promotion + epilogue (CPW accumulators per thread).
     regs_inc<kPromoRegs>();
     // ---------------------------------------------------------------- promotion + epilogue
     const int q = warp & 3;
-    const int cg = (warp - kPromoWarp0) >> 2;  // 0..1: 128-column half of the tile
+    const int cg = (warp - kPromoWarp0) >> 2;  // 0..1: column half of the tile
     const int r_local = q * 32 + lane;
-    const int c_local0 = cg * 128;
+    const int c_local0 = cg * CPW;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     const int ptid = threadIdx.x - kPromoWarp0 * 32;
-    constexpr int SLOT = 128 * kTileN;
+    constexpr int SLOT = 128 * TN;
     uint32_t kcount = 0;
     WorkIter it;
     it.init(s, cluster);
@@ -240,12 +264,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       int mt, nt;
       tile_coords(s, seg.tile, mt, nt);
       const int row = mt * 256 + static_cast<int>(rank) * 128 + r_local;
-      float acc[128];
+      float acc[CPW];
 #pragma unroll
-      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < CPW; ++j) acc[j] = 0.0f;
       for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++kcount) {
-        const int buf = static_cast<int>(kcount & 1);
-        const uint32_t bphase = (kcount >> 1) & 1;
+        const int buf = static_cast<int>(kcount % NBUF);
+        const uint32_t bphase = (kcount / NBUF) & 1;
         const int slot = static_cast<int>(kcount % kRing);
         const uint32_t sph = (kcount / kRing) & 1;
         if (!dead) dead = !mbar_wait_inl(sfull_bar(slot), sph, abort_flag, limit);
@@ -253,18 +277,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         dead = __any_sync(0xffffffffu, dead);
         if (dead) continue;
         const float* sl = ring + slot * kSlotFloats;
-        const float sc = sl[r_local] * sl[128 + cg];
+        const float sc = sl[r_local] * sl[128 + c_local0 / 128];
         tc_fence_after();
-        const uint32_t taddr = tmem_base + lane_addr + buf * kTileN + c_local0;
-        // Four 32-column TMEM loads, each followed by its FMAs: a round trip is about 60
-        // cycles, far inside the 512-cycle MMA of the next K-block.
+        const uint32_t taddr = tmem_base + lane_addr + buf * TN + c_local0;
+        // 32-column TMEM loads, each followed by its packed FMAs.
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
+        for (int h = 0; h < CPW / 32; ++h) {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + h * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc[h * 32 + j] = fmaf(sc, __uint_as_float(r[j]), acc[h * 32 + j]);
+          tmem_ld_32x32b_x32_sync(taddr + h * 32, r);
+          fma_scaled32(acc + 32 * h, sc, r);
         }
         tc_fence_before();
         __syncwarp();
@@ -275,15 +296,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       const bool whole = (seg.kb0 == 0 && seg.kb1 == s.kb_total);
-      const int col0 = nt * kTileN + c_local0;
+      const int col0 = nt * TN + c_local0;
       if (whole) {
         if (!dead) {
 #pragma unroll
-          for (int h = 0; h < 4; ++h) epi_row32(p.e, row, col0 + 32 * h, *reinterpret_cast<float(*)[32]>(acc + 32 * h));
+          for (int h = 0; h < CPW / 32; ++h)
+            epi_row32(p.e, row, col0 + 32 * h, *reinterpret_cast<float(*)[32]>(acc + 32 * h));
         }
       } else {
         float* my_slot = p.slots + ((static_cast<size_t>(cluster) * 2 + seg.slot) * 2 + rank) * SLOT;
-        if (!dead) slot_store<128>(my_slot, r_local, c_local0, acc);
+        if (!dead) slot_store<CPW>(my_slot, r_local, c_local0, acc);
         const long long t_sk = seg.tile - s.dp_tiles;
         __threadfence();
         named_barrier_sync(1, kPromoThreads);
@@ -302,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c_lo = sk_owner(s, t_sk * s.kb_total);
           const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
 #pragma unroll 1
-          for (int h = 0; h < 4; ++h) {
+          for (int h = 0; h < CPW / 32; ++h) {
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.0f;
@@ -328,15 +350,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 namespace {
-constexpr int kSmem = 1024 + STAGES * STAGE_BYTES + kRing * kSlotFloats * 4 + 8 * (2 * STAGES + 5 + 2 * kRing) + 16;
-static_assert(kSmem <= 232448, "shared memory budget");
-
+template <int TN>
 cudaError_t prepare() {
-  static cudaError_t st =
-      cudaFuncSetAttribute(gemm_fp8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  static cudaError_t st = cudaFuncSetAttribute(gemm_fp8_pair_kernel<TN>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg<TN>::kSmem);
   return st;
 }
 
+template <int TN>
 cudaLaunchConfig_t pair_config(int clusters, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -345,22 +366,22 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t stream, cudaLaunchAttr
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmem;
+  cfg.dynamicSmemBytes = PairCfg<TN>::kSmem;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cfg;
 }
-}  // namespace
 
-int fp8_pair_max_clusters() {
+template <int TN>
+int max_clusters() {
   static int cached = -1;
   if (cached >= 0) return cached;
-  if (prepare() != cudaSuccess) return 0;
+  if (prepare<TN>() != cudaSuccess) return 0;
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_config(1, nullptr, attr);
+  cudaLaunchConfig_t cfg = pair_config<TN>(1, nullptr, attr);
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_fp8_pair_kernel, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_fp8_pair_kernel<TN>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
@@ -368,15 +389,24 @@ int fp8_pair_max_clusters() {
   return n;
 }
 
-cudaError_t launch_gemm_fp8_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Fp8Params& p,
-                                 int clusters, cudaStream_t stream) {
-  cudaError_t e = prepare();
+template <int TN>
+cudaError_t launch(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Fp8Params& p, int clusters,
+                   cudaStream_t stream) {
+  cudaError_t e = prepare<TN>();
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_config(clusters, stream, attr);
-  e = cudaLaunchKernelEx(&cfg, gemm_fp8_pair_kernel, tm_a, tm_b, p);
+  cudaLaunchConfig_t cfg = pair_config<TN>(clusters, stream, attr);
+  e = cudaLaunchKernelEx(&cfg, gemm_fp8_pair_kernel<TN>, tm_a, tm_b, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+}  // namespace
+
+int fp8_pair_max_clusters(int tn) { return tn == 128 ? max_clusters<128>() : max_clusters<256>(); }
+
+cudaError_t launch_gemm_fp8_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Fp8Params& p,
+                                 int clusters, int tn, cudaStream_t stream) {
+  return tn == 128 ? launch<128>(tm_a, tm_b, p, clusters, stream) : launch<256>(tm_a, tm_b, p, clusters, stream);
 }
 
 unsigned take_error_word_fp8_pair() { return take_error_word(); }

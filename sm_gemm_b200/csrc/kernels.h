@@ -62,11 +62,12 @@ cudaError_t launch_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& tm_b, co
                             int grid, cudaStream_t stream);
 constexpr int kFp8BM = 128, kFp8BN = 128, kFp8BK = 128;
 
-// CTA-pair FP8 kernel (256 x 256 per cluster of 2); p.s counts clusters, p.slots is
-// [clusters][2][2 ranks][256][128] floats, p.counters [stream-K tiles][2].
+// CTA-pair FP8 kernel (256 x tn per cluster of 2, tn = 256 or 128); p.s counts
+// clusters, p.slots is [clusters][2][2 ranks][128][tn] floats, p.counters
+// [stream-K tiles][2].
 cudaError_t launch_gemm_fp8_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Fp8Params& p,
-                                 int clusters, cudaStream_t stream);
-int fp8_pair_max_clusters();
+                                 int clusters, int tn, cudaStream_t stream);
+int fp8_pair_max_clusters(int tn);
 
 // C[m, n] = act(bias[n]) (or act(0)) for the K == 0 degenerate GEMM.
 cudaError_t launch_fill_epilogue(int M, int N, const void* bias, int bias_dtype, int act, void* C,

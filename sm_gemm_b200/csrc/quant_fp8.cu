@@ -7,7 +7,8 @@
 // correctly rounded division and the hardware's round-to-nearest-even, saturating
 // conversion (cvt.rn.satfinite.e4m3x2.f32). The result is bit-exact with a plain
 // sequential implementation: the max is order-independent and every other step is
-// a single correctly rounded operation.
+// a single correctly rounded operation (GroupDivider below gives the correctly
+// rounded quotient at a few instructions per element).
 //
 // Plus two small kernels: the K == 0 epilogue fill, and the bounded-wait self-test.
 #include <cuda_fp8.h>
@@ -24,9 +25,49 @@ __device__ __forceinline__ float group_scale(float amax) {
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
 }
 
+// Correctly rounded x / s for every element of a group that shares the scale s.
+// Markstein's FMA division (P. Markstein, "IA-64 and Elementary Functions", 2000,
+// chapter 8; also Muller et al., "Handbook of Floating-Point Arithmetic", the
+// section on division with an FMA): with r = RN(1/s), y = RN(x r) and the residual
+// e = x - y s (exact in one FMA), RN(y + e r) is the correctly rounded quotient
+// provided r is the correctly rounded reciprocal and the significand of s is not
+// all ones. The residual is exact only while x - y s stays out of the subnormal
+// range, which holds for every quotient E4M3 can tell from zero (|x/s| > 2^-11)
+// once s >= 2^-90; smaller quotients become a signed zero code either way, and
+// the sign survives every step. A group whose scale fails a condition (all-ones
+// significand, s < 2^-90, s not finite) divides with __fdiv_rn instead
+// (ExactDiv); the choice is made once per group, outside the element loops.
+__device__ __forceinline__ bool markstein_ok(float s) {
+  const uint32_t b = __float_as_uint(s);
+  const uint32_t ex = (b >> 23) & 0xffu;
+  return ex >= 127u - 90u && ex < 255u && (b & 0x7fffffu) != 0x7fffffu;
+}
+
+struct MarksteinDiv {
+  float s, r;  // r = RN(1 / s)
+  __device__ __forceinline__ float operator()(float x) const {
+    const float y = __fmul_rn(x, r);
+    const float e = __fmaf_rn(-y, s, x);
+    return e == 0.0f ? y : __fmaf_rn(e, r, y);  // e == 0 keeps the sign of a zero x
+  }
+};
+
+struct ExactDiv {
+  float s;
+  __device__ __forceinline__ float operator()(float x) const { return __fdiv_rn(x, s); }
+};
+
+__device__ __forceinline__ MarksteinDiv markstein_div(float s) { return MarksteinDiv{s, __frcp_rn(s)}; }
+
 // Two codes packed little-endian: x0 -> low byte, x1 -> high byte.
 __device__ __forceinline__ uint32_t e4m3x2(float x0, float x1) {
   return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3));
+}
+
+// Four codes of x[0..3] / s, little-endian in one word.
+template <class Div>
+__device__ __forceinline__ uint32_t pack4(const Div& div, const float (&x)[4]) {
+  return e4m3x2(div(x[0]), div(x[1])) | (e4m3x2(div(x[2]), div(x[3])) << 16);
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -48,32 +89,42 @@ __global__ void __launch_bounds__(256) quant_1x128_rows_kernel(const float* __re
   if (g0 >= total) return;
   const int lane = threadIdx.x & 31;
   const bool vec_ld = (ldx & 3) == 0;
+  // (row, group) of each of the warp's groups: one division, then carries.
+  long long gr[kGroupsPerWarp], gk[kGroupsPerWarp];
+  gr[0] = g0 / kbn;
+  gk[0] = g0 - gr[0] * kbn;
+#pragma unroll
+  for (int i = 1; i < kGroupsPerWarp; ++i) {
+    gr[i] = gr[i - 1];
+    gk[i] = gk[i - 1] + 1;
+    if (gk[i] == kbn) {
+      gk[i] = 0;
+      ++gr[i];
+    }
+  }
   float v[kGroupsPerWarp][4];
 #pragma unroll
   for (int i = 0; i < kGroupsPerWarp; ++i) {
-    const long long g = g0 + i;
-    const long long r = g / kbn, kb = g - r * kbn;
-    const long long c0 = kb * 128 + lane * 4;
-    const float* src = X + r * ldx;
-    if (g < total && vec_ld && kb * 128 + 128 <= cols) {
+    const bool live = g0 + i < total;
+    const long long c0 = gk[i] * 128 + lane * 4;
+    const float* src = X + gr[i] * ldx;
+    if (live && vec_ld && gk[i] * 128 + 128 <= cols) {
       const float4 t = __ldcs(reinterpret_cast<const float4*>(src + c0));
       v[i][0] = t.x; v[i][1] = t.y; v[i][2] = t.z; v[i][3] = t.w;
     } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[i][j] = (g < total && c0 + j < cols) ? src[c0 + j] : 0.0f;
+      for (int j = 0; j < 4; ++j) v[i][j] = (live && c0 + j < cols) ? src[c0 + j] : 0.0f;
     }
   }
 #pragma unroll
   for (int i = 0; i < kGroupsPerWarp; ++i) {
-    const long long g = g0 + i;
-    if (g >= total) break;
-    const long long r = g / kbn, kb = g - r * kbn;
+    if (g0 + i >= total) break;
+    const long long r = gr[i], kb = gk[i];
     const long long c0 = kb * 128 + lane * 4;
     float amax = fmaxf(fmaxf(fabsf(v[i][0]), fabsf(v[i][1])), fmaxf(fabsf(v[i][2]), fabsf(v[i][3])));
     amax = warp_max(amax);
     const float sc = group_scale(amax);
-    const uint32_t w = e4m3x2(__fdiv_rn(v[i][0], sc), __fdiv_rn(v[i][1], sc)) |
-                       (e4m3x2(__fdiv_rn(v[i][2], sc), __fdiv_rn(v[i][3], sc)) << 16);
+    const uint32_t w = markstein_ok(sc) ? pack4(markstein_div(sc), v[i]) : pack4(ExactDiv{sc}, v[i]);
     uint8_t* dst = Q + r * cols + c0;
     if (kb * 128 + 128 <= cols && (cols & 3) == 0) {
       *reinterpret_cast<uint32_t*>(dst) = w;
@@ -83,6 +134,19 @@ __global__ void __launch_bounds__(256) quant_1x128_rows_kernel(const float* __re
         if (c0 + j < cols) dst[j] = static_cast<uint8_t>(w >> (8 * j));
     }
     if (lane == 0) S[kb * rows + r] = sc;
+  }
+}
+
+// Codes of one row's group [c0, c1) of a column-major X, two columns at a time.
+template <class Div>
+__device__ __forceinline__ void quant_col_group(const Div& div, const float* __restrict__ X, long long ldx,
+                                                long long r, long long c0, long long c1, uint8_t* dst) {
+  for (long long c = c0; c < c1; c += 2) {
+    const float x0 = X[c * ldx + r];
+    const float x1 = (c + 1 < c1) ? X[(c + 1) * ldx + r] : 0.0f;
+    const uint32_t w = e4m3x2(div(x0), div(x1));
+    dst[c] = static_cast<uint8_t>(w);
+    if (c + 1 < c1) dst[c + 1] = static_cast<uint8_t>(w >> 8);
   }
 }
 
@@ -101,13 +165,8 @@ __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(const float* __re
   for (long long c = c0; c < c1; ++c) amax = fmaxf(amax, fabsf(X[c * ldx + r]));
   const float s = group_scale(amax);
   uint8_t* dst = Q + r * cols;
-  for (long long c = c0; c < c1; c += 2) {
-    const float x0 = X[c * ldx + r];
-    const float x1 = (c + 1 < c1) ? X[(c + 1) * ldx + r] : 0.0f;
-    const uint32_t w = e4m3x2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
-    dst[c] = static_cast<uint8_t>(w);
-    if (c + 1 < c1) dst[c + 1] = static_cast<uint8_t>(w >> 8);
-  }
+  if (markstein_ok(s)) quant_col_group(markstein_div(s), X, ldx, r, c0, c1, dst);
+  else quant_col_group(ExactDiv{s}, X, ldx, r, c0, c1, dst);
   S[kb * rows + r] = s;
 }
 
@@ -119,6 +178,31 @@ __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(const float* __re
 // so both the transposing stores of phase 1 and the row reads of phase 2 are free of
 // bank conflicts.
 __device__ __forceinline__ int qswz(int n) { return ((n >> 2) ^ ((n & 3) << 3)) & 31; }
+
+// Phase 2 of quant_128x128_kernel: codes of k in [kh, kh + 64) of one staged row,
+// written as four 16-byte chunks (bytewise for the last K-block when K % 16 != 0
+// or the block is ragged; kvalid = the number of valid k from kh on).
+template <class Div>
+__device__ __forceinline__ void encode_half_row(const Div& div, const float* row, int g, int kh, uint8_t* dst,
+                                                bool vec, int kvalid) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const int kk = kh + u * 16 + h * 4;
+      const float x[4] = {row[(kk + 0) ^ g], row[(kk + 1) ^ g], row[(kk + 2) ^ g], row[(kk + 3) ^ g]};
+      w[h] = pack4(div, x);
+    }
+    if (vec) {
+      *reinterpret_cast<uint4*>(dst + u * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (u * 16 + j < kvalid) dst[u * 16 + j] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
+    }
+  }
+}
 
 __global__ void __launch_bounds__(256) quant_128x128_kernel(const float* __restrict__ X, long long K, long long N,
                                                             long long rs, long long cs, uint8_t* __restrict__ Q,
@@ -201,28 +285,12 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(const float* __restr
   const int kh = 64 * (t >> 7);
   const long long n = n0 + nn;
   if (n >= N) return;
-  const int g = qswz(nn);
+  const float* row = tile + nn * 128;
   uint8_t* dst = Q + n * K + k0 + kh;
   const bool vec = (k0 + kh + 64 <= K) && ((K & 15) == 0);
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    uint32_t w[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const int kk = kh + u * 16 + h * 4;
-      const float* row = tile + nn * 128;
-      const uint32_t lo = e4m3x2(__fdiv_rn(row[(kk + 0) ^ g], sc), __fdiv_rn(row[(kk + 1) ^ g], sc));
-      const uint32_t hi = e4m3x2(__fdiv_rn(row[(kk + 2) ^ g], sc), __fdiv_rn(row[(kk + 3) ^ g], sc));
-      w[h] = lo | (hi << 16);
-    }
-    if (vec) {
-      *reinterpret_cast<uint4*>(dst + u * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (k0 + kh + u * 16 + j < K) dst[u * 16 + j] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
-    }
-  }
+  const int kvalid = static_cast<int>(K - k0 - kh);
+  if (markstein_ok(sc)) encode_half_row(markstein_div(sc), row, qswz(nn), kh, dst, vec, kvalid);
+  else encode_half_row(ExactDiv{sc}, row, qswz(nn), kh, dst, vec, kvalid);
 }
 
 __global__ void fill_epilogue_kernel(int M, int N, const void* bias, int bias_dtype, int act, void* C,

@@ -1,0 +1,55 @@
+"""Multi-rank plumbing of bench.py on CPU: two gloo ranks (the GPU runs use one
+process per GPU over NCCL with the same calls). Each rank times its own replica of
+the workload; the job's time is the slowest rank's, and the whole-job throughput
+counts every rank's steps."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
+    try:
+        # Rank r reports (r + 1) * 3 ms: the job time is the largest, 3 * world ms.
+        ms = bench.max_over_ranks(3.0 * (rank + 1), dist)
+        out[rank] = (ms, bench.whole_job_tflops(2e12, 10, world, ms))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2])
+def test_max_over_ranks_and_aggregate(world):
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_rank_main, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(60)
+        assert all(p.exitcode == 0 for p in procs)
+        res = dict(out)
+    assert sorted(res) == list(range(world))
+    for ms, tf in res.values():
+        assert ms == 3.0 * world
+        # world replicas x 10 steps x 2e12 FLOP in 6 ms
+        assert tf == pytest.approx(2e12 * 10 * world / 6e-3 / 1e12)
+
+
+def test_single_process_passthrough():
+    assert bench.max_over_ranks(1.25, None) == 1.25
+    assert bench.whole_job_tflops(1e12, 4, 1, 2.0) == pytest.approx(2000.0)

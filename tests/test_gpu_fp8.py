@@ -72,6 +72,70 @@ def test_quant_special_values(cuda_device):
         assert np.array_equal(Q, Qr)
 
 
+def _scale_hitting(target: np.float32):
+    """An amax whose group scale RN(amax / 448) is exactly `target`, or None."""
+    a = np.float32(target * np.float32(448.0))
+    for _ in range(16):
+        s = np.float32(a / np.float32(448.0))
+        if s == target:
+            return a
+        a = np.nextafter(a, np.float32(np.inf) if s < target else np.float32(0.0), dtype=np.float32)
+    return None
+
+
+def _edge_scales():
+    """Scales that stress the division by the group scale: significands of all ones
+    (where a reciprocal-based quotient needs special care), powers of two, scales
+    near 2^-90 and near the largest finite amax, and ordinary random ones."""
+    f = np.float32
+    out = []
+    for e in (-120, -95, -91, -90, -89, -60, -20, -7, -1, 0, 1, 7, 40, 110, 119):
+        out += [f(2.0 ** e), f(np.nextafter(f(2.0 ** (e + 1)), f(0))),   # 1.0 and all-ones significands
+                f(1.5 * 2.0 ** e), f(np.nextafter(f(2.0 ** e), f(np.inf)))]
+    rng = np.random.default_rng(5)
+    out += list((rng.uniform(1, 2, 24) * 2.0 ** rng.integers(-40, 40, 24)).astype(np.float32))
+    with np.errstate(over="ignore"):
+        return [s for s in out if np.isfinite(s) and np.isfinite(f(s * f(448.0)))]
+
+
+def _tie_group(amax: np.float32, s: np.float32, n: int, rng) -> np.ndarray:
+    """n values whose quotients by s sit on and next to the E4M3 rounding midpoints
+    (where one ulp of the FP32 quotient decides the code), plus +-amax."""
+    vals = oracle.e4m3_decode(np.arange(0, 127, dtype=np.uint8)).astype(np.float64)
+    mids = (vals[:-1] + vals[1:]) / 2.0
+    m = rng.choice(mids, n)
+    x = (m * np.float64(s)).astype(np.float32)
+    step = rng.integers(-1, 2, n)
+    x = np.where(step > 0, np.nextafter(x, np.float32(np.inf)), np.where(step < 0, np.nextafter(x, np.float32(0)), x))
+    x = np.minimum(np.abs(x), amax).astype(np.float32) * rng.choice(np.float32([-1, 1]), n)
+    x[0], x[1] = amax, -amax
+    return x.astype(np.float32)
+
+
+def test_quant_division_edge_scales(cuda_device):
+    """Bit-exact codes for groups whose scales stress the quotient x / s: elements on
+    and one FP32 ulp beside the E4M3 rounding midpoints, under each edge scale."""
+    rng = np.random.default_rng(11)
+    groups, blocks = [], []
+    for s in _edge_scales():
+        amax = _scale_hitting(s)
+        if amax is None:
+            continue
+        groups.append(_tie_group(amax, s, 128, rng))
+        blocks.append(_tie_group(amax, s, 128 * 128, rng).reshape(128, 128))
+    assert len(groups) >= 60
+    X1 = np.stack(groups)
+    Q, S = _gpu_quant(X1, 1)
+    Qr, Sr = oracle.quant_1x128(X1)
+    assert np.array_equal(S.view(np.uint32), Sr.view(np.uint32))
+    assert np.array_equal(Q, Qr)
+    X2 = np.concatenate(blocks, axis=1)  # [K = 128, N = 128 * blocks]
+    Q, S = _gpu_quant(X2, 128)
+    Qr, Sr = oracle.quant_128x128(X2)
+    assert np.array_equal(S.view(np.uint32), Sr.view(np.uint32))
+    assert np.array_equal(Q, Qr)
+
+
 def _quantised_problem(M, N, K, seed):
     A = synth.normal_with_outliers(seed, 0, (M, K))
     B = synth.normal_with_outliers(seed, 1, (K, N))
