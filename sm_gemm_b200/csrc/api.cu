@@ -159,7 +159,8 @@ Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, siz
 // ------------------------------------------------------------------ TMA maps
 
 bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   PFN_encodeTiled fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
@@ -167,7 +168,7 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint6
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -452,10 +453,18 @@ smgemm_status quantize_fp8_blockwise(const float* X, int64_t rows, int64_t cols,
     return SMGEMM_ERR_ALIGNMENT;
   DevInfo d;
   if (current_device(d) != SMGEMM_OK) return SMGEMM_ERR_CUDA;
-  const long long rs = layout_x == SMGEMM_ROW_MAJOR ? ldx : 1;
-  const long long cs = layout_x == SMGEMM_ROW_MAJOR ? 1 : ldx;
-  cudaError_t e = group_rows == 1 ? launch_quant_1x128(X, rows, cols, rs, cs, Q, scales, stream)
-                                  : launch_quant_128x128(X, rows, cols, rs, cs, Q, scales, stream);
+  const bool row_major = layout_x == SMGEMM_ROW_MAJOR;
+  if (group_rows == 1 && !row_major)
+    return launch_status(launch_quant_1x128_cols(X, rows, cols, ldx, Q, scales, stream));
+  // Row-major: [rows][cols]; column-major: [cols][rows] (for 128x128, rows = K, cols = N).
+  CUtensorMap tm;
+  const uint64_t inner = row_major ? cols : rows, outer = row_major ? rows : cols;
+  if (!encode_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, X, inner, outer, static_cast<uint64_t>(ldx) * 4, 128,
+                 group_rows == 1 ? 32 : 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SMGEMM_ERR_CUDA;
+  cudaError_t e = group_rows == 1
+                      ? launch_quant_1x128_tma(tm, rows, cols, Q, scales, d.sms, wait_limit(), stream)
+                      : launch_quant_128x128_tma(tm, row_major, rows, cols, Q, scales, d.sms, wait_limit(), stream);
   return launch_status(e);
 }
 

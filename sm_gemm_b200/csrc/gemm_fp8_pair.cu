@@ -47,7 +47,10 @@ constexpr int A_BYTES = 128 * BKB;       // this CTA's 128 rows of A
 constexpr int TCOLS = 512;               // all of TMEM: 512 / TN partial buffers
 constexpr int kRing = 8;                 // scale ring slots
 constexpr int kSlotFloats = 132;         // 128 row scales + up to 2 block scales, padded to 16 B
-constexpr int kRoleRegs = 40, kPromoRegs = 232;  // setmaxnreg split (384 x 168 at launch)
+// setmaxnreg split: 128 x 40 + 256 x 232 = 64512 registers, all of the 384 x 168 the
+// block launches with (prepare() checks the compiled count before any launch).
+constexpr int kRoleRegs = 40, kPromoRegs = 232;
+static_assert(128 * kRoleRegs + kPromoThreads * kPromoRegs <= kThreads * 168, "register split");
 
 // Per-tile-width constants: this CTA's B rows (TN / 2), stage size, pipeline depth and
 // the number of TMEM partial buffers.
@@ -350,10 +353,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 namespace {
+// Sets the shared-memory limit and checks that the registers the kernel launches with
+// cover the setmaxnreg split (otherwise the promotion warps' increase would never be
+// granted); a build that breaks the split fails here instead of launching.
+template <int TN>
+cudaError_t prepare_once() {
+  cudaError_t e = cudaFuncSetAttribute(gemm_fp8_pair_kernel<TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       PairCfg<TN>::kSmem);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes attr{};
+  e = cudaFuncGetAttributes(&attr, gemm_fp8_pair_kernel<TN>);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs * kThreads < 128 * kRoleRegs + kPromoThreads * kPromoRegs) return cudaErrorInvalidConfiguration;
+  return cudaSuccess;
+}
+
 template <int TN>
 cudaError_t prepare() {
-  static cudaError_t st = cudaFuncSetAttribute(gemm_fp8_pair_kernel<TN>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg<TN>::kSmem);
+  static cudaError_t st = prepare_once<TN>();
   return st;
 }
 

@@ -73,10 +73,15 @@ int fp8_pair_max_clusters(int tn);
 cudaError_t launch_fill_epilogue(int M, int N, const void* bias, int bias_dtype, int act, void* C,
                                  int c_dtype, long long ldc, cudaStream_t stream);
 
-cudaError_t launch_quant_1x128(const float* X, long long rows, long long cols, long long rs,
-                               long long cs, uint8_t* Q, float* S, cudaStream_t stream);
-cudaError_t launch_quant_128x128(const float* X, long long K, long long N, long long rs,
-                                 long long cs, uint8_t* Q, float* S, cudaStream_t stream);
+// FP8 quantisers. Row-major 1x128 and both 128x128 layouts take a 2-D FLOAT32 tensor map
+// without swizzle: 1x128 box {128 columns, 32 rows} over [rows][cols]; 128x128 box
+// {128, 128} over [K][N] (n_contig) or [N][K]. Column-major 1x128 takes X itself.
+cudaError_t launch_quant_1x128_tma(const CUtensorMap& tm_x, long long rows, long long cols, uint8_t* Q, float* S,
+                                   int sms, unsigned long long limit, cudaStream_t stream);
+cudaError_t launch_quant_1x128_cols(const float* X, long long rows, long long cols, long long ldx, uint8_t* Q,
+                                    float* S, cudaStream_t stream);
+cudaError_t launch_quant_128x128_tma(const CUtensorMap& tm_x, bool n_contig, long long K, long long N, uint8_t* Q,
+                                     float* S, int sms, unsigned long long limit, cudaStream_t stream);
 
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
 

@@ -7,8 +7,13 @@
 // correctly rounded division and the hardware's round-to-nearest-even, saturating
 // conversion (cvt.rn.satfinite.e4m3x2.f32). The result is bit-exact with a plain
 // sequential implementation: the max is order-independent and every other step is
-// a single correctly rounded operation (GroupDivider below gives the correctly
+// a single correctly rounded operation (MarksteinDiv below gives the correctly
 // rounded quotient at a few instructions per element).
+//
+// Both row-major group shapes are fed by TMA: a persistent CTA streams fp32 tiles
+// through a shared-memory ring (one producer thread, eight encoding warps), so HBM
+// sees a few hundred KB in flight per SM while the warps encode. Column-major 1x128
+// input (rows contiguous) uses a plain per-thread kernel.
 //
 // Plus two small kernels: the K == 0 epilogue fill, and the bounded-wait self-test.
 #include <cuda_fp8.h>
@@ -45,10 +50,23 @@ __device__ __forceinline__ bool markstein_ok(float s) {
 
 struct MarksteinDiv {
   float s, r;  // r = RN(1 / s)
+  // The residual step with e == 0 returns y + 0, which is +0 for x = -0: the sign of x
+  // is ORed back in (a no-op for every other x, whose quotient already carries it).
   __device__ __forceinline__ float operator()(float x) const {
     const float y = __fmul_rn(x, r);
     const float e = __fmaf_rn(-y, s, x);
-    return e == 0.0f ? y : __fmaf_rn(e, r, y);  // e == 0 keeps the sign of a zero x
+    const float q = __fmaf_rn(e, r, y);
+    return __uint_as_float(__float_as_uint(q) | (__float_as_uint(x) & 0x80000000u));
+  }
+  // Two quotients with packed FP32x2 arithmetic (mul/fma.rn.f32x2; each half is
+  // rounded exactly like the scalar operation).
+  __device__ __forceinline__ float2 div2(float2 x) const {
+    const float2 s2 = make_float2(s, s), r2 = make_float2(r, r);
+    const float2 y = __fmul2_rn(x, r2);
+    const float2 e = __ffma2_rn(make_float2(-y.x, -y.y), s2, x);
+    const float2 q = __ffma2_rn(e, r2, y);
+    return make_float2(__uint_as_float(__float_as_uint(q.x) | (__float_as_uint(x.x) & 0x80000000u)),
+                       __uint_as_float(__float_as_uint(q.y) | (__float_as_uint(x.y) & 0x80000000u)));
   }
 };
 
@@ -65,8 +83,13 @@ __device__ __forceinline__ uint32_t e4m3x2(float x0, float x1) {
 }
 
 // Four codes of x[0..3] / s, little-endian in one word.
-template <class Div>
-__device__ __forceinline__ uint32_t pack4(const Div& div, const float (&x)[4]) {
+__device__ __forceinline__ uint32_t pack4(const MarksteinDiv& div, const float (&x)[4]) {
+  const float2 a = div.div2(make_float2(x[0], x[1]));
+  const float2 b = div.div2(make_float2(x[2], x[3]));
+  return e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack4(const ExactDiv& div, const float (&x)[4]) {
   return e4m3x2(div(x[0]), div(x[1])) | (e4m3x2(div(x[2]), div(x[3])) << 16);
 }
 
@@ -74,67 +97,6 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
-}
-
-// Row-major X (element (r, c) at r*ldx + c): each warp quantises kGroupsPerWarp
-// consecutive 1x128 groups; every lane issues all of its 16-byte loads before using
-// any, so enough bytes are in flight to keep HBM busy.
-constexpr int kGroupsPerWarp = 4;
-__global__ void __launch_bounds__(256) quant_1x128_rows_kernel(const float* __restrict__ X, long long rows,
-                                                               long long cols, long long ldx,
-                                                               uint8_t* __restrict__ Q, float* __restrict__ S) {
-  const long long kbn = (cols + 127) / 128;
-  const long long total = rows * kbn;
-  const long long g0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kGroupsPerWarp;
-  if (g0 >= total) return;
-  const int lane = threadIdx.x & 31;
-  const bool vec_ld = (ldx & 3) == 0;
-  // (row, group) of each of the warp's groups: one division, then carries.
-  long long gr[kGroupsPerWarp], gk[kGroupsPerWarp];
-  gr[0] = g0 / kbn;
-  gk[0] = g0 - gr[0] * kbn;
-#pragma unroll
-  for (int i = 1; i < kGroupsPerWarp; ++i) {
-    gr[i] = gr[i - 1];
-    gk[i] = gk[i - 1] + 1;
-    if (gk[i] == kbn) {
-      gk[i] = 0;
-      ++gr[i];
-    }
-  }
-  float v[kGroupsPerWarp][4];
-#pragma unroll
-  for (int i = 0; i < kGroupsPerWarp; ++i) {
-    const bool live = g0 + i < total;
-    const long long c0 = gk[i] * 128 + lane * 4;
-    const float* src = X + gr[i] * ldx;
-    if (live && vec_ld && gk[i] * 128 + 128 <= cols) {
-      const float4 t = __ldcs(reinterpret_cast<const float4*>(src + c0));
-      v[i][0] = t.x; v[i][1] = t.y; v[i][2] = t.z; v[i][3] = t.w;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v[i][j] = (live && c0 + j < cols) ? src[c0 + j] : 0.0f;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kGroupsPerWarp; ++i) {
-    if (g0 + i >= total) break;
-    const long long r = gr[i], kb = gk[i];
-    const long long c0 = kb * 128 + lane * 4;
-    float amax = fmaxf(fmaxf(fabsf(v[i][0]), fabsf(v[i][1])), fmaxf(fabsf(v[i][2]), fabsf(v[i][3])));
-    amax = warp_max(amax);
-    const float sc = group_scale(amax);
-    const uint32_t w = markstein_ok(sc) ? pack4(markstein_div(sc), v[i]) : pack4(ExactDiv{sc}, v[i]);
-    uint8_t* dst = Q + r * cols + c0;
-    if (kb * 128 + 128 <= cols && (cols & 3) == 0) {
-      *reinterpret_cast<uint32_t*>(dst) = w;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (c0 + j < cols) dst[j] = static_cast<uint8_t>(w >> (8 * j));
-    }
-    if (lane == 0) S[kb * rows + r] = sc;
-  }
 }
 
 // Codes of one row's group [c0, c1) of a column-major X, two columns at a time.
@@ -170,127 +132,288 @@ __global__ void __launch_bounds__(256) quant_1x128_cols_kernel(const float* __re
   S[kb * rows + r] = s;
 }
 
-// One CTA per 128x128 block of the weight X[K, N] (element (k, n) at k*rs + n*cs).
-// Phase 1 loads the block with 16-byte loads (16 per thread, all issued before use)
-// and stages it transposed in shared memory as [n][k]; phase 2 has each thread encode
-// 64 consecutive k of one n and write them as 16-byte rows of Q[n][k]. The shared tile
-// is XOR-swizzled (column k of row n stored at k ^ g(n), g(n) = ((n >> 2) ^ ((n & 3) << 3)) & 31)
-// so both the transposing stores of phase 1 and the row reads of phase 2 are free of
-// bank conflicts.
-__device__ __forceinline__ int qswz(int n) { return ((n >> 2) ^ ((n & 3) << 3)) & 31; }
-
-// Phase 2 of quant_128x128_kernel: codes of k in [kh, kh + 64) of one staged row,
-// written as four 16-byte chunks (bytewise for the last K-block when K % 16 != 0
-// or the block is ragged; kvalid = the number of valid k from kh on).
+// 16 codes of one lane's elements v[j][e] (group columns c0 + 32j + e) into dst (the
+// code of column c0); bytewise with bounds when the group is ragged or cols % 4 != 0.
 template <class Div>
-__device__ __forceinline__ void encode_half_row(const Div& div, const float* row, int g, int kh, uint8_t* dst,
-                                                bool vec, int kvalid) {
+__device__ __forceinline__ void store_codes16(const Div& div, const float (&v)[4][4], uint8_t* dst, long long c0,
+                                              long long cols, bool vec) {
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    uint32_t w[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const int kk = kh + u * 16 + h * 4;
-      const float x[4] = {row[(kk + 0) ^ g], row[(kk + 1) ^ g], row[(kk + 2) ^ g], row[(kk + 3) ^ g]};
-      w[h] = pack4(div, x);
-    }
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t w = pack4(div, v[j]);
     if (vec) {
-      *reinterpret_cast<uint4*>(dst + u * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint32_t*>(dst + 32 * j) = w;
     } else {
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (u * 16 + j < kvalid) dst[u * 16 + j] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
+      for (int e = 0; e < 4; ++e)
+        if (c0 + 32 * j + e < cols) dst[32 * j + e] = static_cast<uint8_t>(w >> (8 * e));
     }
   }
 }
 
-__global__ void __launch_bounds__(256) quant_128x128_kernel(const float* __restrict__ X, long long K, long long N,
-                                                            long long rs, long long cs, uint8_t* __restrict__ Q,
-                                                            float* __restrict__ S) {
-  extern __shared__ float tile[];  // [128 n][128 k], swizzled
-  __shared__ float warp_amax[8];
-  const long long kb = blockIdx.y, nb = blockIdx.x;
-  const long long k0 = kb * 128, n0 = nb * 128;
-  const long long nbn = (N + 127) / 128;
-  const int t = threadIdx.x;
-  float amax = 0.0f;
-  if (cs == 1) {
-    // N contiguous: float4 = 4 consecutive n of one k. idx -> (kk = idx / 32, n4 = idx % 32).
-    const bool vec = (rs & 3) == 0 && n0 + 128 <= N;
-    float4 r4[16];
+// Pass 2 of quant_128x128_tma_kernel (see there) for block (kb, nb).
+template <bool kNContig, class Div>
+__device__ __forceinline__ void encode_block(const Div& div, const float* tile, int ptid, long long kb, long long nb,
+                                             long long K, long long N, uint8_t* __restrict__ Q) {
+  const long long k0 = kb * 128;
+  if (kNContig) {
+    const int n = ptid & 127, kh = (ptid >> 7) * 64;
+    const long long ng = nb * 128 + n;
+    if (ng >= N) return;
+    uint8_t* dst = Q + ng * K + k0 + kh;
+    const bool vec = (K & 15) == 0 && k0 + kh + 64 <= K;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int idx = i * 256 + t, kk = idx >> 5, n4 = idx & 31;
-      const long long k = k0 + kk, n = n0 + 4 * n4;
-      if (k < K && vec) {
-        r4[i] = __ldcs(reinterpret_cast<const float4*>(X + k * rs + n));
-      } else {
-        float e[4];
+    for (int u = 0; u < 4; ++u) {
+      uint32_t w[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) e[q] = (k < K && n + q < N) ? X[k * rs + n + q] : 0.0f;
-        r4[i] = make_float4(e[0], e[1], e[2], e[3]);
+      for (int h = 0; h < 4; ++h) {
+        const int k = kh + 16 * u + 4 * h;
+        const float x[4] = {tile[k * 128 + n], tile[(k + 1) * 128 + n], tile[(k + 2) * 128 + n],
+                            tile[(k + 3) * 128 + n]};
+        w[h] = pack4(div, x);
       }
-    }
+      if (vec) {
+        *reinterpret_cast<uint4*>(dst + 16 * u) = make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int idx = i * 256 + t, kk = idx >> 5, n4 = idx & 31;
-      const float e[4] = {r4[i].x, r4[i].y, r4[i].z, r4[i].w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int n = 4 * n4 + q;
-        amax = fmaxf(amax, fabsf(e[q]));
-        tile[n * 128 + (kk ^ qswz(n))] = e[q];
+        for (int j = 0; j < 16; ++j)
+          if (k0 + kh + 16 * u + j < K) dst[16 * u + j] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
       }
     }
   } else {
-    // K contiguous (rs == 1) or general strides: float4 = 4 consecutive k of one n when
-    // possible. idx -> (n = idx / 32, k4 = idx % 32).
-    const bool vec = rs == 1 && (cs & 3) == 0 && k0 + 128 <= K;
-    float4 r4[16];
-#pragma unroll
+    const int warp = ptid >> 5, lane = ptid & 31;
+    const long long kg = k0 + 4 * lane;
+    const bool vec = (K & 3) == 0 && kg + 4 <= K;
+#pragma unroll 4
     for (int i = 0; i < 16; ++i) {
-      const int idx = i * 256 + t, nn = idx >> 5, k4 = idx & 31;
-      const long long n = n0 + nn, k = k0 + 4 * k4;
-      if (n < N && vec) {
-        r4[i] = __ldcs(reinterpret_cast<const float4*>(X + n * cs + k));
+      const int n = warp * 16 + i;
+      const long long ng = nb * 128 + n;
+      if (ng >= N) break;
+      const float4 t4 = reinterpret_cast<const float4*>(tile + n * 128)[lane];
+      const float x[4] = {t4.x, t4.y, t4.z, t4.w};
+      const uint32_t w = pack4(div, x);
+      uint8_t* dst = Q + ng * K + kg;
+      if (vec) {
+        *reinterpret_cast<uint32_t*>(dst) = w;
       } else {
-        float e[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) e[q] = (n < N && k + q < K) ? X[(k + q) * rs + n * cs] : 0.0f;
-        r4[i] = make_float4(e[0], e[1], e[2], e[3]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int idx = i * 256 + t, nn = idx >> 5, k4 = idx & 31;
-      const float e[4] = {r4[i].x, r4[i].y, r4[i].z, r4[i].w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        amax = fmaxf(amax, fabsf(e[q]));
-        tile[nn * 128 + ((4 * k4 + q) ^ qswz(nn))] = e[q];
+        for (int e = 0; e < 4; ++e)
+          if (kg + e < K) dst[e] = static_cast<uint8_t>(w >> (8 * e));
       }
     }
   }
-  amax = warp_max(amax);
-  if ((t & 31) == 0) warp_amax[t >> 5] = amax;
-  __syncthreads();
-  float m = warp_amax[0];
-#pragma unroll
-  for (int w = 1; w < 8; ++w) m = fmaxf(m, warp_amax[w]);
-  const float sc = group_scale(m);
-  if (t == 0) S[kb * nbn + nb] = sc;
+}
 
-  // Phase 2: warp w, lane l -> row n = 32*(w & 3) + l, k in [64*(w >> 2), +64).
-  const int nn = 32 * ((t >> 5) & 3) + (t & 31);
-  const int kh = 64 * (t >> 7);
-  const long long n = n0 + nn;
-  if (n >= N) return;
-  const float* row = tile + nn * 128;
-  uint8_t* dst = Q + n * K + k0 + kh;
-  const bool vec = (k0 + kh + 64 <= K) && ((K & 15) == 0);
-  const int kvalid = static_cast<int>(K - k0 - kh);
-  if (markstein_ok(sc)) encode_half_row(markstein_div(sc), row, qswz(nn), kh, dst, vec, kvalid);
-  else encode_half_row(ExactDiv{sc}, row, qswz(nn), kh, dst, vec, kvalid);
+// ---------------------------------------------------------------- TMA-fed quantisers
+//
+// Shared structure: warp 8 is the producer (lane 0 issues one 2-D TMA load per tile into
+// the next ring stage, completing on full[stage]); warps 0-7 read the stage, release it
+// on empty[stage] (8 arrivals) and encode. All waits are bounded (abort flag + limit).
+constexpr int kQConsumers = 8;
+constexpr int kQThreads = (kQConsumers + 1) * 32;
+
+struct QRing {
+  uint32_t base;      // shared address of stage 0 (1024-byte aligned)
+  const uint8_t* gen; // generic address of stage 0
+  uint32_t bars;      // full[0..S), empty[0..S)
+  volatile int* abort_flag;
+};
+
+template <int kStages, int kTileBytes>
+__device__ __forceinline__ QRing q_ring_setup(uint8_t* smem_raw) {
+  QRing q;
+  q.base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  q.gen = smem_raw + (q.base - smem_u32(smem_raw));
+  q.bars = q.base + kStages * kTileBytes;
+  q.abort_flag = reinterpret_cast<volatile int*>(const_cast<uint8_t*>(q.gen) + kStages * kTileBytes + 16 * kStages);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(q.bars + 8u * i, 1);
+      mbar_init(q.bars + 8u * (kStages + i), kQConsumers);
+    }
+    *q.abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  return q;
+}
+
+// Producer loop: tile i of this CTA is tile blockIdx.x + i * gridDim.x; coords(t, x, y)
+// gives its TMA box origin. After an abort it waits (bounded) for the loads in flight.
+template <int kStages, int kTileBytes, class Coords>
+__device__ __forceinline__ void q_produce(const QRing& q, const CUtensorMap* tm, long long T, Coords coords,
+                                          unsigned long long limit) {
+  tma_prefetch_desc(tm);
+  int stage = 0;
+  uint32_t phase = 0;
+  long long issued = 0;
+  for (long long t = blockIdx.x; t < T; t += gridDim.x) {
+    if (!mbar_wait(q.bars + 8u * (kStages + stage), phase ^ 1u, q.abort_flag, limit)) break;
+    int x, y;
+    coords(t, x, y);
+    mbar_arrive_expect_tx(q.bars + 8u * stage, kTileBytes);
+    tma_load_2d(q.base + stage * kTileBytes, tm, q.bars + 8u * stage, x, y);
+    ++issued;
+    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+  }
+  if (*q.abort_flag) {
+    volatile int no_abort = 0;
+    for (long long i = 0; i < issued && i < kStages; ++i) {
+      if (--stage < 0) { stage = kStages - 1; phase ^= 1u; }
+      mbar_wait(q.bars + 8u * stage, phase, &no_abort, limit);
+    }
+  }
+}
+
+// 1x128 groups of a row-major X[rows][cols]: one tile = 32 rows x 128 columns (16 KB, one
+// group per row). Warp w encodes rows 4w..4w+3 of the tile, eight lanes per row: lane l
+// reads the float4s at columns 32j + 4(l % 8), j < 4 (each quarter-warp reads 128
+// contiguous bytes, free of bank conflicts), reduces the row's amax in three shuffle
+// steps, releases the stage, then encodes and stores its 16 codes.
+constexpr int kQ1Rows = 32;
+constexpr int kQ1TileBytes = kQ1Rows * 128 * 4;
+constexpr int kQ1Stages = 4;
+constexpr int kQ1Smem = 1024 + kQ1Stages * kQ1TileBytes + 16 * kQ1Stages + 16;
+
+__global__ void __launch_bounds__(kQThreads) quant_1x128_tma_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                                     long long rows, long long cols,
+                                                                     uint8_t* __restrict__ Q, float* __restrict__ S,
+                                                                     unsigned long long limit) {
+  extern __shared__ uint8_t smem_raw[];
+  const QRing q = q_ring_setup<kQ1Stages, kQ1TileBytes>(smem_raw);
+  const long long kbn = (cols + 127) / 128;
+  const long long T = (rows + kQ1Rows - 1) / kQ1Rows * kbn;
+  const int warp = static_cast<int>(warp_id()), lane = static_cast<int>(lane_id());
+  if (warp == kQConsumers) {
+    if (lane == 0)
+      q_produce<kQ1Stages, kQ1TileBytes>(q, &tm_x, T, [&](long long t, int& x, int& y) {
+        const long long rt = t / kbn;
+        x = static_cast<int>((t - rt * kbn) * 128);
+        y = static_cast<int>(rt * kQ1Rows);
+      }, limit);
+    return;
+  }
+  const int gi = lane >> 3, sub = lane & 7;
+  const int trow = warp * 4 + gi;
+  const bool vec_st = (cols & 3) == 0;
+  // (row tile, group) of this CTA's current tile, advanced by gridDim.x tiles per step.
+  long long rt = blockIdx.x / kbn, kb = blockIdx.x - (blockIdx.x / kbn) * kbn;
+  const long long step_rt = gridDim.x / kbn, step_kb = gridDim.x - step_rt * kbn;
+  int stage = 0;
+  uint32_t phase = 0;
+  bool dead = false;
+  for (long long t = blockIdx.x; t < T; t += gridDim.x) {
+    if (!dead) dead = !mbar_wait(q.bars + 8u * stage, phase, q.abort_flag, limit);
+    dead = __any_sync(0xffffffffu, dead);
+    float v[4][4];
+    if (!dead) {
+      const float* src = reinterpret_cast<const float*>(q.gen + stage * kQ1TileBytes) + trow * 128 + 4 * sub;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 t4 = *reinterpret_cast<const float4*>(src + 32 * j);
+        v[j][0] = t4.x; v[j][1] = t4.y; v[j][2] = t4.z; v[j][3] = t4.w;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q.bars + 8u * (kQ1Stages + stage));
+    if (!dead) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(v[j][e]));
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const long long r = rt * kQ1Rows + trow;
+      if (r < rows) {
+        const float sc = group_scale(amax);
+        const long long c0 = kb * 128 + 4 * sub;
+        uint8_t* dst = Q + r * cols + c0;
+        const bool vec = vec_st && kb * 128 + 128 <= cols;
+        if (markstein_ok(sc)) store_codes16(markstein_div(sc), v, dst, c0, cols, vec);
+        else store_codes16(ExactDiv{sc}, v, dst, c0, cols, vec);
+        if (sub == 0) S[kb * rows + r] = sc;
+      }
+    }
+    kb += step_kb;
+    rt += step_rt;
+    if (kb >= kbn) {
+      kb -= kbn;
+      ++rt;
+    }
+    if (++stage == kQ1Stages) { stage = 0; phase ^= 1u; }
+  }
+}
+
+// 128x128 blocks of the weight X[K, N]; codes are written transposed, Q[n][k]. One tile
+// = one block (64 KB), three stages, one CTA per SM. kNContig: X row-major (n
+// contiguous), the stage holds T[k][n]; otherwise X column-major (k contiguous) and the
+// stage holds T[n][k]. Pass 1: every consumer thread takes the amax of 64 elements (16
+// float4 reads), the block's amax is reduced through shared memory (one named barrier).
+// Pass 2 reads the stage again in the order the codes are stored:
+//  - T[k][n]: thread (n = i % 128, kh = i / 128) walks 64 k of column n (a warp reads 32
+//    consecutive n of one k row: no bank conflicts) and stores 4 x 16 codes;
+//  - T[n][k]: warp w walks rows n = 16w..16w+15, lane l encodes k = 4l..4l+3 of each
+//    (a warp reads one 512-byte row) and stores 4 codes.
+constexpr int kQ2TileBytes = 128 * 128 * 4;
+constexpr int kQ2Stages = 3;
+constexpr int kQ2Smem = 1024 + kQ2Stages * kQ2TileBytes + 16 * kQ2Stages + 16 + 2 * kQConsumers * 4;
+
+template <bool kNContig>
+__global__ void __launch_bounds__(kQThreads, 1) quant_128x128_tma_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                                          long long K, long long N,
+                                                                          uint8_t* __restrict__ Q,
+                                                                          float* __restrict__ S,
+                                                                          unsigned long long limit) {
+  extern __shared__ uint8_t smem_raw[];
+  const QRing q = q_ring_setup<kQ2Stages, kQ2TileBytes>(smem_raw);
+  float* red = reinterpret_cast<float*>(const_cast<uint8_t*>(q.gen) + kQ2Stages * kQ2TileBytes + 16 * kQ2Stages + 16);
+  const long long kbn = (K + 127) / 128, nbn = (N + 127) / 128;
+  const long long T = kbn * nbn;
+  const int warp = static_cast<int>(warp_id()), lane = static_cast<int>(lane_id());
+  if (warp == kQConsumers) {
+    if (lane == 0)
+      q_produce<kQ2Stages, kQ2TileBytes>(q, &tm_x, T, [&](long long t, int& x, int& y) {
+        const long long kb = t / nbn, nb = t - kb * nbn;
+        x = static_cast<int>((kNContig ? nb : kb) * 128);
+        y = static_cast<int>((kNContig ? kb : nb) * 128);
+      }, limit);
+    return;
+  }
+  const int ptid = static_cast<int>(threadIdx.x);
+  int stage = 0;
+  uint32_t phase = 0;
+  bool dead = false;
+  uint32_t it = 0;
+  for (long long t = blockIdx.x; t < T; t += gridDim.x, ++it) {
+    if (!dead) dead = !mbar_wait(q.bars + 8u * stage, phase, q.abort_flag, limit);
+    dead = __any_sync(0xffffffffu, dead);
+    const float* tile = reinterpret_cast<const float*>(q.gen + stage * kQ2TileBytes);
+    float amax = 0.0f;
+    if (!dead) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float4 t4 = reinterpret_cast<const float4*>(tile)[i * 256 + ptid];
+        amax = fmaxf(fmaxf(amax, fmaxf(fabsf(t4.x), fabsf(t4.y))), fmaxf(fabsf(t4.z), fabsf(t4.w)));
+      }
+    }
+    amax = warp_max(amax);
+    float* rb = red + (it & 1) * kQConsumers;
+    if (lane == 0) rb[warp] = amax;
+    named_barrier_sync(1, kQConsumers * 32);
+    float m = rb[0];
+#pragma unroll
+    for (int w = 1; w < kQConsumers; ++w) m = fmaxf(m, rb[w]);
+    const long long kb = t / nbn, nb = t - kb * nbn;
+    const float sc = group_scale(m);
+    if (!dead) {
+      if (ptid == 0) S[kb * nbn + nb] = sc;
+      if (markstein_ok(sc)) encode_block<kNContig>(markstein_div(sc), tile, ptid, kb, nb, K, N, Q);
+      else encode_block<kNContig>(ExactDiv{sc}, tile, ptid, kb, nb, K, N, Q);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q.bars + 8u * (kQ2Stages + stage));
+    if (++stage == kQ2Stages) { stage = 0; phase ^= 1u; }
+  }
 }
 
 __global__ void fill_epilogue_kernel(int M, int N, const void* bias, int bias_dtype, int act, void* C,
@@ -321,27 +444,48 @@ __global__ void wait_selftest_kernel(unsigned long long limit_cycles) {
 
 }  // namespace
 
-cudaError_t launch_quant_1x128(const float* X, long long rows, long long cols, long long rs,
-                               long long cs, uint8_t* Q, float* S, cudaStream_t stream) {
-  const long long kbn = (cols + 127) / 128;
-  if (cs == 1) {
-    const long long groups = rows * kbn;
-    const long long blocks = (groups + 8 * kGroupsPerWarp - 1) / (8 * kGroupsPerWarp);
-    quant_1x128_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(X, rows, cols, rs, Q, S);
-  } else {
-    dim3 grid(static_cast<unsigned>((rows + 255) / 256), static_cast<unsigned>(kbn));
-    quant_1x128_cols_kernel<<<grid, 256, 0, stream>>>(X, rows, cols, cs, Q, S);
+cudaError_t launch_quant_1x128_tma(const CUtensorMap& tm_x, long long rows, long long cols, uint8_t* Q, float* S,
+                                   int sms, unsigned long long limit, cudaStream_t stream) {
+  static cudaError_t attr = cudaFuncSetAttribute(quant_1x128_tma_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kQ1Smem);
+  if (attr != cudaSuccess) return attr;
+  static int per_sm = 0;
+  if (per_sm == 0 && cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_1x128_tma_kernel, kQThreads,
+                                                                    kQ1Smem) != cudaSuccess) {
+    cudaGetLastError();
+    per_sm = 1;
   }
+  const long long tiles = (rows + kQ1Rows - 1) / kQ1Rows * ((cols + 127) / 128);
+  const long long cap = static_cast<long long>(per_sm > 0 ? per_sm : 1) * sms;
+  const long long blocks = tiles < cap ? tiles : cap;
+  quant_1x128_tma_kernel<<<static_cast<unsigned>(blocks), kQThreads, kQ1Smem, stream>>>(tm_x, rows, cols, Q, S,
+                                                                                        limit);
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_128x128(const float* X, long long K, long long N, long long rs, long long cs,
-                                 uint8_t* Q, float* S, cudaStream_t stream) {
-  const int smem = 128 * 128 * static_cast<int>(sizeof(float));
-  cudaError_t e = cudaFuncSetAttribute(quant_128x128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((K + 127) / 128));
-  quant_128x128_kernel<<<grid, 256, smem, stream>>>(X, K, N, rs, cs, Q, S);
+cudaError_t launch_quant_1x128_cols(const float* X, long long rows, long long cols, long long ldx, uint8_t* Q,
+                                    float* S, cudaStream_t stream) {
+  const long long kbn = (cols + 127) / 128;
+  dim3 grid(static_cast<unsigned>((rows + 255) / 256), static_cast<unsigned>(kbn));
+  quant_1x128_cols_kernel<<<grid, 256, 0, stream>>>(X, rows, cols, ldx, Q, S);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_128x128_tma(const CUtensorMap& tm_x, bool n_contig, long long K, long long N, uint8_t* Q,
+                                     float* S, int sms, unsigned long long limit, cudaStream_t stream) {
+  const long long tiles = ((K + 127) / 128) * ((N + 127) / 128);
+  const unsigned blocks = static_cast<unsigned>(tiles < sms ? tiles : sms);
+  if (n_contig) {
+    static cudaError_t attr = cudaFuncSetAttribute(quant_128x128_tma_kernel<true>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kQ2Smem);
+    if (attr != cudaSuccess) return attr;
+    quant_128x128_tma_kernel<true><<<blocks, kQThreads, kQ2Smem, stream>>>(tm_x, K, N, Q, S, limit);
+  } else {
+    static cudaError_t attr = cudaFuncSetAttribute(quant_128x128_tma_kernel<false>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kQ2Smem);
+    if (attr != cudaSuccess) return attr;
+    quant_128x128_tma_kernel<false><<<blocks, kQThreads, kQ2Smem, stream>>>(tm_x, K, N, Q, S, limit);
+  }
   return cudaGetLastError();
 }
 
