@@ -135,44 +135,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warpgroup 0: producer, MMA issuer, scale loader (few registers each).
     regs_dec<kRoleRegs>();
   if (warp == 0) {
-    if (lane == 0) {
-      // -------------------------------------------------------------- TMA producer
-      int stage = 0;
-      uint32_t phase = 0;
-      long long issued = 0;
-      WorkIter it;
-      it.init(s, cluster);
-      Seg seg;
-      bool ok = true;
-      while (ok && it.next(s, seg)) {
-        int mt, nt;
-        tile_coords(s, seg.tile, mt, nt);
-        const int a_row = mt * 256 + static_cast<int>(rank) * 128;
-        const int b_row = nt * TN + static_cast<int>(rank) * Cfg::kBRows;
-        for (int kb = seg.kb0; kb < seg.kb1; ++kb) {
-          if (!mbar_wait_inl(empty_bar(stage), phase ^ 1u, abort_flag, limit)) { ok = false; break; }
-          const uint32_t sa_s = smem_base + stage * STAGE_BYTES;
-          const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
+    // ---------------------------------------------------------------- TMA producer
+    // The whole warp runs the loop (its addresses stay warp-uniform); one elected lane
+    // issues the copies.
+    int stage = 0;
+    uint32_t phase = 0;
+    long long issued = 0;
+    WorkIter it;
+    it.init(s, cluster);
+    Seg seg;
+    bool ok = true;
+    while (ok && it.next(s, seg)) {
+      int mt, nt;
+      tile_coords(s, seg.tile, mt, nt);
+      const int a_row = mt * 256 + static_cast<int>(rank) * 128;
+      const int b_row = nt * TN + static_cast<int>(rank) * Cfg::kBRows;
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb) {
+        const bool w = mbar_wait_inl(empty_bar(stage), phase ^ 1u, abort_flag, limit);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        const uint32_t sa_s = smem_base + stage * STAGE_BYTES;
+        const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
+        if (elect_one()) {
           if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
           tma_load_2d_pair(sa_s, &tm_a, leader_full, kb * BKB, a_row);
           tma_load_2d_pair(sa_s + A_BYTES, &tm_b, leader_full, kb * BKB, b_row);
-          ++issued;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        __syncwarp();
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-      if (!ok && rank == 0) {
-        int st = stage;
-        uint32_t ph = phase;
-        volatile int no_abort = 0;
-        for (long long i = 0; i < issued && i < STAGES; ++i) {
-          if (--st < 0) { st = STAGES - 1; ph ^= 1u; }
-          mbar_wait_inl(full_bar(st), ph, &no_abort, limit);
-        }
+    }
+    if (!ok && rank == 0 && lane == 0) {
+      int st = stage;
+      uint32_t ph = phase;
+      volatile int no_abort = 0;
+      for (long long i = 0; i < issued && i < STAGES; ++i) {
+        if (--st < 0) { st = STAGES - 1; ph ^= 1u; }
+        mbar_wait_inl(full_bar(st), ph, &no_abort, limit);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
+    if (rank == 0) {
       // -------------------------------------------------------------- MMA issuer
+      // Warp-wide loop, one elected lane issues (always the same lane, so its commits
+      // cover every MMA it issued).
       int stage = 0;
       uint32_t phase = 0;
       long long kcount = 0;
@@ -184,20 +190,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++kcount) {
           const int buf = static_cast<int>(kcount % NBUF);
           const uint32_t bphase = static_cast<uint32_t>((kcount / NBUF) & 1);
-          if (!mbar_wait_inl(pempty_bar(buf), bphase ^ 1u, abort_flag, limit)) { ok = false; break; }
-          if (!mbar_wait_inl(full_bar(stage), phase, abort_flag, limit)) { ok = false; break; }
+          bool w = mbar_wait_inl(pempty_bar(buf), bphase ^ 1u, abort_flag, limit);
+          w = w && mbar_wait_inl(full_bar(stage), phase, abort_flag, limit);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa_s = smem_base + stage * STAGE_BYTES;
           const uint32_t d_tmem = tmem_base + buf * TN;
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < BKB / 32; ++k)
-            umma_f8_pair(d_tmem, kmajor_desc(sa_s, k), kmajor_desc(sa_s + A_BYTES, k), p.idesc, k > 0 ? 1u : 0u);
-          umma_commit_pair(empty_bar(stage), 0x3);
-          umma_commit_pair(pfull_bar(buf), 0x3);
+            for (int k = 0; k < BKB / 32; ++k)
+              umma_f8_pair(d_tmem, kmajor_desc(sa_s, k), kmajor_desc(sa_s + A_BYTES, k), p.idesc, k > 0 ? 1u : 0u);
+            umma_commit_pair(empty_bar(stage), 0x3);
+            umma_commit_pair(pfull_bar(buf), 0x3);
+          }
+          __syncwarp();
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      umma_commit_pair(drain_bar, 0x1);
+      if (elect_one()) umma_commit_pair(drain_bar, 0x1);
+      __syncwarp();
       volatile int no_abort = 0;
       mbar_wait_inl(drain_bar, 0, &no_abort, limit);
     }

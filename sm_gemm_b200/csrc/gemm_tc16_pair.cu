@@ -13,6 +13,8 @@
 //           both CTAs' copies completes on the rank-0 CTA's "full" barrier.
 //  warp 1   MMA issuer (rank 0 only): 4 x K=16 MMAs of 256 x 256 per stage; commits
 //           free the stage in both CTAs and signal both CTAs' accumulators.
+//  Both run their loops on the whole warp, so descriptors and coordinates stay in
+//  warp-uniform registers, and one elected lane issues.
 //  warp 2   TMEM allocator (cta_group::2, 512 columns = two 256-column accumulators).
 //  warps 4-7 epilogue: each CTA drains its own 128 rows; they release the accumulator
 //           to the rank-0 MMA issuer with a cluster-scope arrive.
@@ -90,8 +92,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const TileSched& s = p.s;
   const uint64_t limit = p.wait_limit_cycles;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
+    // The whole warp runs the loop (its addresses stay warp-uniform); one elected lane
+    // issues the copies.
     int stage = 0;
     uint32_t phase = 0;
     long long issued = 0;
@@ -105,17 +109,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int a_row = mt * 256 + static_cast<int>(rank) * 128;
       const int b_row = nt * kTileN + static_cast<int>(rank) * 128;
       for (int kb = seg.kb0; kb < seg.kb1; ++kb) {
-        if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit)) { ok = false; break; }
+        const bool w = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         const uint32_t sa = smem_base + stage * STAGE_BYTES;
         const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
-        if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-        load_operand_pair<128, BK>(sa, &tm_a, leader_full, p.a_mn_major, a_row, kb * BK);
-        load_operand_pair<128, BK>(sa + A_BYTES, &tm_b, leader_full, p.b_mn_major, b_row, kb * BK);
+        if (elect_one()) {
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          load_operand_pair<128, BK>(sa, &tm_a, leader_full, p.a_mn_major, a_row, kb * BK);
+          load_operand_pair<128, BK>(sa + A_BYTES, &tm_b, leader_full, p.b_mn_major, b_row, kb * BK);
+        }
+        __syncwarp();
         ++issued;
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
     }
-    if (!ok && rank == 0) {
+    if (!ok && rank == 0 && lane == 0) {
       // Wait (bounded, independent of the abort flag) for copies still in flight.
       int st = stage;
       uint32_t ph = phase;
@@ -125,8 +133,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(full_bar(st), ph, &no_abort, limit);
       }
     }
-  } else if (warp == 1 && lane == 0 && rank == 0) {
+  } else if (warp == 1 && rank == 0) {
     // ---------------------------------------------------------------- MMA issuer
+    // Warp-wide loop, one elected lane issues (always the same lane, so its commits
+    // cover every MMA it issued).
     int stage = 0;
     uint32_t phase = 0;
     int local = 0;
@@ -137,27 +147,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (ok && it.next(s, seg)) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, limit)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, limit))) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * kTileN;
       for (int kb = seg.kb0; kb < seg.kb1; ++kb) {
-        if (!mbar_wait(full_bar(stage), phase, abort_flag, limit)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, abort_flag, limit))) { ok = false; break; }
         tc_fence_after();
         const uint32_t sa = smem_base + stage * STAGE_BYTES;
         const uint32_t sb = sa + A_BYTES;
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < KSTEPS; ++k) {
-          umma_f16_pair(d_tmem, operand_desc<128, BK>(sa, p.a_mn_major, k),
-                        operand_desc<128, BK>(sb, p.b_mn_major, k), p.idesc, (kb > seg.kb0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < KSTEPS; ++k) {
+            umma_f16_pair(d_tmem, operand_desc<128, BK>(sa, p.a_mn_major, k),
+                          operand_desc<128, BK>(sb, p.b_mn_major, k), p.idesc, (kb > seg.kb0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit_pair(empty_bar(stage), 0x3);
         }
-        umma_commit_pair(empty_bar(stage), 0x3);
+        __syncwarp();
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
-      umma_commit_pair(tfull_bar(acc), 0x3);
+      if (elect_one()) umma_commit_pair(tfull_bar(acc), 0x3);
+      __syncwarp();
       ++local;
     }
-    umma_commit_pair(drain_bar, 0x1);
+    if (elect_one()) umma_commit_pair(drain_bar, 0x1);
+    __syncwarp();
     volatile int no_abort = 0;
     mbar_wait(drain_bar, 0, &no_abort, limit);
   } else if (warp >= kEpiWarp0) {
