@@ -5,9 +5,10 @@
 One step is one call of the hot path on one batch of synthetic input. The headline
 workload is the square BF16 GEMM (A[4096,4096] row-major x B[4096,4096] column-major,
 FP32 accumulation, BF16 out); its throughput in TFLOP/s is ``value``. The other
-workloads (tiny FP16, the FFN pair, FP8 block-scaled GEMM and its quantiser, the
-LM-head GEMM at M in {1,4,16,64}) are timed the same way and reported under
-``configs``. FLOPs are 2*M*N*K; bytes count every operand once.
+workloads (tiny FP16, the FFN pair and the backward GEMMs of its first layer, eight
+grouped GEMMs in one launch and as eight calls, FP8 block-scaled GEMM and its
+quantiser, the LM-head GEMM at M in {1,4,16,64}) are timed the same way and reported
+under ``configs``. FLOPs are 2*M*N*K; bytes count every operand once.
 
 Timing: W untimed warm-up steps, then K steps between CUDA events on the launching
 stream, bracketed by a barrier and a device synchronise; the maximum over ranks is
@@ -299,6 +300,49 @@ def wl_ffn(c: Ctx):
     c.record("ffn_pair", ms1 + ms2, c.K, flops=2 * fl, peak_tf=pk)
 
 
+def wl_ffn_backward(c: Ctx):
+    """Backward GEMMs of the FFN's first layer through layout flags: dX = dH W1^T (W1 read
+    as a column-major B) and dW1 = X^T dH (X read as a column-major A). Each call moves
+    more than L2 (W1 is 128 MB; dW1 writes 128 MB)."""
+    torch, sg, m = c.torch, c.sg, c.metrics
+    f = c.synth.ffn_backward()
+    X, W1, dH = c.t(f["X"]), c.t(f["W1"]), c.t(f["dH"])
+    dX = torch.empty((1024, 4096), dtype=torch.bfloat16, device=c.dev)
+    dW1 = torch.empty((4096, 16384), dtype=torch.bfloat16, device=c.dev)
+    ws = torch.empty(max(sg.workspace_size(1024, 4096, 16384), sg.workspace_size(4096, 16384, 1024), 16),
+                     dtype=torch.uint8, device=c.dev)
+    ms1 = c.time(lambda i: sg.gemm_bf16(dH, W1.t(), out=dX, workspace=ws))
+    p1 = sg.last_config()
+    ms2 = c.time(lambda i: sg.gemm_bf16(X.t(), dH, out=dW1, workspace=ws))
+    p2 = sg.last_config()
+    fl = m.gemm_flops(1024, 4096, 16384)
+    pk = c.peaks["bf16_tflops"]
+    c.record("ffn_backward_dX", ms1, c.K, flops=fl, peak_tf=pk, extra={"plan": p1})
+    c.record("ffn_backward_dW1", ms2, c.K, flops=fl, peak_tf=pk, extra={"plan": p2})
+
+
+def wl_grouped(c: Ctx):
+    """Eight independent GEMMs X_g[128(g+1), 4096] x W_g[4096, 4096] (4608 rows in all):
+    one grouped launch against the same GEMMs issued one call each. W is 256 MB."""
+    torch, sg, m = c.torch, c.sg, c.metrics
+    d = c.synth.grouped_experts()
+    Xs, Ws = [c.t(x) for x in d["X"]], [c.t(w) for w in d["W"]]
+    Ys = [torch.empty((x.shape[0], 4096), dtype=torch.bfloat16, device=c.dev) for x in Xs]
+    ws = torch.empty(max([sg.workspace_size(x.shape[0], 4096, 4096) for x in Xs] +
+                         [int(sg.lib().smgemm_grouped_workspace_size(len(Xs))), 16]), dtype=torch.uint8, device=c.dev)
+    fl = sum(m.gemm_flops(x.shape[0], 4096, 4096) for x in Xs)
+    pk = c.peaks["bf16_tflops"]
+    ms = c.time(lambda i: sg.gemm_bf16_grouped(Xs, Ws, outs=Ys, workspace=ws))
+    plan = sg.last_config()
+
+    def separate(i):
+        for x, w, y in zip(Xs, Ws, Ys):
+            sg.gemm_bf16(x, w, out=y, workspace=ws)
+    ms_sep = c.time(separate, launches_per_step=len(Xs))
+    c.record("grouped_experts_8x4096x4096", ms, c.K, flops=fl, peak_tf=pk, extra={"plan": plan})
+    c.record("grouped_experts_8x4096x4096_as_8_calls", ms_sep, c.K, flops=fl, peak_tf=pk)
+
+
 def wl_fp8(c: Ctx, quant=True, gemm=True):
     torch, sg, m = c.torch, c.sg, c.metrics
     f8 = c.synth.fp8_blockscaled()
@@ -353,6 +397,7 @@ def run_gpu(args, rank: int, world: int, dist):
     if args.only is not None and args.only != "square_bf16":
         {"tiny_fp16": lambda: wl_tiny_fp16(c), "ffn": lambda: wl_ffn(c),
          "fp8": lambda: wl_fp8(c, quant=False), "quant": lambda: wl_fp8(c, gemm=False),
+         "ffn_bwd": lambda: wl_ffn_backward(c), "grouped": lambda: wl_grouped(c),
          "lm_head": lambda: wl_lm_head(c)}[args.only]()
         assert c.sg.check() == c.sg.OK
         return {"only": args.only, "steps": c.K, "warmup": c.W, "gpu_launches": c.launches, "configs": c.results}
@@ -361,6 +406,8 @@ def run_gpu(args, rank: int, world: int, dist):
     if args.only is None and not args.headline_only:
         wl_tiny_fp16(c)
         wl_ffn(c)
+        wl_ffn_backward(c)
+        wl_grouped(c)
         wl_fp8(c)
         wl_lm_head(c)
     assert c.sg.check() == c.sg.OK
@@ -471,7 +518,7 @@ def main():
     ap.add_argument("--impl", default="smgemm", choices=["smgemm", "reference"])
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--only", default=None,
-                    choices=["square_bf16", "tiny_fp16", "ffn", "fp8", "quant", "lm_head"],
+                    choices=["square_bf16", "tiny_fp16", "ffn", "ffn_bwd", "grouped", "fp8", "quant", "lm_head"],
                     help="time one workload and print its line (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

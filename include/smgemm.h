@@ -105,6 +105,31 @@ smgemm_status gemm_bf16_noalloc(int64_t M, int64_t N, int64_t K,
                                 void* C, smgemm_dtype c_dtype, int64_t ldc, smgemm_stream_t stream);
 
 /*
+ * gemm_bf16_grouped: for g < G, C_g[M_g,N_g] = cast_c( act( A_g[M_g,K_g] * B_g[K_g,N_g] + bias_g ) ),
+ * all groups in one persistent launch ("为什么我们要死磕GEMM" (kwkr.cn), section 5.3:
+ * batch many small GEMMs instead of launching them one by one).
+ *   G          number of groups (0: no-op).
+ *   M,N,K,lda,ldb,ldc   host arrays of G sizes / leading dimensions, meaning as in gemm_bf16.
+ *   A,B,C      host arrays of G device pointers; bias: nullable host array of G
+ *              (nullable) device pointers.
+ *   ab_dtype, layout_a, layout_b, bias_dtype, act, c_dtype: shared by all groups, as in
+ *              gemm_bf16. Groups with M or N = 0 are skipped; K = 0 writes act(bias).
+ *   workspace  device, at least smgemm_grouped_workspace_size(G) bytes: the host writes
+ *              the groups' TMA descriptors and sizes there (an asynchronous copy on
+ *              `stream`, from pageable memory) before the launch; calls that can overlap
+ *              on the GPU must not share it.
+ * Every group is validated before anything is enqueued; errors as in gemm_bf16. Each
+ * output tile is one unit of work (no split-K); results are deterministic.
+ */
+size_t smgemm_grouped_workspace_size(int G);
+smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const int64_t* K,
+                                const void* const* A, smgemm_dtype ab_dtype, smgemm_layout layout_a,
+                                const int64_t* lda, const void* const* B, smgemm_layout layout_b,
+                                const int64_t* ldb, const void* const* bias, smgemm_dtype bias_dtype,
+                                smgemm_act act, void* const* C, smgemm_dtype c_dtype, const int64_t* ldc,
+                                void* workspace, size_t workspace_bytes, smgemm_stream_t stream);
+
+/*
  * gemm_fp8_blockscaled: C[i,j] = cast_c( act( sum_kb sa[kb,i] * sb[kb, j/128] *
  *                                         sum_{k in kb} dec(Aq[i,k]) * dec(Bq[j,k]) + bias[j] ) )
  *

@@ -8,6 +8,7 @@ is no fallback: if the library is missing or a call fails, an exception is raise
     C = sg.gemm_bf16(A, B, bias=b, act="gelu_tanh", out_dtype=torch.bfloat16)
     Q, S = sg.quantize_fp8_blockwise(X, group_rows=1)
     C = sg.gemm_fp8_blockscaled(Aq, sa, Bq, sb, out_dtype=torch.bfloat16)
+    Cs = sg.gemm_bf16_grouped([A0, A1], [B0, B1])
 """
 from __future__ import annotations
 
@@ -61,6 +62,12 @@ def lib():
             L.smgemm_selftest_wait_timeout.restype = I
             L.smgemm_schedule_dump.argtypes = [I64, I64, I64, I, I, I, P, I64]
             L.smgemm_schedule_dump.restype = I64
+            PI64, PP = C.POINTER(C.c_int64), C.POINTER(C.c_void_p)
+            L.gemm_bf16_grouped.argtypes = [I, PI64, PI64, PI64, PP, I, I, PI64, PP, I, PI64, PP, I, I, PP, I,
+                                            PI64, P, SZ, P]
+            L.gemm_bf16_grouped.restype = I
+            L.smgemm_grouped_workspace_size.argtypes = [I]
+            L.smgemm_grouped_workspace_size.restype = SZ
             _lib = L
     return _lib
 
@@ -88,6 +95,18 @@ def _layout(t, name):
     if t.stride(0) == 1:
         return COL_MAJOR, max(t.stride(1), t.shape[0])
     raise ValueError(f"{name} must have a unit stride in one dimension")
+
+
+def _layout_as(t, name, want):
+    """(layout, leading dimension) of a 2-D tensor read in layout `want` (grouped calls
+    share one layout): a single row or column fits either layout, and its unused
+    leading dimension is rounded up to 8 elements (16 bytes)."""
+    rows, cols = t.shape
+    if want == ROW_MAJOR and (t.stride(1) == 1 or cols <= 1):
+        return ROW_MAJOR, (max(t.stride(0), cols) if rows > 1 else -(-max(cols, 1) // 8) * 8)
+    if want == COL_MAJOR and (t.stride(0) == 1 or rows <= 1):
+        return COL_MAJOR, (max(t.stride(1), rows) if cols > 1 else -(-max(rows, 1) // 8) * 8)
+    raise ValueError(f"{name} cannot be read in the layout the other groups use")
 
 
 def _stream(stream):
@@ -146,6 +165,49 @@ def gemm_bf16(A, B, *, bias=None, act="none", out=None, out_dtype=None, workspac
                          None if ws is None else ws.data_ptr(), wsb, _stream(stream))
     _check(st, "gemm_bf16")
     return out
+
+
+def gemm_bf16_grouped(As, Bs, *, biases=None, act="none", outs=None, out_dtype=None, workspace=None,
+                      stream=None):
+    """C_g = act(A_g @ B_g + bias_g) for every group g in one launch. All A_g share one
+    layout and dtype, all B_g one layout; sizes may differ. ``outs`` (row-major) are
+    allocated when not given. Returns the list of outputs."""
+    torch = _torch()
+    G = len(As)
+    if len(Bs) != G or (biases is not None and len(biases) != G) or (outs is not None and len(outs) != G):
+        raise ValueError("As, Bs, biases and outs must have one entry per group")
+    if G == 0:
+        return []
+    Ms, Ns, Ks, ldas, ldbs, ldcs = [], [], [], [], [], []
+    # The shared layouts: those of the first group whose operand is not a single row or column.
+    lay_a = next((_layout(A, "A")[0] for A in As if min(A.shape) > 1), ROW_MAJOR)
+    lay_b = next((_layout(B, "B")[0] for B in Bs if min(B.shape) > 1), ROW_MAJOR)
+    res = []
+    for g, (A, B) in enumerate(zip(As, Bs)):
+        M, K = A.shape
+        K2, N = B.shape
+        if K != K2 or A.dtype != B.dtype or A.dtype != As[0].dtype:
+            raise ValueError(f"group {g}: A and B must agree in K and dtype")
+        _, lda = _layout_as(A, f"A[{g}]", lay_a)
+        _, ldb = _layout_as(B, f"B[{g}]", lay_b)
+        out = outs[g] if outs is not None else torch.empty((M, N), dtype=out_dtype or A.dtype, device=A.device)
+        if out.stride(1) != 1:
+            raise ValueError("outputs must be row-major")
+        res.append(out)
+        Ms.append(M); Ns.append(N); Ks.append(K); ldas.append(lda); ldbs.append(ldb)
+        ldcs.append(max(out.stride(0), N))
+    arr = lambda xs: (C.c_int64 * G)(*xs)
+    ptrs = lambda ts: (C.c_void_p * G)(*[None if t is None else t.data_ptr() for t in ts])
+    nbytes = int(lib().smgemm_grouped_workspace_size(G))
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(nbytes, As[0].device)
+    bias_dt = next((_dtype_code(b.dtype) for b in (biases or []) if b is not None), 0)
+    st = lib().gemm_bf16_grouped(G, arr(Ms), arr(Ns), arr(Ks), ptrs(As), _dtype_code(As[0].dtype), lay_a,
+                                 arr(ldas), ptrs(Bs), lay_b, arr(ldbs),
+                                 None if biases is None else ptrs(biases), bias_dt, ACTS[act],
+                                 ptrs(res), _dtype_code(res[0].dtype), arr(ldcs),
+                                 None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+    _check(st, "gemm_bf16_grouped")
+    return res
 
 
 def gemm_fp8_blockscaled(Aq, sa, Bq, sb, *, bias=None, act="none", out=None, out_dtype=None,

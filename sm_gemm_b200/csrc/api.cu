@@ -14,6 +14,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/smgemm.h"
 #include "kernels.h"
@@ -392,6 +393,104 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_d
   return launch_status(launch_gemm_tc16(tm_a, tm_b, p, g.v, g.pl.grid, stream));
 }
 
+size_t smgemm_grouped_workspace_size(int G) {
+  return G > 0 ? static_cast<size_t>(G) * sizeof(GroupDesc) + 64 : 0;
+}
+
+smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const int64_t* K, const void* const* A,
+                                smgemm_dtype ab_dtype, smgemm_layout layout_a, const int64_t* lda,
+                                const void* const* B, smgemm_layout layout_b, const int64_t* ldb,
+                                const void* const* bias, smgemm_dtype bias_dtype, smgemm_act act, void* const* C,
+                                smgemm_dtype c_dtype, const int64_t* ldc, void* workspace, size_t workspace_bytes,
+                                smgemm_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (G < 0 || (G > 0 && (M == nullptr || N == nullptr || K == nullptr || A == nullptr || lda == nullptr ||
+                          B == nullptr || ldb == nullptr || C == nullptr || ldc == nullptr)))
+    return SMGEMM_ERR_INVALID_ARG;
+  if (ab_dtype != SMGEMM_BF16 && ab_dtype != SMGEMM_F16) return SMGEMM_ERR_UNSUPPORTED;
+  if (!valid_layout(layout_a) || !valid_layout(layout_b)) return SMGEMM_ERR_INVALID_ARG;
+  if (!valid_out_dtype(c_dtype) || !valid_act(act)) return SMGEMM_ERR_INVALID_ARG;
+  if (G == 0) return SMGEMM_OK;
+  // Validate every group before anything is launched.
+  for (int g = 0; g < G; ++g) {
+    if (!fits_int(M[g]) || !fits_int(N[g]) || !fits_int(K[g])) return SMGEMM_ERR_INVALID_ARG;
+    if (M[g] == 0 || N[g] == 0) continue;
+    const void* bg = bias != nullptr ? bias[g] : nullptr;
+    smgemm_status st = check_output(M[g], N[g], C[g], c_dtype, ldc[g], bg, bias_dtype, act);
+    if (st != SMGEMM_OK) return st;
+    if (K[g] > 0) {
+      if (A[g] == nullptr || B[g] == nullptr) return SMGEMM_ERR_INVALID_ARG;
+      if (lda[g] < (layout_a == SMGEMM_ROW_MAJOR ? K[g] : M[g]) || ldb[g] < (layout_b == SMGEMM_ROW_MAJOR ? N[g] : K[g]))
+        return SMGEMM_ERR_INVALID_ARG;
+      if (!aligned16(A[g]) || !aligned16(B[g]) || (lda[g] * 2) % 16 != 0 || (ldb[g] * 2) % 16 != 0)
+        return SMGEMM_ERR_ALIGNMENT;
+    }
+  }
+  if (workspace == nullptr || workspace_bytes < smgemm_grouped_workspace_size(G)) return SMGEMM_ERR_WORKSPACE;
+  DevInfo d;
+  if (current_device(d) != SMGEMM_OK) return SMGEMM_ERR_CUDA;
+  const CUtensorMapDataType dt =
+      ab_dtype == SMGEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const uint32_t fmt = ab_dtype == SMGEMM_BF16 ? 1u : 0u;
+  const bool a_mn = (layout_a == SMGEMM_COL_MAJOR);
+  const bool b_mn = (layout_b == SMGEMM_ROW_MAJOR);
+  const int bk = grouped_bk();
+  std::vector<GroupDesc> table(static_cast<size_t>(G));
+  long long tiles = 0;
+  for (int g = 0; g < G; ++g) {
+    GroupDesc& e = table[static_cast<size_t>(g)];
+    std::memset(&e, 0, sizeof(e));
+    e.tile0 = tiles;
+    e.M = static_cast<int>(M[g]);
+    e.N = static_cast<int>(N[g]);
+    e.ldc = ldc[g];
+    e.C = C[g];
+    e.bias = bias != nullptr ? bias[g] : nullptr;
+    if (M[g] == 0 || N[g] == 0) continue;
+    if (K[g] == 0) {  // no products: the output is act(bias) (or act(0))
+      smgemm_status st = launch_status(launch_fill_epilogue(e.M, e.N, e.bias, bias_dtype, act, C[g], c_dtype,
+                                                            ldc[g], stream));
+      if (st != SMGEMM_OK) return st;
+      continue;
+    }
+    bool ok;
+    if (a_mn) ok = encode_2d(&e.tm_a, dt, A[g], M[g], K[g], lda[g] * 2, 64, bk);
+    else ok = encode_2d(&e.tm_a, dt, A[g], K[g], M[g], lda[g] * 2, 64, 128);
+    if (b_mn) ok = ok && encode_2d(&e.tm_b, dt, B[g], N[g], K[g], ldb[g] * 2, 64, bk);
+    else ok = ok && encode_2d(&e.tm_b, dt, B[g], K[g], N[g], ldb[g] * 2, 64, 128);
+    if (!ok) return SMGEMM_ERR_CUDA;
+    e.m_tiles = static_cast<int>((M[g] + 255) / 256);
+    e.n_tiles = static_cast<int>((N[g] + 255) / 256);
+    e.kb_total = static_cast<int>((K[g] + bk - 1) / bk);
+    tiles += static_cast<long long>(e.m_tiles) * e.n_tiles;
+  }
+  if (tiles == 0) return SMGEMM_OK;
+  GroupDesc* dev_table = reinterpret_cast<GroupDesc*>((reinterpret_cast<uintptr_t>(workspace) + 63) & ~uintptr_t(63));
+  // Pageable source: the copy has consumed `table` by the time the call returns.
+  if (cudaMemcpyAsync(dev_table, table.data(), table.size() * sizeof(GroupDesc), cudaMemcpyHostToDevice, stream) !=
+      cudaSuccess)
+    return launch_status(cudaGetLastError());
+  const int clusters_max = grouped_max_clusters();
+  if (clusters_max <= 0) return SMGEMM_ERR_CUDA;
+  GroupedParams p{};
+  p.groups = dev_table;
+  p.G = G;
+  p.total_tiles = tiles;
+  p.group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", 8));
+  p.bias_dtype = bias_dtype;
+  p.act = act;
+  p.c_dtype = c_dtype;
+  p.a_mn_major = a_mn ? 1 : 0;
+  p.b_mn_major = b_mn ? 1 : 0;
+  p.idesc = idesc_f32acc(fmt, fmt, a_mn ? 1u : 0u, b_mn ? 1u : 0u, 256, 256);
+  p.wait_limit_cycles = wait_limit();
+  const int clusters = static_cast<int>(std::min<long long>(tiles, clusters_max));
+  std::snprintf(g_last_config, sizeof(g_last_config), "path=grouped groups=%d tiles=%lld grid=%d tile=128x256", G,
+                tiles, clusters);
+  if (env_ll("SMGEMM_LOG", 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
+  return launch_status(launch_gemm_grouped(p, clusters, stream));
+}
+
 smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_t* Aq, const float* sa,
                                    const uint8_t* Bq, const float* sb, const void* bias, smgemm_dtype bias_dtype,
                                    smgemm_act act, void* C, smgemm_dtype c_dtype, int64_t ldc, void* workspace,
@@ -475,7 +574,7 @@ smgemm_status smgemm_check(smgemm_stream_t stream_) {
     return SMGEMM_ERR_CUDA;
   }
   const unsigned e = take_error_word_tc16() | take_error_word_fp8() | take_error_word_misc() | take_error_word_pair() |
-                     take_error_word_fp8_pair();
+                     take_error_word_fp8_pair() | take_error_word_grouped();
   return (e & kErrTimeout) ? SMGEMM_ERR_TIMEOUT : SMGEMM_OK;
 }
 

@@ -1,0 +1,290 @@
+// Grouped 16-bit GEMM: G independent problems C_g = act(A_g B_g + bias_g) in one
+// persistent launch on CTA pairs (256 x 256 tiles, tcgen05.mma.cta_group::2).
+//
+// This is the batching remedy of "为什么我们要死磕GEMM" (kwkr.cn), section 5.3: many small
+// GEMMs issued one by one each pay a launch and a ragged last wave, while one launch
+// over all of their tiles keeps every SM busy until the last tile. Tiles are numbered
+// group by group (grouped raster inside a group); cluster c takes tiles c, c + P, c + 2P,
+// ... over the whole list, so consecutive tiles of one group run side by side.
+//
+// Per-group data lives in a device table (GroupDesc: both TMA descriptors, sizes, output
+// and bias pointers) that the host writes into the caller's workspace before the launch.
+// Every role finds a tile's group by binary search over the groups' first-tile indices.
+// The producer issues fence.proxy.tensormap acquire on a group's descriptors before its
+// first copy from them, since the table may have been rewritten since an earlier launch.
+//
+// Roles as in gemm_tc16_pair.cu: warp 0 TMA producer and warp 1 MMA issuer (warp-wide
+// loops, one elected lane issues; MMA on the rank-0 CTA only), warp 2 TMEM allocator,
+// warps 4-7 epilogue (each CTA drains its own 128 rows of the two TMEM accumulators).
+// No stream-K: each tile is one work unit.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "operands.cuh"
+#include "sm100.cuh"
+
+namespace smg {
+
+namespace {
+constexpr int kThreads = 256;
+constexpr int kEpiWarp0 = 4;
+constexpr int kTileN = 256;
+constexpr int kTcols = 512;
+
+__device__ __forceinline__ void tensormap_acquire(const CUtensorMap* map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(map))
+               : "memory");
+}
+
+// Group of tile t (the last group whose first tile is <= t; empty groups share their
+// successor's first tile and are skipped) and the tile's (mt, nt) inside it.
+__device__ __forceinline__ int locate(const GroupedParams& p, long long t, int& mt, int& nt) {
+  int lo = 0, hi = p.G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.groups[mid].tile0 <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  const GroupDesc& d = p.groups[lo];
+  TileSched ts{};
+  ts.m_tiles = d.m_tiles;
+  ts.n_tiles = d.n_tiles;
+  ts.group_m = p.group_m < d.m_tiles ? p.group_m : d.m_tiles;
+  tile_coords(ts, static_cast<int>(t - d.tile0), mt, nt);
+  return lo;
+}
+}  // namespace
+
+template <int BK, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_constant__ GroupedParams p) {
+  constexpr int A_BYTES = 128 * BK * 2;
+  constexpr int B_BYTES = 128 * BK * 2;
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr int KSTEPS = BK / 16;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
+  const uint32_t bar_base = smem_base + STAGES * STAGE_BYTES;
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
+  uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();
+  const int cluster = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 8);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTcols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint64_t limit = p.wait_limit_cycles;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    long long issued = 0;
+    int last_g = -1;
+    bool ok = true;
+    for (long long t = cluster; ok && t < p.total_tiles; t += nclusters) {
+      int mt, nt;
+      const int g = locate(p, t, mt, nt);
+      const GroupDesc* d = p.groups + g;
+      if (g != last_g && elect_one()) {
+        tensormap_acquire(&d->tm_a);
+        tensormap_acquire(&d->tm_b);
+      }
+      last_g = g;
+      const int a_row = mt * 256 + static_cast<int>(rank) * 128;
+      const int b_row = nt * kTileN + static_cast<int>(rank) * 128;
+      for (int kb = 0; kb < d->kb_total; ++kb) {
+        const bool w = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
+        if (elect_one()) {
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          load_operand_pair<128, BK>(sa, &d->tm_a, leader_full, p.a_mn_major, a_row, kb * BK);
+          load_operand_pair<128, BK>(sa + A_BYTES, &d->tm_b, leader_full, p.b_mn_major, b_row, kb * BK);
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok && rank == 0 && lane == 0) {
+      int st = stage;
+      uint32_t ph = phase;
+      volatile int no_abort = 0;
+      for (long long i = 0; i < issued && i < STAGES; ++i) {
+        if (--st < 0) { st = STAGES - 1; ph ^= 1u; }
+        mbar_wait(full_bar(st), ph, &no_abort, limit);
+      }
+    }
+  } else if (warp == 1 && rank == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int local = 0;
+    bool ok = true;
+    for (long long t = cluster; ok && t < p.total_tiles; t += nclusters) {
+      int mt, nt;
+      const int kbn = p.groups[locate(p, t, mt, nt)].kb_total;
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, limit))) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * kTileN;
+      for (int kb = 0; kb < kbn; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, abort_flag, limit))) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        const uint32_t sb = sa + A_BYTES;
+        if (elect_one()) {
+#pragma unroll
+          for (int k = 0; k < KSTEPS; ++k) {
+            umma_f16_pair(d_tmem, operand_desc<128, BK>(sa, p.a_mn_major, k),
+                          operand_desc<128, BK>(sb, p.b_mn_major, k), p.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit_pair(empty_bar(stage), 0x3);
+        }
+        __syncwarp();
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      if (elect_one()) umma_commit_pair(tfull_bar(acc), 0x3);
+      __syncwarp();
+      ++local;
+    }
+    if (elect_one()) umma_commit_pair(drain_bar, 0x1);
+    __syncwarp();
+    volatile int no_abort = 0;
+    mbar_wait(drain_bar, 0, &no_abort, limit);
+  } else if (warp >= kEpiWarp0) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int r_local = q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    int local = 0;
+    bool dead = false;
+    for (long long t = cluster; t < p.total_tiles; t += nclusters) {
+      int mt, nt;
+      const GroupDesc* d = p.groups + locate(p, t, mt, nt);
+      const EpiArgs e{d->M, d->N, d->bias, p.bias_dtype, p.act, d->C, p.c_dtype, d->ldc};
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!dead) dead = !mbar_wait(tfull_bar(acc), acc_phase, abort_flag, limit);
+      dead = __any_sync(0xffffffffu, dead);
+      const int row = mt * 256 + static_cast<int>(rank) * 128 + r_local;
+      const uint32_t tacc = tmem_base + lane_addr + acc * kTileN;
+      if (!dead) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < kTileN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tacc + c * 32, r);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          epi_row32(e, row, nt * kTileN + c * 32, v);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+      }
+      ++local;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc_pair(tmem_base, kTcols);
+}
+
+namespace {
+constexpr int kBK = 64, kStages = 6;
+constexpr int kSmem = 1024 + kStages * (2 * 128 * kBK * 2) + 8 * (2 * kStages + 5) + 16;
+static_assert(kSmem <= 232448, "shared memory budget");
+
+cudaError_t prepare() {
+  static cudaError_t st = cudaFuncSetAttribute(gemm_grouped_kernel<kBK, kStages>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  return st;
+}
+
+cudaLaunchConfig_t config(int clusters, cudaStream_t stream, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+}  // namespace
+
+int grouped_max_clusters() {
+  static int cached = -1;
+  if (cached >= 0) return cached;
+  if (prepare() != cudaSuccess) return 0;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = config(1, nullptr, attr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_grouped_kernel<kBK, kStages>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cached = n;
+  return n;
+}
+
+int grouped_bk() { return kBK; }
+
+cudaError_t launch_gemm_grouped(const GroupedParams& p, int clusters, cudaStream_t stream) {
+  cudaError_t e = prepare();
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = config(clusters, stream, attr);
+  e = cudaLaunchKernelEx(&cfg, gemm_grouped_kernel<kBK, kStages>, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+unsigned take_error_word_grouped() { return take_error_word(); }
+
+}  // namespace smg

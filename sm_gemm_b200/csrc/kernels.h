@@ -45,6 +45,34 @@ cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm
 int tc16_pair_max_clusters();   // co-resident clusters of 2 on the current device (0 if unknown)
 int tc16_pair_bk();
 
+// Grouped GEMM (gemm_grouped.cu): one record per group in device memory, 64-byte
+// aligned (the TMA descriptors must be). tile0 = index of the group's first tile in the
+// launch's tile order; groups with no tiles share their successor's tile0.
+struct alignas(64) GroupDesc {
+  CUtensorMap tm_a, tm_b;   // A tiles 128 rows x BK, B tiles 128 columns x BK (per CTA)
+  long long tile0;
+  int M, N, kb_total, m_tiles, n_tiles, pad0;
+  const void* bias;         // nullable
+  void* C;
+  long long ldc;
+};
+static_assert(sizeof(GroupDesc) % 64 == 0, "GroupDesc keeps the descriptors 64-byte aligned in an array");
+
+struct GroupedParams {
+  const GroupDesc* groups;  // G records
+  int G;
+  long long total_tiles;
+  int group_m;
+  int bias_dtype, act, c_dtype;
+  int a_mn_major, b_mn_major;
+  uint32_t idesc;
+  unsigned long long wait_limit_cycles;
+};
+
+cudaError_t launch_gemm_grouped(const GroupedParams& p, int clusters, cudaStream_t stream);
+int grouped_max_clusters();
+int grouped_bk();
+
 struct Fp8Params {
   TileSched s;
   EpiArgs e;
@@ -91,5 +119,6 @@ unsigned take_error_word_fp8();
 unsigned take_error_word_misc();
 unsigned take_error_word_pair();
 unsigned take_error_word_fp8_pair();
+unsigned take_error_word_grouped();
 
 }  // namespace smg

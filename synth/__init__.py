@@ -126,7 +126,7 @@ def integers(seed: int, tensor_id: int, shape, lo: int, hi: int) -> np.ndarray:
 # the caller casts them to the input dtype (round to nearest even) where needed.
 # --------------------------------------------------------------------------------------
 
-SEEDS = {"tiny_fp16": 0, "square_bf16": 1, "ffn_pair": 2, "fp8_blockscaled": 3, "lm_head": 4}
+SEEDS = {"tiny_fp16": 0, "square_bf16": 1, "ffn_pair": 2, "fp8_blockscaled": 3, "lm_head": 4, "grouped": 5}
 
 
 def tiny_fp16():
@@ -149,6 +149,23 @@ def ffn_pair(tokens: int = 1024, d_model: int = 4096, d_ff: int = 16384):
             "W1": normal(s, 1, (d_model, d_ff), 0.02),
             "b1": normal(s, 2, (d_ff,), 0.01),
             "W2": normal(s, 3, (d_ff, d_model), 0.02)}
+
+
+def ffn_backward(tokens: int = 1024, d_model: int = 4096, d_ff: int = 16384):
+    """The FFN layer's X and W1 (same streams as ffn_pair) and an upstream gradient
+    dH[tokens,d_ff] N(0,1): dX = dH W1^T and dW1 = X^T dH."""
+    s = SEEDS["ffn_pair"]
+    return {"X": normal(s, 0, (tokens, d_model)),
+            "W1": normal(s, 1, (d_model, d_ff), 0.02),
+            "dH": normal(s, 4, (tokens, d_ff))}
+
+
+def grouped_experts(tokens=(128, 256, 384, 512, 640, 768, 896, 1024), d_model: int = 4096, d_out: int = 4096):
+    """One small GEMM per group g: X_g[tokens[g], d_model] N(0,1) times W_g[d_model, d_out]
+    N(0,0.02) row-major (the shape of routing tokens to several weight matrices)."""
+    s = SEEDS["grouped"]
+    return {"X": [normal(s, g, (m, d_model)) for g, m in enumerate(tokens)],
+            "W": [normal(s, 100 + g, (d_model, d_out), 0.02) for g in range(len(tokens))]}
 
 
 def fp8_blockscaled(m: int = 2048, k: int = 4096, n: int = 16384):

@@ -128,6 +128,42 @@ def test_fp8_and_quant_argument_errors():
     assert q() == sg.ERR_CUDA
 
 
+def _grouped(shapes, ab=sg.BF16, la=sg.ROW_MAJOR, lb=sg.ROW_MAJOR, ptr=FAKE, ws=FAKE, wsb=None, act=0,
+             c_dt=sg.BF16, ld_pad=0):
+    import ctypes as C
+    G = len(shapes)
+    arr = lambda xs: (C.c_int64 * max(G, 1))(*xs)
+    ptrs = lambda: (C.c_void_p * max(G, 1))(*([ptr] * G))
+    Ms, Ns, Ks = [s[0] for s in shapes], [s[1] for s in shapes], [s[2] for s in shapes]
+    lda = [(k if la == sg.ROW_MAJOR else m) + ld_pad for m, n, k in shapes]
+    ldb = [(n if lb == sg.ROW_MAJOR else k) for m, n, k in shapes]
+    wsb = sg.lib().smgemm_grouped_workspace_size(G) if wsb is None else wsb
+    return sg.lib().gemm_bf16_grouped(G, arr(Ms), arr(Ns), arr(Ks), ptrs(), ab, la, arr(lda), ptrs(), lb, arr(ldb),
+                                      None, 0, act, ptrs(), c_dt, arr(Ns), ws, wsb, None)
+
+
+def test_grouped_workspace_size():
+    L = sg.lib()
+    assert L.smgemm_grouped_workspace_size(0) == 0
+    one = L.smgemm_grouped_workspace_size(1)
+    assert one >= 320 and L.smgemm_grouped_workspace_size(8) == one + 7 * (one - 64)
+
+
+@needs_cpu
+def test_grouped_argument_errors():
+    good = [(256, 256, 256), (128, 512, 64)]
+    assert _grouped([]) == sg.OK
+    assert _grouped(good, ab=sg.F32) == sg.ERR_UNSUPPORTED
+    assert _grouped(good, act=9) == sg.ERR_INVALID_ARG
+    assert _grouped([(256, 256, 256), (-1, 8, 8)]) == sg.ERR_INVALID_ARG
+    assert _grouped(good, ld_pad=4) == sg.ERR_ALIGNMENT        # lda * 2 bytes not a multiple of 16
+    assert _grouped(good, ptr=FAKE + 2) == sg.ERR_ALIGNMENT
+    assert _grouped(good, wsb=16) == sg.ERR_WORKSPACE
+    assert _grouped(good, ws=None) == sg.ERR_WORKSPACE
+    assert _grouped([(0, 256, 256), (256, 0, 64)]) == sg.ERR_CUDA  # valid: needs a device
+    assert _grouped(good) == sg.ERR_CUDA
+
+
 # ------------------------------------------------------------------ persistent schedule
 
 def _check_schedule(M, N, K, kind=0, layout_a=sg.ROW_MAJOR, sms=148, bk=None):

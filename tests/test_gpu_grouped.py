@@ -1,0 +1,96 @@
+"""Grouped GEMM (gemm_bf16_grouped): several independent GEMMs in one launch (the
+batching remedy of "为什么我们要死磕GEMM" (kwkr.cn), section 5.3). Every group is checked
+against the oracle: in full on ragged shapes in every layout pair (with empty groups,
+a K = 0 group and per-group bias), bit for bit on integer-valued inputs, and on sampled
+outputs for eight 4096-wide groups of 128..1024 rows."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sm_gemm_b200 as sg
+import synth
+from _parity import check_tolerance, orc_view, sample_indices, to_dtype
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(300, 520, 136), (1, 64, 64), (256, 256, 1024), (0, 128, 64), (77, 40, 0), (640, 1000, 200),
+          (129, 8, 72)]
+
+
+def _operand(x, layout):
+    """bf16 CUDA tensor holding x in the given layout: row-major as is; column-major as
+    the transposed view of a [cols, ld] buffer whose ld is rows rounded up to 8 (the
+    16-byte pitch TMA needs)."""
+    t = to_dtype(x, torch.bfloat16)
+    if layout == "row":
+        return t.cuda()
+    rows, cols = t.shape
+    ld = max(8, -(-rows // 8) * 8)
+    buf = torch.zeros((cols, ld), dtype=torch.bfloat16)
+    buf[:, :rows] = t.t()
+    return buf.cuda()[:, :rows].t()
+
+
+@pytest.mark.parametrize("la,lb", [("row", "row"), ("row", "col"), ("col", "row"), ("col", "col")])
+def test_grouped_ragged_all_layouts(cuda_device, la, lb):
+    As, Bs, bs, Ah, Bh, bh = [], [], [], [], [], []
+    for g, (M, N, K) in enumerate(SHAPES):
+        a = synth.normal(41, 3 * g, (M, K))
+        b = synth.normal(41, 3 * g + 1, (K, N), 0.1)
+        As.append(_operand(a, la))
+        Bs.append(_operand(b, lb))
+        Ah.append(to_dtype(a, torch.bfloat16))
+        Bh.append(to_dtype(b, torch.bfloat16))
+        bias = to_dtype(synth.normal(41, 3 * g + 2, (N,), 0.5), torch.bfloat16) if g % 2 == 0 else None
+        bs.append(None if bias is None else bias.cuda())
+        bh.append(bias)
+    outs = sg.gemm_bf16_grouped(As, Bs, biases=bs, act="gelu_tanh", out_dtype=torch.bfloat16)
+    assert sg.check() == sg.OK
+    for g, (M, N, K) in enumerate(SHAPES):
+        if M == 0 or N == 0:
+            assert outs[g].numel() == 0
+            continue
+        a, ad = orc_view(Ah[g])
+        b, bd = orc_view(Bh[g])
+        kw = {} if bh[g] is None else dict(zip(("bias", "bias_dtype"), orc_view(bh[g])))
+        ref, acc = oracle.gemm(a, b, a_dtype=ad, b_dtype=bd, act=oracle.ACT_GELU_TANH, out_dtype=oracle.BF16,
+                               want_absacc=True, **kw)
+        check_tolerance(outs[g].float().cpu().numpy(), ref, acc, torch.bfloat16, what=f"group {g} {M}x{N}x{K}")
+
+
+def test_grouped_integer_exact_and_deterministic(cuda_device):
+    shapes = [(200, 136, 264), (512, 384, 128), (33, 520, 64)]
+    As, Bs, refs = [], [], []
+    for g, (M, N, K) in enumerate(shapes):
+        a = torch.from_numpy(synth.integers(42, 2 * g, (M, K), -3, 3)).to(torch.bfloat16)
+        b = torch.from_numpy(synth.integers(42, 2 * g + 1, (K, N), -3, 3)).to(torch.bfloat16)
+        As.append(a.cuda())
+        Bs.append(b.cuda())
+        av, ad = orc_view(a)
+        bv, bd = orc_view(b)
+        refs.append(oracle.gemm(av, bv, a_dtype=ad, b_dtype=bd, out_dtype=oracle.F32))
+    o1 = sg.gemm_bf16_grouped(As, Bs, out_dtype=torch.float32)
+    o2 = sg.gemm_bf16_grouped(As, Bs, out_dtype=torch.float32)
+    assert sg.check() == sg.OK
+    for g in range(len(shapes)):
+        assert np.array_equal(o1[g].cpu().numpy(), refs[g].astype(np.float32))
+        assert torch.equal(o1[g], o2[g])
+
+
+def test_grouped_experts_full_size(cuda_device):
+    d = synth.grouped_experts()
+    Xs = [to_dtype(x, torch.bfloat16) for x in d["X"]]
+    Ws = [to_dtype(w, torch.bfloat16) for w in d["W"]]
+    outs = sg.gemm_bf16_grouped([x.cuda() for x in Xs], [w.cuda() for w in Ws], out_dtype=torch.bfloat16)
+    assert sg.check() == sg.OK
+    assert "path=grouped" in sg.last_config()
+    for g, (X, W) in enumerate(zip(Xs, Ws)):
+        rows = sample_indices(X.shape[0], 128, 1, 20 + g)
+        cols = sample_indices(4096, 256, 1, 40 + g)
+        a, ad = orc_view(X)
+        b, bd = orc_view(W)
+        ref, acc = oracle.gemm(a, b, a_dtype=ad, b_dtype=bd, out_dtype=oracle.BF16, rows=rows, cols=cols,
+                               want_absacc=True)
+        check_tolerance(outs[g].float().cpu().numpy()[np.ix_(rows, cols)], ref, acc, torch.bfloat16,
+                        what=f"expert {g}")
