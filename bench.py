@@ -7,8 +7,8 @@ workload is the square BF16 GEMM (A[4096,4096] row-major x B[4096,4096] column-m
 FP32 accumulation, BF16 out); its throughput in TFLOP/s is ``value``. The other
 workloads (tiny FP16, the FFN pair and the backward GEMMs of its first layer, eight
 grouped GEMMs in one launch and as eight calls, FP8 block-scaled GEMM and its
-quantiser, the LM-head GEMM at M in {1,4,16,64}) are timed the same way and reported
-under ``configs``. FLOPs are 2*M*N*K; bytes count every operand once.
+quantiser, the LM-head GEMM at M in {1,4,16,64} and, at M = 16, fused with the row
+log-softmax) are timed the same way and reported under ``configs``. FLOPs are 2*M*N*K; bytes count every operand once.
 
 Timing: W untimed warm-up steps, then K steps between CUDA events on the launching
 stream, bracketed by a barrier and a device synchronise; the maximum over ranks is
@@ -390,6 +390,18 @@ def wl_lm_head(c: Ctx, ms_list=(1, 4, 16, 64)):
         ms = c.time(lambda i: sg.gemm_bf16(Xl, Wl, out=Cl, workspace=ws))
         c.record(f"lm_head_m{mm}", ms, c.K, flops=m.gemm_flops(mm, 128256, 4096),
                  nbytes=m.gemm_bytes(mm, 128256, 4096, "bf16", "bf16", "f32"), extra={"plan": sg.last_config()})
+    # The same LM head fused with the row log-softmax (3 launches: GEMM with per-tile
+    # max/sum partials, lse merge, in-place subtract). Bytes add the second pass's read
+    # and write of the FP32 output.
+    mm = 16
+    Xl = c.t(c.synth.lm_head(m=mm, vocab=8)["X"])
+    Cl = torch.empty((mm, 128256), dtype=torch.float32, device=c.dev)
+    wsl = torch.empty(max(int(sg.lib().smgemm_logsoftmax_workspace_size(mm, 128256, 4096)), 16), dtype=torch.uint8,
+                      device=c.dev)
+    ms = c.time(lambda i: sg.gemm_bf16_logsoftmax(Xl, Wl, out=Cl, workspace=wsl), launches_per_step=3)
+    c.record(f"lm_head_logsoftmax_m{mm}", ms, c.K, flops=m.gemm_flops(mm, 128256, 4096),
+             nbytes=m.gemm_bytes(mm, 128256, 4096, "bf16", "bf16", "f32") + 2 * mm * 128256 * 4,
+             extra={"plan": sg.last_config()})
 
 
 def run_gpu(args, rank: int, world: int, dist):

@@ -130,6 +130,26 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
                                 void* workspace, size_t workspace_bytes, smgemm_stream_t stream);
 
 /*
+ * gemm_bf16_logsoftmax: C[m,n] = z[m,n] - log sum_n' exp(z[m,n']), z = A[M,K] * B[K,N] + bias[N]
+ * in FP32: the LM-head projection fused with the row log-softmax that follows it
+ * ("为什么我们要死磕GEMM" (kwkr.cn), section 7.2, scheme B: GEMM + bias + LogSoftmax).
+ *   A, B, bias, lda, ldb, layouts: as in gemm_bf16 (no activation).
+ *   C          device float [M,N] row-major, ldc >= N (16-byte aligned rows): the
+ *              log-probabilities (the logits are written there first and normalised in place).
+ *   workspace  device, >= smgemm_logsoftmax_workspace_size(M,N,K) bytes, 16-byte aligned.
+ * On the skinny path (M <= 64, row-major A) the GEMM epilogue also reduces every 128
+ * logits of a row to (max, sum of exp) and the second pass only merges those and
+ * subtracts; otherwise the second pass reads the row's logits. Deterministic.
+ */
+size_t smgemm_logsoftmax_workspace_size(int64_t M, int64_t N, int64_t K);
+smgemm_status gemm_bf16_logsoftmax(int64_t M, int64_t N, int64_t K,
+                                   const void* A, smgemm_dtype ab_dtype, smgemm_layout layout_a, int64_t lda,
+                                   const void* B, smgemm_layout layout_b, int64_t ldb,
+                                   const void* bias, smgemm_dtype bias_dtype,
+                                   float* C, int64_t ldc,
+                                   void* workspace, size_t workspace_bytes, smgemm_stream_t stream);
+
+/*
  * gemm_fp8_blockscaled: C[i,j] = cast_c( act( sum_kb sa[kb,i] * sb[kb, j/128] *
  *                                         sum_{k in kb} dec(Aq[i,k]) * dec(Bq[j,k]) + bias[j] ) )
  *

@@ -193,3 +193,13 @@ def act(x: float, which: int) -> float:
 
 def load_elem(a: np.ndarray, dtype: int, idx: int) -> float:
     return _load().orc_load(_ptr(np.ascontiguousarray(a)), dtype, idx)
+
+
+def log_softmax_rows(z):
+    """out[m, n] = z[m, n] - lse_m, lse_m = mx_m + log(sum_n exp(z[m, n] - mx_m)),
+    mx_m = max_n z[m, n], in FP64: the plain row log-softmax that follows the LM-head
+    GEMM ("为什么我们要死磕GEMM", section 7.2). Returns (out, lse)."""
+    z = np.asarray(z, dtype=np.float64)
+    mx = z.max(axis=1, keepdims=True)
+    lse = mx + np.log(np.exp(z - mx).sum(axis=1, keepdims=True))
+    return z - lse, lse[:, 0]

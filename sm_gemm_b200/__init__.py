@@ -68,6 +68,10 @@ def lib():
             L.gemm_bf16_grouped.restype = I
             L.smgemm_grouped_workspace_size.argtypes = [I]
             L.smgemm_grouped_workspace_size.restype = SZ
+            L.gemm_bf16_logsoftmax.argtypes = [I64, I64, I64, P, I, I, I64, P, I, I64, P, I, P, I64, P, SZ, P]
+            L.gemm_bf16_logsoftmax.restype = I
+            L.smgemm_logsoftmax_workspace_size.argtypes = [I64, I64, I64]
+            L.smgemm_logsoftmax_workspace_size.restype = SZ
             _lib = L
     return _lib
 
@@ -164,6 +168,31 @@ def gemm_bf16(A, B, *, bias=None, act="none", out=None, out_dtype=None, workspac
                          out.data_ptr(), _dtype_code(out.dtype), ldc,
                          None if ws is None else ws.data_ptr(), wsb, _stream(stream))
     _check(st, "gemm_bf16")
+    return out
+
+
+def gemm_bf16_logsoftmax(A, B, *, bias=None, out=None, workspace=None, stream=None):
+    """log_softmax(A @ B + bias) over each row, FP32 [M, N] (the LM head and its
+    log-softmax, fused). A, B, bias as in gemm_bf16; ``out`` is allocated if not given."""
+    torch = _torch()
+    M, K = A.shape
+    K2, N = B.shape
+    if K != K2 or A.dtype != B.dtype:
+        raise ValueError("A and B must agree in K and dtype")
+    la, lda = _layout(A, "A")
+    lb, ldb = _layout(B, "B")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    if out.dtype != torch.float32 or out.stride(1) != 1:
+        raise ValueError("out must be row-major float32")
+    ldc = max(out.stride(0), N)
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
+        _workspace(int(lib().smgemm_logsoftmax_workspace_size(M, N, K)), A.device)
+    st = lib().gemm_bf16_logsoftmax(M, N, K, A.data_ptr(), _dtype_code(A.dtype), la, lda, B.data_ptr(), lb, ldb,
+                                    None if bias is None else bias.data_ptr(),
+                                    _dtype_code(bias.dtype) if bias is not None else 0,
+                                    out.data_ptr(), ldc, None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+    _check(st, "gemm_bf16_logsoftmax")
     return out
 
 

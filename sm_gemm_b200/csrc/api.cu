@@ -324,11 +324,17 @@ size_t smgemm_workspace_size(int64_t M, int64_t N, int64_t K, int kind) {
                   plan_gemm16(M, N, K, SMGEMM_COL_MAJOR, d.sms, pc).pl.ws_bytes());
 }
 
-smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_dtype ab_dtype,
-                        smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b, int64_t ldb,
-                        const void* bias, smgemm_dtype bias_dtype, smgemm_act act, void* C, smgemm_dtype c_dtype,
-                        int64_t ldc, void* workspace, size_t workspace_bytes, smgemm_stream_t stream_) {
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+}  // extern "C"
+
+namespace {
+// gemm_bf16 with, on the swap-AB path, the log-softmax tile partials written to
+// lse_part (nullable; see Tc16Params). *used_partials tells whether they were.
+smgemm_status gemm16_impl(int64_t M, int64_t N, int64_t K, const void* A, smgemm_dtype ab_dtype,
+                          smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b, int64_t ldb,
+                          const void* bias, smgemm_dtype bias_dtype, smgemm_act act, void* C, smgemm_dtype c_dtype,
+                          int64_t ldc, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                          float2* lse_part, bool* used_partials) {
+  if (used_partials != nullptr) *used_partials = false;
   if (!fits_int(M) || !fits_int(N) || !fits_int(K)) return SMGEMM_ERR_INVALID_ARG;
   if (ab_dtype != SMGEMM_BF16 && ab_dtype != SMGEMM_F16) return SMGEMM_ERR_UNSUPPORTED;
   if (!valid_layout(layout_a) || !valid_layout(layout_b)) return SMGEMM_ERR_INVALID_ARG;
@@ -383,6 +389,8 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_d
   p.s = g.pl.s;
   p.e = EpiArgs{static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C, c_dtype, ldc};
   p.wait_limit_cycles = wait_limit();
+  p.lse_part = g.skinny ? lse_part : nullptr;
+  if (used_partials != nullptr) *used_partials = p.lse_part != nullptr;
   st = prepare_workspace(g.pl, workspace, workspace_bytes, stream, &p.slots, &p.counters);
   if (st != SMGEMM_OK) return st;
   if (g.pair) {
@@ -391,6 +399,50 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_d
   }
   note_config(g.skinny ? "skinny" : "large", g.pl, g.mma_n);
   return launch_status(launch_gemm_tc16(tm_a, tm_b, p, g.v, g.pl.grid, stream));
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+}  // namespace
+
+extern "C" {
+
+smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_dtype ab_dtype,
+                        smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b, int64_t ldb,
+                        const void* bias, smgemm_dtype bias_dtype, smgemm_act act, void* C, smgemm_dtype c_dtype,
+                        int64_t ldc, void* workspace, size_t workspace_bytes, smgemm_stream_t stream) {
+  return gemm16_impl(M, N, K, A, ab_dtype, layout_a, lda, B, layout_b, ldb, bias, bias_dtype, act, C, c_dtype, ldc,
+                     workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+size_t smgemm_logsoftmax_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0) return 0;
+  return align256(smgemm_workspace_size(M, N, K, 0)) + align256(static_cast<size_t>(M) * sizeof(float)) +
+         align256(static_cast<size_t>((N + 127) / 128) * static_cast<size_t>(M) * sizeof(float2));
+}
+
+smgemm_status gemm_bf16_logsoftmax(int64_t M, int64_t N, int64_t K, const void* A, smgemm_dtype ab_dtype,
+                                   smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b,
+                                   int64_t ldb, const void* bias, smgemm_dtype bias_dtype, float* C, int64_t ldc,
+                                   void* workspace, size_t workspace_bytes, smgemm_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (M < 0 || N < 0 || K < 0) return SMGEMM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return SMGEMM_OK;
+  const size_t need = smgemm_logsoftmax_workspace_size(M, N, K);
+  if (need == 0) return SMGEMM_ERR_CUDA;  // no usable device
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return SMGEMM_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t gemm_ws = align256(smgemm_workspace_size(M, N, K, 0));
+  float* lse = reinterpret_cast<float*>(ws + gemm_ws);
+  float2* part = reinterpret_cast<float2*>(ws + gemm_ws + align256(static_cast<size_t>(M) * sizeof(float)));
+  bool used = false;
+  smgemm_status st = gemm16_impl(M, N, K, A, ab_dtype, layout_a, lda, B, layout_b, ldb, bias, bias_dtype,
+                                 SMGEMM_ACT_NONE, C, SMGEMM_F32, ldc, ws, gemm_ws, stream, part, &used);
+  if (st != SMGEMM_OK) return st;
+  DevInfo d;
+  if (current_device(d) != SMGEMM_OK) return SMGEMM_ERR_CUDA;
+  return launch_status(launch_log_softmax_rows(C, ldc, static_cast<int>(M), static_cast<int>(N),
+                                               used ? part : nullptr, static_cast<int>((N + 127) / 128), lse, d.sms,
+                                               stream));
 }
 
 size_t smgemm_grouped_workspace_size(int G) {

@@ -30,6 +30,46 @@ namespace {
 constexpr int kEpiWarp0 = 4;
 constexpr int kThreads = 256;
 
+// Log-softmax partials of one epilogue chunk (swap-AB layout: thread = output column n,
+// v[j] = accumulator of token tok0 + j). For each token, the 128 columns' max logit
+// (bias included) and sum of exp(logit - max) are reduced across the 4 epilogue warps
+// (shuffles, then `red`: 8 x CH floats of shared memory) and written to
+// part[vt * M + token]. Every epilogue thread calls it (named barrier 2, 128 threads);
+// dead threads and columns past N contribute nothing.
+template <int CH>
+__device__ __forceinline__ void lse_partial(const Tc16Params& p, int n, int tok0, int vt, const float* v, bool dead,
+                                            float* red, int epi_tid) {
+  const bool valid = !dead && n < p.e.N;
+  const float b = (valid && p.e.bias != nullptr) ? load_bias(p.e.bias, p.e.bias_dtype, n) : 0.0f;
+  const int w = epi_tid >> 5, ln = epi_tid & 31;
+  float x[CH];
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    x[j] = valid ? v[j] + b : -INFINITY;
+    float m = x[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (ln == 0) red[w * CH + j] = m;
+  }
+  named_barrier_sync(2, 128);
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    const float mx = fmaxf(fmaxf(red[j], red[CH + j]), fmaxf(red[2 * CH + j], red[3 * CH + j]));
+    float e = valid ? expf(x[j] - mx) : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+    if (ln == 0) red[4 * CH + w * CH + j] = e;
+  }
+  named_barrier_sync(2, 128);
+  if (epi_tid < CH && tok0 + epi_tid < p.e.M) {
+    const int j = epi_tid;
+    const float mx = fmaxf(fmaxf(red[j], red[CH + j]), fmaxf(red[2 * CH + j], red[3 * CH + j]));
+    const float sum = ((red[4 * CH + j] + red[5 * CH + j]) + red[6 * CH + j]) + red[7 * CH + j];
+    p.lse_part[static_cast<size_t>(vt) * p.e.M + tok0 + j] = make_float2(mx, sum);
+  }
+  named_barrier_sync(2, 128);
+}
+
 }  // namespace
 
 template <int MMA_N, int BK, int STAGES, bool SWAP>
@@ -56,6 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   volatile int* reduce_flag = reinterpret_cast<volatile int*>(misc + 8);
+  float* lse_red = reinterpret_cast<float*>(misc + 16);  // 8 x CH floats (log-softmax partials)
 
   const uint32_t warp = warp_id(), lane = lane_id();
 
@@ -180,33 +221,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tacc = tmem_base + lane_addr + acc * MMA_N;
       const bool whole = (seg.kb0 == 0 && seg.kb1 == s.kb_total);
       float* my_slot = p.slots + (static_cast<size_t>(blockIdx.x) * 2 + seg.slot) * (128 * MMA_N);
-      if (!dead) {
-        tc_fence_after();
+      // Log-softmax partials (swap-AB only): every epilogue warp, dead or not, takes part
+      // in their named barriers, so the chunk loop then runs on all warps.
+      const bool lse_on = SWAP && p.lse_part != nullptr;
+      if (!dead || (lse_on && whole)) {
+        if (!dead) tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < MMA_N / CH; ++c) {
-          uint32_t r[32];
-          if constexpr (CH == 32) {
-            tmem_ld_32x32b_x32(tacc + c * 32, r);
-          } else {
-            uint32_t r16[16];
-            tmem_ld_32x32b_x16(tacc + c * 16, r16);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) r[j] = r16[j];
-          }
-          tmem_ld_wait();
           float v[32];
+          if (!dead) {
+            uint32_t r[32];
+            if constexpr (CH == 32) {
+              tmem_ld_32x32b_x32(tacc + c * 32, r);
+            } else {
+              uint32_t r16[16];
+              tmem_ld_32x32b_x16(tacc + c * 16, r16);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          if (whole) {
-            if constexpr (SWAP) epi_col<CH>(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
-            else epi_row32(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
+              for (int j = 0; j < 16; ++j) r[j] = r16[j];
+            }
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
           } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+          }
+          if (whole) {
+            if constexpr (SWAP) {
+              if (lse_on) lse_partial<CH>(p, mt * 128 + r_local, nt * MMA_N + c * CH, mt, v, dead, lse_red, epi_tid);
+              if (!dead) epi_col<CH>(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
+            } else {
+              if (!dead) epi_row32(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
+            }
+          } else if (!dead) {
             slot_store<CH>(my_slot, r_local, c * CH, v);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar(acc));
+        if (!dead) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(acc));
+        }
       }
 
       if (!whole) {
@@ -240,8 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float* src = p.slots + (static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * (128 * MMA_N);
               slot_accumulate<CH>(src, r_local, c * CH, v);
             }
-            if constexpr (SWAP) epi_col<CH>(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
-            else epi_row32(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
+            if constexpr (SWAP) {
+              if (lse_on) lse_partial<CH>(p, mt * 128 + r_local, nt * MMA_N + c * CH, mt, v, false, lse_red, epi_tid);
+              epi_col<CH>(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
+            } else {
+              epi_row32(p.e, mt * 128 + r_local, nt * MMA_N + c * CH, v);
+            }
           }
         }
         named_barrier_sync(1, 128);
@@ -262,7 +321,7 @@ template <int MMA_N, int BK, int STAGES, bool SWAP>
 static cudaError_t launch_tc16(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Tc16Params& p,
                                int grid, cudaStream_t stream) {
   constexpr int STAGE_BYTES = 128 * BK * 2 + MMA_N * BK * 2;
-  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5) + 16;
+  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5) + 16 + 8 * 32 * 4;
   static_assert(SMEM <= 232448, "shared memory budget");
   auto kern = gemm_tc16_kernel<MMA_N, BK, STAGES, SWAP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);

@@ -29,6 +29,9 @@ struct Tc16Params {
   float* slots;             // stream-K partial tiles: [num_ctas][2][MMA_N][128] floats
   int* counters;            // stream-K arrival counters, one per stream-K tile, zeroed per call
   unsigned long long wait_limit_cycles;
+  // Swap-AB (skinny) kernels only, nullable: per 128-column tile of the output and per
+  // token row, the tile's max logit and sum of exp(logit - max) (float2 [m_tiles][M]).
+  float2* lse_part;
 };
 
 enum class Tc16Variant { kLarge, kSkinny16, kSkinny32, kSkinny64 };
@@ -44,6 +47,12 @@ cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm
                                   int clusters, cudaStream_t stream);
 int tc16_pair_max_clusters();   // co-resident clusters of 2 on the current device (0 if unknown)
 int tc16_pair_bk();
+
+// Row log-softmax of an FP32 [M, N] logit matrix in place (logsoftmax.cu): lse[m] from the
+// GEMM's per-tile partials (part != nullptr, [n_tiles][M]) or from the logits, then
+// C[m, n] -= lse[m].
+cudaError_t launch_log_softmax_rows(float* C, long long ldc, int M, int N, const float2* part, int n_tiles,
+                                    float* lse, int sms, cudaStream_t stream);
 
 // Grouped GEMM (gemm_grouped.cu): one record per group in device memory, 64-byte
 // aligned (the TMA descriptors must be). tile0 = index of the group's first tile in the

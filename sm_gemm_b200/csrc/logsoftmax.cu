@@ -1,0 +1,116 @@
+// Row log-softmax of the LM-head logits, the second, light pass of the GEMM + bias +
+// LogSoftmax fusion of "为什么我们要死磕GEMM" (kwkr.cn), section 7.2 (scheme B):
+// out[m, n] = logit[m, n] - lse[m], lse[m] = log sum_n exp(logit[m, n]).
+//
+// The swap-AB GEMM epilogue already reduced every 128-column tile of a row to a pair
+// (max, sum of exp(logit - max)); this pass merges a row's pairs with the online rule
+//   (m1, s1) + (m2, s2) = (M, s1 e^(m1 - M) + s2 e^(m2 - M)),  M = max(m1, m2)
+// (a pair with s = 0 is the identity), so the logits are read once more, only to
+// subtract lse. Without partials (logits from the large-tile kernels) the same merge
+// runs over the row's logits themselves. Reductions use a fixed order: results are
+// deterministic run to run.
+#include <math.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace smg {
+
+namespace {
+
+struct MaxSum {
+  float m, s;
+};
+
+__device__ __forceinline__ MaxSum merge(MaxSum a, MaxSum b) {
+  if (a.s == 0.0f) return b;
+  if (b.s == 0.0f) return a;
+  const float M = fmaxf(a.m, b.m);
+  return {M, a.s * expf(a.m - M) + b.s * expf(b.m - M)};
+}
+
+// Block-wide merge (256 threads) in a fixed order; the result is returned to thread 0.
+__device__ __forceinline__ MaxSum block_merge(MaxSum v, MaxSum* sh) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    MaxSum u{__shfl_xor_sync(0xffffffffu, v.m, o), __shfl_xor_sync(0xffffffffu, v.s, o)};
+    v = merge(v, u);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) sh[w] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < static_cast<int>(blockDim.x >> 5); ++i) v = merge(v, sh[i]);
+  }
+  return v;
+}
+
+// One CTA per row: lse[m] from the row's tile partials part[t * M + m], t < n_tiles.
+__global__ void __launch_bounds__(256) lse_from_partials_kernel(const float2* __restrict__ part, int n_tiles, int M,
+                                                                float* __restrict__ lse) {
+  __shared__ MaxSum sh[8];
+  const int m = blockIdx.x;
+  MaxSum v{-INFINITY, 0.0f};
+  for (int t = threadIdx.x; t < n_tiles; t += blockDim.x) {
+    const float2 q = part[static_cast<size_t>(t) * M + m];
+    v = merge(v, MaxSum{q.x, q.y});
+  }
+  v = block_merge(v, sh);
+  if (threadIdx.x == 0) lse[m] = v.s > 0.0f ? v.m + logf(v.s) : -INFINITY;
+}
+
+// One CTA per row: lse[m] straight from the logits (online max and sum per thread).
+__global__ void __launch_bounds__(256) lse_from_logits_kernel(const float* __restrict__ C, long long ldc, int N,
+                                                              float* __restrict__ lse) {
+  __shared__ MaxSum sh[8];
+  const float* row = C + static_cast<long long>(blockIdx.x) * ldc;
+  MaxSum v{-INFINITY, 0.0f};
+  for (int n = threadIdx.x; n < N; n += blockDim.x) v = merge(v, MaxSum{row[n], 1.0f});
+  v = block_merge(v, sh);
+  if (threadIdx.x == 0) lse[blockIdx.x] = v.s > 0.0f ? v.m + logf(v.s) : -INFINITY;
+}
+
+// C[m, n] -= lse[m] over the whole matrix (grid-stride; float4 when rows are 16-byte
+// aligned and N is a multiple of 4).
+__global__ void __launch_bounds__(256) subtract_lse_kernel(float* __restrict__ C, long long ldc, int M, int N,
+                                                           const float* __restrict__ lse) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if ((N & 3) == 0 && (ldc & 3) == 0) {
+    const int n4 = N >> 2;
+    const long long total = static_cast<long long>(M) * n4;
+    for (long long i = tid; i < total; i += stride) {
+      const long long m = i / n4, c = i - m * n4;
+      float4* p = reinterpret_cast<float4*>(C + m * ldc) + c;
+      const float l = lse[m];
+      float4 x = *p;
+      x.x -= l; x.y -= l; x.z -= l; x.w -= l;
+      *p = x;
+    }
+  } else {
+    const long long total = static_cast<long long>(M) * N;
+    for (long long i = tid; i < total; i += stride) {
+      const long long m = i / N, n = i - m * N;
+      C[m * ldc + n] -= lse[m];
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_log_softmax_rows(float* C, long long ldc, int M, int N, const float2* part, int n_tiles,
+                                    float* lse, int sms, cudaStream_t stream) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  if (part != nullptr) lse_from_partials_kernel<<<M, 256, 0, stream>>>(part, n_tiles, M, lse);
+  else lse_from_logits_kernel<<<M, 256, 0, stream>>>(C, ldc, N, lse);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long work = static_cast<long long>(M) * N / 4;
+  const long long want = (work + 255) / 256;
+  const long long cap = 4LL * (sms > 0 ? sms : 1);
+  subtract_lse_kernel<<<static_cast<unsigned>(want < cap ? (want > 0 ? want : 1) : cap), 256, 0, stream>>>(C, ldc, M,
+                                                                                                         N, lse);
+  return cudaGetLastError();
+}
+
+}  // namespace smg

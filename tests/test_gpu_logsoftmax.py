@@ -1,0 +1,72 @@
+"""LM-head GEMM fused with the row log-softmax (gemm_bf16_logsoftmax; "为什么我们要死磕GEMM"
+(kwkr.cn), section 7.2, scheme B), against the oracle: the FP64 GEMM, then the FP64 row
+log-softmax.
+
+Tolerance, from the GEMM contract: every logit z_n of a row is within
+e_n = 1e-3 * sum_k |a_k||b_kn| + ulp_f32(z_n) of the exact one; the log-sum-exp is
+1-Lipschitz in the max norm, so it is within max_n e_n, plus the FP32 evaluation of
+exp/sum/log (a fixed-order tree of at most log2(N) additions: far below 1e-5 relative
+to 1 + |lse|). Hence |out_n - ref_n| <= e_n + max_n' e_n' + 1e-5 (1 + |lse|)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sm_gemm_b200 as sg
+import synth
+from _parity import orc_view, to_dtype
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(out, X, W, b, rows=None):
+    xa, xd = orc_view(X)
+    wa, wd = orc_view(W)
+    kw = {} if b is None else dict(zip(("bias", "bias_dtype"), orc_view(b)))
+    z, acc = oracle.gemm(xa, wa, a_dtype=xd, b_dtype=wd, out_dtype=oracle.F64, rows=rows, want_absacc=True, **kw)
+    ref, lse = oracle.log_softmax_rows(z)
+    got = out.cpu().numpy().astype(np.float64)
+    if rows is not None:
+        got = got[rows]
+    e = 1e-3 * acc + np.spacing(np.abs(z).astype(np.float32)).astype(np.float64)
+    bound = e + e.max(axis=1, keepdims=True) + 1e-5 * (1.0 + np.abs(lse))[:, None]
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all()
+    assert (err <= bound).all(), f"max err/bound {np.max(err / bound):.3g}"
+    # the probabilities of every checked row sum to one
+    assert np.allclose(np.exp(got).sum(axis=1), 1.0, atol=1e-4)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 64])
+@pytest.mark.parametrize("N", [1000, 4096])
+def test_logsoftmax_skinny(cuda_device, M, N):
+    X = to_dtype(synth.normal(51, M, (M, 256)), torch.bfloat16)
+    W = to_dtype(synth.normal(51, 100 + N, (256, N), 0.2), torch.bfloat16)
+    b = to_dtype(synth.normal(51, 200, (N,), 0.5), torch.bfloat16)
+    out = sg.gemm_bf16_logsoftmax(X.cuda(), W.cuda(), bias=b.cuda())
+    assert sg.check() == sg.OK
+    assert "path=skinny" in sg.last_config()
+    _check(out, X, W, b)
+
+
+@pytest.mark.parametrize("M,layout", [(200, "row"), (16, "col")])
+def test_logsoftmax_large_path(cuda_device, M, layout):
+    N = 1000
+    X = to_dtype(synth.normal(52, M, (M, 264)), torch.bfloat16)
+    W = to_dtype(synth.normal(52, 1, (264, N), 0.2), torch.bfloat16)
+    Xd = X.cuda() if layout == "row" else X.t().contiguous().cuda().t()
+    out = sg.gemm_bf16_logsoftmax(Xd, W.cuda())
+    assert sg.check() == sg.OK
+    assert "path=skinny" not in sg.last_config()
+    _check(out, X, W, None)
+
+
+def test_logsoftmax_lm_head_full_size(cuda_device):
+    d = synth.lm_head(16)
+    X = to_dtype(d["X"], torch.bfloat16)
+    W = to_dtype(d["W"], torch.bfloat16)
+    out = sg.gemm_bf16_logsoftmax(X.cuda(), W.cuda())
+    assert sg.check() == sg.OK
+    p = torch.exp(out.double()).sum(dim=1)
+    assert torch.allclose(p, torch.ones_like(p), atol=1e-4)
+    _check(out, X, W, None, rows=np.array([0, 15]))
