@@ -41,7 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Sources of the headline kernel (gemm_tc16_pair_kernel): a recorded DRAM-traffic figure
 # is only reported while these are unchanged since its ncu capture.
 KERNEL_SOURCES = ["sm_gemm_b200/csrc/gemm_tc16_pair.cu", "sm_gemm_b200/csrc/operands.cuh",
-                  "sm_gemm_b200/csrc/sm100.cuh", "sm_gemm_b200/csrc/epilogue.cuh"]
+                  "sm_gemm_b200/csrc/sm100.cuh", "sm_gemm_b200/csrc/epilogue.cuh",
+                  "sm_gemm_b200/csrc/fp8_codec.cuh", "sm_gemm_b200/csrc/kernels.h"]
 
 
 # ----------------------------------------------------------------------------- utilities
@@ -289,6 +290,7 @@ def wl_ffn(c: Ctx):
     Y = torch.empty((1024, 4096), dtype=torch.bfloat16, device=c.dev)
     ws = torch.empty(max(sg.workspace_size(1024, 16384, 4096), sg.workspace_size(1024, 4096, 16384), 16),
                      dtype=torch.uint8, device=c.dev)
+    ws8 = torch.empty(max(sg.workspace_size(1024, 4096, 16384, 1), 16), dtype=torch.uint8, device=c.dev)
     ms1 = c.time(lambda i: sg.gemm_bf16(X, W1, bias=b1, act="gelu_tanh", out=H, workspace=ws))
     p1 = sg.last_config()
     ms2 = c.time(lambda i: sg.gemm_bf16(H, W2, out=Y, workspace=ws))
@@ -298,6 +300,16 @@ def wl_ffn(c: Ctx):
     c.record("ffn_gemm1_bias_gelu", ms1, c.K, flops=fl, peak_tf=pk, extra={"plan": p1})
     c.record("ffn_gemm2", ms2, c.K, flops=fl, peak_tf=pk, extra={"plan": p2})
     c.record("ffn_pair", ms1 + ms2, c.K, flops=2 * fl, peak_tf=pk)
+    # The same layer with FP8 activations between the GEMMs: GEMM1's epilogue emits H as
+    # E4M3 codes + 1x128 scales, GEMM2 is the block-scaled FP8 GEMM on them (W2 quantised
+    # once, outside the timed region).
+    Hq = torch.empty((1024, 16384), dtype=torch.uint8, device=c.dev)
+    Hs = torch.empty((128, 1024), dtype=torch.float32, device=c.dev)
+    W2q, W2s = sg.quantize_fp8_blockwise(c.t(f["W2"], torch.float32), 128)
+    ms3 = c.time(lambda i: sg.gemm_bf16_fp8out(X, W1, bias=b1, act="gelu_tanh", Q=Hq, scales=Hs, workspace=ws))
+    ms4 = c.time(lambda i: sg.gemm_fp8_blockscaled(Hq, Hs, W2q, W2s, out=Y, workspace=ws8))
+    c.record("ffn_gemm1_bias_gelu_fp8out", ms3, c.K, flops=fl, peak_tf=pk)
+    c.record("ffn_gemm2_fp8", ms4, c.K, flops=fl, peak_tf=c.fp8_peak)
 
 
 def wl_ffn_backward(c: Ctx):

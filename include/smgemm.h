@@ -130,6 +130,27 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
                                 void* workspace, size_t workspace_bytes, smgemm_stream_t stream);
 
 /*
+ * gemm_bf16_fp8out: the gemm_bf16 epilogue quantised to FP8 on the way out: with
+ * Z = act(A[M,K] * B[K,N] + bias[N]) in FP32, every 1x128 row group of Z (columns
+ * 128g .. 128g+127) is encoded as quantize_fp8_blockwise does (amax over the group's
+ * present elements, s = amax/448 or 1 for an all-zero group, code = E4M3(z / s) with
+ * a correctly rounded division, RN satfinite) - "fuse activation, quantization and
+ * scaling" (DeepGEMM kernel-library walkthrough, zwxr.cn, sections 1.2 and 2.4). The
+ * output is exactly the A operand gemm_fp8_blockscaled takes (K' = N).
+ *   A, B, bias, act, lda, ldb, layouts, workspace: as in gemm_bf16.
+ *   Cq      device uint8 E4M3 codes [M][N] row-major, 16-byte aligned, ldc >= N and a
+ *           multiple of 16.
+ *   scales  device float [ceil(N/128)][M], 4-byte aligned.
+ * Runs on the CTA-pair kernel (any M); K = 0 returns SMGEMM_ERR_UNSUPPORTED.
+ */
+smgemm_status gemm_bf16_fp8out(int64_t M, int64_t N, int64_t K,
+                               const void* A, smgemm_dtype ab_dtype, smgemm_layout layout_a, int64_t lda,
+                               const void* B, smgemm_layout layout_b, int64_t ldb,
+                               const void* bias, smgemm_dtype bias_dtype, smgemm_act act,
+                               uint8_t* Cq, int64_t ldc, float* scales,
+                               void* workspace, size_t workspace_bytes, smgemm_stream_t stream);
+
+/*
  * gemm_bf16_logsoftmax: C[m,n] = z[m,n] - log sum_n' exp(z[m,n']), z = A[M,K] * B[K,N] + bias[N]
  * in FP32: the LM-head projection fused with the row log-softmax that follows it
  * ("为什么我们要死磕GEMM" (kwkr.cn), section 7.2, scheme B: GEMM + bias + LogSoftmax).

@@ -72,6 +72,8 @@ def lib():
             L.gemm_bf16_logsoftmax.restype = I
             L.smgemm_logsoftmax_workspace_size.argtypes = [I64, I64, I64]
             L.smgemm_logsoftmax_workspace_size.restype = SZ
+            L.gemm_bf16_fp8out.argtypes = [I64, I64, I64, P, I, I, I64, P, I, I64, P, I, I, P, I64, P, P, SZ, P]
+            L.gemm_bf16_fp8out.restype = I
             _lib = L
     return _lib
 
@@ -169,6 +171,35 @@ def gemm_bf16(A, B, *, bias=None, act="none", out=None, out_dtype=None, workspac
                          None if ws is None else ws.data_ptr(), wsb, _stream(stream))
     _check(st, "gemm_bf16")
     return out
+
+
+def gemm_bf16_fp8out(A, B, *, bias=None, act="none", Q=None, scales=None, workspace=None, stream=None):
+    """act(A @ B + bias) quantised to E4M3 with one FP32 scale per 1x128 row group:
+    returns (codes uint8 [M, N], scales float32 [ceil(N/128), M]), the A operand of
+    gemm_fp8_blockscaled."""
+    torch = _torch()
+    M, K = A.shape
+    K2, N = B.shape
+    if K != K2 or A.dtype != B.dtype:
+        raise ValueError("A and B must agree in K and dtype")
+    la, lda = _layout(A, "A")
+    lb, ldb = _layout(B, "B")
+    if Q is None:
+        Q = torch.empty((M, -(-N // 16) * 16), dtype=torch.uint8, device=A.device)[:, :N]
+    if scales is None:
+        scales = torch.empty((-(-N // 128), M), dtype=torch.float32, device=A.device)
+    if Q.stride(1) != 1:
+        raise ValueError("Q must be row-major")
+    ldc = max(Q.stride(0), N)
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
+        _workspace(workspace_size(M, N, K, 0), A.device)
+    st = lib().gemm_bf16_fp8out(M, N, K, A.data_ptr(), _dtype_code(A.dtype), la, lda, B.data_ptr(), lb, ldb,
+                                None if bias is None else bias.data_ptr(),
+                                _dtype_code(bias.dtype) if bias is not None else 0, ACTS[act],
+                                Q.data_ptr(), ldc, scales.data_ptr(), None if ws is None else ws.data_ptr(), wsb,
+                                _stream(stream))
+    _check(st, "gemm_bf16_fp8out")
+    return Q, scales
 
 
 def gemm_bf16_logsoftmax(A, B, *, bias=None, out=None, workspace=None, stream=None):

@@ -215,9 +215,10 @@ struct Gemm16Plan {
 // Large tiles run on CTA pairs unless SMGEMM_PAIR=0 or the device reports no
 // co-resident pair clusters; `sms` is then the SM count and `pair_clusters` the number
 // of co-resident clusters of two.
-Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms, int pair_clusters) {
+Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms, int pair_clusters,
+                       bool allow_skinny = true) {
   Gemm16Plan g;
-  const bool force_large = env_ll("SMGEMM_FORCE_LARGE", 0) != 0;
+  const bool force_large = env_ll("SMGEMM_FORCE_LARGE", 0) != 0 || !allow_skinny;
   g.skinny = (M <= 64 && layout_a == SMGEMM_ROW_MAJOR && !force_large);
   g.pair = !g.skinny && pair_clusters > 0 && env_ll("SMGEMM_PAIR", 1) != 0;
   if (g.skinny) g.v = M <= 16 ? Tc16Variant::kSkinny16 : (M <= 32 ? Tc16Variant::kSkinny32 : Tc16Variant::kSkinny64);
@@ -333,15 +334,26 @@ smgemm_status gemm16_impl(int64_t M, int64_t N, int64_t K, const void* A, smgemm
                           smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b, int64_t ldb,
                           const void* bias, smgemm_dtype bias_dtype, smgemm_act act, void* C, smgemm_dtype c_dtype,
                           int64_t ldc, void* workspace, size_t workspace_bytes, cudaStream_t stream,
-                          float2* lse_part, bool* used_partials) {
+                          float2* lse_part, bool* used_partials, float* fp8_scales = nullptr) {
   if (used_partials != nullptr) *used_partials = false;
+  const bool fp8_out = fp8_scales != nullptr;  // c_dtype E4M3: codes + 1x128 scales
   if (!fits_int(M) || !fits_int(N) || !fits_int(K)) return SMGEMM_ERR_INVALID_ARG;
   if (ab_dtype != SMGEMM_BF16 && ab_dtype != SMGEMM_F16) return SMGEMM_ERR_UNSUPPORTED;
   if (!valid_layout(layout_a) || !valid_layout(layout_b)) return SMGEMM_ERR_INVALID_ARG;
-  if (!valid_out_dtype(c_dtype) || !valid_act(act)) return SMGEMM_ERR_INVALID_ARG;
+  if ((fp8_out ? c_dtype != SMGEMM_E4M3 : !valid_out_dtype(c_dtype)) || !valid_act(act)) return SMGEMM_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return SMGEMM_OK;
-  smgemm_status st = check_output(M, N, C, c_dtype, ldc, bias, bias_dtype, act);
-  if (st != SMGEMM_OK) return st;
+  smgemm_status st = SMGEMM_OK;
+  if (fp8_out) {
+    if (!valid_act(act) || (bias != nullptr && !valid_bias_dtype(bias_dtype))) return SMGEMM_ERR_INVALID_ARG;
+    if (C == nullptr || ldc < N) return SMGEMM_ERR_INVALID_ARG;
+    if (!aligned16(C) || ldc % 16 != 0 || (reinterpret_cast<uintptr_t>(fp8_scales) & 3u)) return SMGEMM_ERR_ALIGNMENT;
+    if (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) % elem_size(bias_dtype)) != 0)
+      return SMGEMM_ERR_ALIGNMENT;
+    if (K == 0) return SMGEMM_ERR_UNSUPPORTED;
+  } else {
+    st = check_output(M, N, C, c_dtype, ldc, bias, bias_dtype, act);
+    if (st != SMGEMM_OK) return st;
+  }
   if (K > 0) {
     if (A == nullptr || B == nullptr) return SMGEMM_ERR_INVALID_ARG;
     if (lda < (layout_a == SMGEMM_ROW_MAJOR ? K : M) || ldb < (layout_b == SMGEMM_ROW_MAJOR ? N : K))
@@ -355,7 +367,8 @@ smgemm_status gemm16_impl(int64_t M, int64_t N, int64_t K, const void* A, smgemm
     return launch_status(launch_fill_epilogue(static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C,
                                               c_dtype, ldc, stream));
   }
-  const Gemm16Plan g = plan_gemm16(M, N, K, layout_a, d.sms, tc16_pair_max_clusters());
+  const Gemm16Plan g = plan_gemm16(M, N, K, layout_a, d.sms, tc16_pair_max_clusters(), !fp8_out);
+  if (fp8_out && !g.pair) return SMGEMM_ERR_UNSUPPORTED;  // the FP8 epilogue runs on the CTA-pair kernel
   const CUtensorMapDataType dt =
       ab_dtype == SMGEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const uint32_t fmt = ab_dtype == SMGEMM_BF16 ? 1u : 0u;
@@ -387,7 +400,7 @@ smgemm_status gemm16_impl(int64_t M, int64_t N, int64_t K, const void* A, smgemm
   }
   if (!ok) return SMGEMM_ERR_CUDA;
   p.s = g.pl.s;
-  p.e = EpiArgs{static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C, c_dtype, ldc};
+  p.e = EpiArgs{static_cast<int>(M), static_cast<int>(N), bias, bias_dtype, act, C, c_dtype, ldc, fp8_scales};
   p.wait_limit_cycles = wait_limit();
   p.lse_part = g.skinny ? lse_part : nullptr;
   if (used_partials != nullptr) *used_partials = p.lse_part != nullptr;
@@ -412,6 +425,15 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_d
                         int64_t ldc, void* workspace, size_t workspace_bytes, smgemm_stream_t stream) {
   return gemm16_impl(M, N, K, A, ab_dtype, layout_a, lda, B, layout_b, ldb, bias, bias_dtype, act, C, c_dtype, ldc,
                      workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+smgemm_status gemm_bf16_fp8out(int64_t M, int64_t N, int64_t K, const void* A, smgemm_dtype ab_dtype,
+                               smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b, int64_t ldb,
+                               const void* bias, smgemm_dtype bias_dtype, smgemm_act act, uint8_t* Cq, int64_t ldc,
+                               float* scales, void* workspace, size_t workspace_bytes, smgemm_stream_t stream) {
+  if (scales == nullptr) return SMGEMM_ERR_INVALID_ARG;
+  return gemm16_impl(M, N, K, A, ab_dtype, layout_a, lda, B, layout_b, ldb, bias, bias_dtype, act, Cq, SMGEMM_E4M3,
+                     ldc, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, scales);
 }
 
 size_t smgemm_logsoftmax_workspace_size(int64_t M, int64_t N, int64_t K) {

@@ -9,6 +9,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "fp8_codec.cuh"
+
 namespace smg {
 
 struct EpiArgs {
@@ -17,8 +19,9 @@ struct EpiArgs {
   int bias_dtype;      // kF32 / kBF16 / kF16
   int act;             // kActNone / kActGeluTanh / kActSilu
   void* C;
-  int c_dtype;         // kF32 / kBF16 / kF16
+  int c_dtype;         // kF32 / kBF16 / kF16, or 3 = E4M3 codes with per-1x128 scales
   long long ldc;
+  float* scales;       // E4M3 output only: [ceil(N/128)][M] group scales
 };
 
 // Activations in FP32. The GEMM epilogues use the hardware tanh.approx.f32 (maximum
@@ -66,17 +69,50 @@ __device__ __forceinline__ void store_one(void* C, int dtype, long long off, flo
 // chunk, outside the per-element loops, so the common plain path jumps over these
 // blocks in one step and stays a short, straight run of instructions (the epilogue
 // warps share instruction caches with the producer and MMA-issuer warps).
+// bias[col0 .. col0 + 32) added to v with 16-byte loads (two 16-bit values per word);
+// one branch on the bias type and alignment per chunk, none per element.
+__device__ __forceinline__ void add_bias32_vec(const EpiArgs& e, int col0, float (&v)[32]) {
+  if (e.bias_dtype == 0) {
+    const float4* b4 = reinterpret_cast<const float4*>(static_cast<const float*>(e.bias) + col0);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 b = __ldg(b4 + q);
+      v[4 * q] += b.x;
+      v[4 * q + 1] += b.y;
+      v[4 * q + 2] += b.z;
+      v[4 * q + 3] += b.w;
+    }
+  } else {
+    const uint4* b4 = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(e.bias) + col0);
+    const bool is_bf16 = e.bias_dtype == 1;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 b = __ldg(b4 + q);
+      const uint32_t w[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float2 f;
+        if (is_bf16) {
+          f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[h]));
+        } else {
+          f = __half22float2(*reinterpret_cast<const __half2*>(&w[h]));
+        }
+        v[8 * q + 2 * h] += f.x;
+        v[8 * q + 2 * h + 1] += f.y;
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ void epi_bias_act32(const EpiArgs& e, int col0, float (&v)[32]) {
   if (e.bias != nullptr) {
-    if (col0 + 32 <= e.N) {
-      if (e.bias_dtype == 0) {
-        const float* b = static_cast<const float*>(e.bias) + col0;
+    const int esz = e.bias_dtype == 0 ? 4 : 2;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(e.bias) + static_cast<uintptr_t>(col0) * esz) & 15u) == 0;
+    if (col0 + 32 <= e.N && aligned) {
+      add_bias32_vec(e, col0, v);
+    } else if (col0 + 32 <= e.N) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] += b[j];
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] += load_bias(e.bias, e.bias_dtype, col0 + j);
-      }
+      for (int j = 0; j < 32; ++j) v[j] += load_bias(e.bias, e.bias_dtype, col0 + j);
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j)
@@ -138,6 +174,62 @@ __device__ __forceinline__ void epi_store_row32(const EpiArgs& e, int row, int c
 __device__ __forceinline__ void epi_row32(const EpiArgs& e, int row, int col0, float (&v)[32]) {
   if (e.bias != nullptr || e.act != 0) epi_bias_act32(e, col0, v);
   epi_store_row32(e, row, col0, v);
+}
+
+// 32 codes of v / s, four per word.
+template <class Div>
+__device__ __forceinline__ void encode32(const Div& div, const float (&v)[32], uint32_t (&w)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float x[4] = {v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]};
+    w[q] = pack4(div, x);
+  }
+}
+
+// FP8 output: the 128 columns col0.. of one row form one 1x128 group, quantised as the
+// group quantiser does (group_scale, correctly rounded x / s, RN satfinite E4M3), after
+// bias and activation. g holds the group's 128 raw accumulators (registers); bias and
+// activation are applied in place. Columns past N take no part in the amax and are not
+// written; the codes leave as 16-byte stores (ldc and the code pointer are 16-byte
+// aligned), the scale as one float at scales[(col0 / 128) * M + row].
+__device__ __forceinline__ void epi_group_fp8_regs(const EpiArgs& e, int row, int col0, float (&g)[128]) {
+  if (row >= e.M || col0 >= e.N) return;
+  const bool full = col0 + 128 <= e.N;
+  float amax = 0.0f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float (&v)[32] = *reinterpret_cast<float(*)[32]>(g + 32 * c);
+    if (e.bias != nullptr || e.act != 0) epi_bias_act32(e, col0 + 32 * c, v);
+    if (full) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + 32 * c + j < e.N) amax = fmaxf(amax, fabsf(v[j]));
+    }
+  }
+  const float sc = group_scale(amax);
+  uint8_t* dst = static_cast<uint8_t*>(e.C) + static_cast<long long>(row) * e.ldc + col0;
+  const bool fast = markstein_ok(sc);
+  const MarksteinDiv md = markstein_div(sc);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float (&v)[32] = *reinterpret_cast<const float(*)[32]>(g + 32 * c);
+    uint32_t w[8];
+    if (fast) encode32(md, v, w);
+    else encode32(ExactDiv{sc}, v, w);
+    if (full) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+      d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + 32 * c + j < e.N) dst[32 * c + j] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
+    }
+  }
+  e.scales[static_cast<long long>(col0 / 128) * e.M + row] = sc;
 }
 
 // CNT consecutive output rows row0.. of one column (transposed accumulator tiles).

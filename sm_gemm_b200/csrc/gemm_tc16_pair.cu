@@ -36,7 +36,9 @@ constexpr int kTileN = 256;  // columns of the pair tile (128 per CTA for B, all
 constexpr int kTcols = 512;
 }  // namespace
 
-template <int BK, int STAGES>
+// FP8OUT: the epilogue emits E4M3 codes + 1x128 scales (c_dtype E4M3); a separate
+// instantiation, so the 16/32-bit-output kernel's code and registers are untouched.
+template <int BK, int STAGES, bool FP8OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc16_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const Tc16Params p) {
@@ -200,18 +202,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* my_slot = p.slots + ((static_cast<size_t>(cluster) * 2 + seg.slot) * 2 + rank) * SLOT;
       if (!dead) {
         tc_fence_after();
+        if constexpr (FP8OUT) {
+          // Each 128-column half of the tile is one 1x128 group of the row, read from
+          // TMEM once into registers (stream-K partials go to the slots unchanged).
 #pragma unroll 1
-        for (int c = 0; c < kTileN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tacc + c * 32, r);
-          tmem_ld_wait();
-          float v[32];
+          for (int gq = 0; gq < kTileN / 128; ++gq) {
+            float g[128];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          if (whole) {
-            epi_row32(p.e, row, nt * kTileN + c * 32, v);
-          } else {
-            slot_store<32>(my_slot, r_local, c * 32, v);
+            for (int c = 0; c < 4; ++c) {
+              uint32_t r[32];
+              tmem_ld_32x32b_x32_sync(tacc + gq * 128 + c * 32, r);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) g[32 * c + j] = __uint_as_float(r[j]);
+            }
+            if (whole) epi_group_fp8_regs(p.e, row, nt * kTileN + gq * 128, g);
+            else slot_store<128>(my_slot, r_local, gq * 128, g);
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < kTileN / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tacc + c * 32, r);
+            tmem_ld_wait();
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            if (whole) {
+              epi_row32(p.e, row, nt * kTileN + c * 32, v);
+            } else {
+              slot_store<32>(my_slot, r_local, c * 32, v);
+            }
           }
         }
         tc_fence_before();
@@ -237,18 +257,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           __threadfence();
           const int c_lo = sk_owner(s, t_sk * s.kb_total);
           const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
-#pragma unroll 1
-          for (int c = 0; c < kTileN / 32; ++c) {
-            float v[32];
+          // Sum of every contributor's partial for 32 columns (CTA order = K order).
+          auto reduce32 = [&](int col, float (&v)[32]) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.0f;
 #pragma unroll 1
             for (int cc = c_lo; cc <= c_hi; ++cc) {
               if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
               const float* src = p.slots + ((static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * 2 + rank) * SLOT;
-              slot_accumulate<32>(src, r_local, c * 32, v);
+              slot_accumulate<32>(src, r_local, col, v);
             }
-            epi_row32(p.e, row, nt * kTileN + c * 32, v);
+          };
+          if constexpr (FP8OUT) {
+#pragma unroll 1
+            for (int gq = 0; gq < kTileN / 128; ++gq) {
+              float g[128];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) reduce32(gq * 128 + c * 32, *reinterpret_cast<float(*)[32]>(g + 32 * c));
+              epi_group_fp8_regs(p.e, row, nt * kTileN + gq * 128, g);
+            }
+          } else {
+#pragma unroll 1
+            for (int c = 0; c < kTileN / 32; ++c) {
+              float v[32];
+              reduce32(c * 32, v);
+              epi_row32(p.e, row, nt * kTileN + c * 32, v);
+            }
           }
         }
         named_barrier_sync(1, 128);
@@ -269,43 +303,15 @@ constexpr int kPairBK = 64, kPairStages = 6;
 constexpr int kPairSmem = 1024 + kPairStages * (2 * 128 * kPairBK * 2) + 8 * (2 * kPairStages + 5) + 16;
 static_assert(kPairSmem <= 232448, "shared memory budget");
 
+template <bool FP8OUT>
 cudaError_t prepare_pair_kernel() {
-  static cudaError_t st = cudaFuncSetAttribute(gemm_tc16_pair_kernel<kPairBK, kPairStages>,
+  static cudaError_t st = cudaFuncSetAttribute(gemm_tc16_pair_kernel<kPairBK, kPairStages, FP8OUT>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
   return st;
 }
-}  // namespace
 
-int tc16_pair_max_clusters() {
-  static int cached = -1;
-  if (cached >= 0) return cached;
-  if (prepare_pair_kernel() != cudaSuccess) return 0;
+cudaLaunchConfig_t pair_config(int clusters, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kPairSmem;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc16_pair_kernel<kPairBK, kPairStages>, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    n = 0;
-  }
-  cached = n;
-  return n;
-}
-
-cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Tc16Params& p,
-                                  int clusters, cudaStream_t stream) {
-  cudaError_t e = prepare_pair_kernel();
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
@@ -316,7 +322,35 @@ cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages>, tm_a, tm_b, p);
+  return cfg;
+}
+}  // namespace
+
+int tc16_pair_max_clusters() {
+  static int cached = -1;
+  if (cached >= 0) return cached;
+  if (prepare_pair_kernel<false>() != cudaSuccess || prepare_pair_kernel<true>() != cudaSuccess) return 0;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_config(1, nullptr, attr);
+  int n = 0, n8 = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc16_pair_kernel<kPairBK, kPairStages, false>, &cfg) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n8, gemm_tc16_pair_kernel<kPairBK, kPairStages, true>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = n8 = 0;
+  }
+  cached = n < n8 ? n : n8;
+  return cached;
+}
+
+cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Tc16Params& p,
+                                  int clusters, cudaStream_t stream) {
+  const bool fp8 = p.e.c_dtype == kE4M3;
+  cudaError_t e = fp8 ? prepare_pair_kernel<true>() : prepare_pair_kernel<false>();
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_config(clusters, stream, attr);
+  e = fp8 ? cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages, true>, tm_a, tm_b, p)
+          : cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages, false>, tm_a, tm_b, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -128,6 +128,29 @@ def test_fp8_and_quant_argument_errors():
     assert q() == sg.ERR_CUDA
 
 
+@needs_cpu
+def test_fp8out_and_logsoftmax_argument_errors():
+    L = sg.lib()
+    def f8(M=256, N=256, K=256, Cq=FAKE, ldc=256, S=FAKE, act=0):
+        return L.gemm_bf16_fp8out(M, N, K, FAKE, sg.BF16, sg.ROW_MAJOR, K, FAKE, sg.ROW_MAJOR, N, None, 0, act,
+                                  Cq, ldc, S, None, 0, None)
+    assert f8(S=None) == sg.ERR_INVALID_ARG
+    assert f8(ldc=200) == sg.ERR_INVALID_ARG                  # ldc < N
+    assert f8(ldc=264) == sg.ERR_ALIGNMENT                    # not a multiple of 16 codes
+    assert f8(Cq=FAKE + 8) == sg.ERR_ALIGNMENT
+    assert f8(S=FAKE + 2) == sg.ERR_ALIGNMENT
+    assert f8(K=0) == sg.ERR_UNSUPPORTED
+    assert f8(act=9) == sg.ERR_INVALID_ARG
+    assert f8(M=0) == sg.OK
+    assert f8() == sg.ERR_CUDA
+    def ls(M=16, N=1000, K=256, ws=FAKE, wsb=1 << 30):
+        return L.gemm_bf16_logsoftmax(M, N, K, FAKE, sg.BF16, sg.ROW_MAJOR, K, FAKE, sg.ROW_MAJOR, N, None, 0,
+                                      FAKE, N, ws, wsb, None)
+    assert ls(M=0) == sg.OK
+    assert ls() == sg.ERR_CUDA                                # workspace size needs a device
+    assert L.smgemm_logsoftmax_workspace_size(0, 10, 10) == 0
+
+
 def _grouped(shapes, ab=sg.BF16, la=sg.ROW_MAJOR, lb=sg.ROW_MAJOR, ptr=FAKE, ws=FAKE, wsb=None, act=0,
              c_dt=sg.BF16, ld_pad=0):
     import ctypes as C
