@@ -82,3 +82,19 @@ def test_fp8out_feeds_fp8_gemm(cuda_device):
     ref, acc = oracle.gemm_fp8(Hq.cpu().numpy(), Hs.cpu().numpy(), W2q.cpu().numpy(), W2s.cpu().numpy(),
                                out_dtype=oracle.BF16, want_absacc=True)
     check_tolerance(Y.float().cpu().numpy(), ref, acc, torch.bfloat16, what="FP8 GEMM on fused codes")
+
+
+def test_fp8out_col_major_a_ragged_k_integer_exact(cuda_device):
+    """Column-major A (the MN-major operand path) and K not a multiple of the 64-wide
+    K-block: still exact on integer inputs."""
+    M, N, K = 264, 384, 200
+    A = torch.from_numpy(synth.integers(64, 0, (M, K), -3, 3)).to(torch.bfloat16)
+    B = torch.from_numpy(synth.integers(64, 1, (K, N), -3, 3)).to(torch.bfloat16)
+    Q, S = sg.gemm_bf16_fp8out(A.t().contiguous().cuda().t(), B.cuda())
+    assert sg.check() == sg.OK
+    a, ad = orc_view(A)
+    b, bd = orc_view(B)
+    Z = oracle.gemm(a, b, a_dtype=ad, b_dtype=bd, out_dtype=oracle.F32).astype(np.float32)
+    Qr, Sr = oracle.quant_1x128(Z)
+    assert np.array_equal(S.cpu().numpy().view(np.uint32), Sr.view(np.uint32))
+    assert np.array_equal(Q.cpu().numpy(), Qr)

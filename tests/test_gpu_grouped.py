@@ -94,3 +94,25 @@ def test_grouped_experts_full_size(cuda_device):
                                want_absacc=True)
         check_tolerance(outs[g].float().cpu().numpy()[np.ix_(rows, cols)], ref, acc, torch.bfloat16,
                         what=f"expert {g}")
+
+
+def test_grouped_many_small_groups(cuda_device):
+    """40 groups of assorted small shapes (many below one tile, some empty): every tile
+    of every group must land in its own group's output."""
+    rng = np.random.RandomState(7)
+    shapes = [(int(rng.choice([0, 1, 8, 64, 136, 256, 300])), int(rng.choice([8, 40, 128, 264])),
+               int(rng.choice([16, 64, 200]))) for _ in range(40)]
+    As, Bs, Ah, Bh = [], [], [], []
+    for g, (M, N, K) in enumerate(shapes):
+        a = to_dtype(synth.normal(43, 2 * g, (M, K)), torch.bfloat16)
+        b = to_dtype(synth.normal(43, 2 * g + 1, (K, N), 0.1), torch.bfloat16)
+        Ah.append(a); Bh.append(b); As.append(a.cuda()); Bs.append(b.cuda())
+    outs = sg.gemm_bf16_grouped(As, Bs, out_dtype=torch.float32)
+    assert sg.check() == sg.OK
+    for g, (M, N, K) in enumerate(shapes):
+        if M == 0:
+            continue
+        a, ad = orc_view(Ah[g])
+        b, bd = orc_view(Bh[g])
+        ref, acc = oracle.gemm(a, b, a_dtype=ad, b_dtype=bd, out_dtype=oracle.F32, want_absacc=True)
+        check_tolerance(outs[g].cpu().numpy(), ref, acc, torch.float32, what=f"group {g} {M}x{N}x{K}")

@@ -70,3 +70,15 @@ def test_logsoftmax_lm_head_full_size(cuda_device):
     p = torch.exp(out.double()).sum(dim=1)
     assert torch.allclose(p, torch.ones_like(p), atol=1e-4)
     _check(out, X, W, None, rows=np.array([0, 15]))
+
+
+def test_logsoftmax_k0_is_log_softmax_of_bias(cuda_device):
+    """K = 0: the logits are the bias alone, so every row is log_softmax(bias)."""
+    M, N = 5, 1000
+    b = to_dtype(synth.normal(53, 0, (N,), 2.0), torch.float32)
+    X = torch.empty((M, 0), dtype=torch.bfloat16, device="cuda")
+    W = torch.empty((0, N), dtype=torch.bfloat16, device="cuda")
+    out = sg.gemm_bf16_logsoftmax(X, W, bias=b.cuda())
+    assert sg.check() == sg.OK
+    ref, _ = oracle.log_softmax_rows(np.tile(b.numpy().astype(np.float64), (M, 1)))
+    assert np.allclose(out.cpu().numpy(), ref, rtol=0, atol=1e-5)
