@@ -467,8 +467,18 @@ smgemm_status gemm_bf16_logsoftmax(int64_t M, int64_t N, int64_t K, const void* 
                                                stream));
 }
 
+// Group table, then (when the device is known) room for splitting a ragged last wave:
+// one 2 x 128 x 256-float partial per cluster and two counters per split tile.
+size_t grouped_table_bytes(int G) { return (static_cast<size_t>(G) * sizeof(GroupDesc) + 64 + 255) / 256 * 256; }
+size_t grouped_split_bytes(int clusters) {
+  return static_cast<size_t>(clusters) * 2 * 128 * 256 * sizeof(float) + static_cast<size_t>(clusters) * 2 * sizeof(int);
+}
+
 size_t smgemm_grouped_workspace_size(int G) {
-  return G > 0 ? static_cast<size_t>(G) * sizeof(GroupDesc) + 64 : 0;
+  if (G <= 0) return 0;
+  DevInfo d;
+  const int P = current_device(d) == SMGEMM_OK ? grouped_max_clusters() : 0;
+  return grouped_table_bytes(G) + (P > 0 ? grouped_split_bytes(P) : 0);
 }
 
 smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const int64_t* K, const void* const* A,
@@ -500,7 +510,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
         return SMGEMM_ERR_ALIGNMENT;
     }
   }
-  if (workspace == nullptr || workspace_bytes < smgemm_grouped_workspace_size(G)) return SMGEMM_ERR_WORKSPACE;
+  if (workspace == nullptr || workspace_bytes < grouped_table_bytes(G)) return SMGEMM_ERR_WORKSPACE;
   DevInfo d;
   if (current_device(d) != SMGEMM_OK) return SMGEMM_ERR_CUDA;
   const CUtensorMapDataType dt =
@@ -558,9 +568,39 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   p.b_mn_major = b_mn ? 1 : 0;
   p.idesc = idesc_f32acc(fmt, fmt, a_mn ? 1u : 0u, b_mn ? 1u : 0u, 256, 256);
   p.wait_limit_cycles = wait_limit();
-  const int clusters = static_cast<int>(std::min<long long>(tiles, clusters_max));
-  std::snprintf(g_last_config, sizeof(g_last_config), "path=grouped groups=%d tiles=%lld grid=%d tile=128x256", G,
-                tiles, clusters);
+  // A ragged last wave (R = tiles mod P tiles for P co-resident clusters; all tiles when
+  // there are fewer than P) is split along K into S pieces when every tail tile keeps at
+  // least 8 K-blocks per piece and the workspace holds the partials.
+  const int P = clusters_max;
+  const long long R = tiles % P;
+  int S = 0;
+  if (R > 0 && env_ll("SMGEMM_SCHED_GROUPED_SPLIT", 1) != 0) {
+    int min_kb = 1 << 30;
+    long long left = R;
+    for (int g = G - 1; g >= 0 && left > 0; --g) {
+      const GroupDesc& e = table[static_cast<size_t>(g)];
+      const long long t = static_cast<long long>(e.m_tiles) * e.n_tiles;
+      if (t == 0) continue;
+      min_kb = std::min(min_kb, e.kb_total);
+      left -= t;
+    }
+    S = static_cast<int>(std::min<long long>(P / R, min_kb / 8));
+    if (S < 2 || workspace_bytes < grouped_table_bytes(G) + grouped_split_bytes(static_cast<int>(R * S))) S = 0;
+  }
+  int clusters = static_cast<int>(std::min<long long>(tiles, P));
+  if (S >= 2) {
+    if (tiles < P) clusters = static_cast<int>(R * S);
+    uint8_t* split_base = static_cast<uint8_t*>(workspace) + grouped_table_bytes(G);
+    p.split_tiles = R;
+    p.splits = S;
+    p.slots = reinterpret_cast<float*>(split_base);
+    p.counters = reinterpret_cast<int*>(split_base + static_cast<size_t>(R * S) * 2 * 128 * 256 * sizeof(float));
+    if (cudaMemsetAsync(p.counters, 0, static_cast<size_t>(R) * 2 * sizeof(int), stream) != cudaSuccess)
+      return launch_status(cudaGetLastError());
+  }
+  std::snprintf(g_last_config, sizeof(g_last_config),
+                "path=grouped groups=%d tiles=%lld grid=%d tile=128x256 split_tiles=%lld splits=%d", G, tiles, clusters,
+                S >= 2 ? R : 0LL, S >= 2 ? S : 0);
   if (env_ll("SMGEMM_LOG", 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
   return launch_status(launch_gemm_grouped(p, clusters, stream));
 }

@@ -16,7 +16,9 @@
 // Roles as in gemm_tc16_pair.cu: warp 0 TMA producer and warp 1 MMA issuer (warp-wide
 // loops, one elected lane issues; MMA on the rank-0 CTA only), warp 2 TMEM allocator,
 // warps 4-7 epilogue (each CTA drains its own 128 rows of the two TMEM accumulators).
-// No stream-K: each tile is one work unit.
+// When the tiles leave a ragged last wave (R = T mod P tiles for P clusters), those R
+// tiles are split along K into S pieces (R S <= P) that run side by side; each piece's
+// partial goes to a workspace slot and the last piece to finish sums them in order.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -57,12 +59,57 @@ __device__ __forceinline__ int locate(const GroupedParams& p, long long t, int& 
 }
 }  // namespace
 
+// One unit of work: tile `tile` of group `g` over K-blocks [kb0, kb1); unit >= 0 marks a
+// piece of a split tail tile (its partial goes to workspace slot `unit`).
+struct GItem {
+  long long tile;
+  int g, mt, nt, kb0, kb1, unit;
+};
+
+// Work of cluster c: its piece of the split tail (if any) first, so the tail's fix-up
+// overlaps later tiles, then the data-parallel tiles c, c + P, ... below T - R.
+struct GIter {
+  int c, P;
+  long long next_dp;
+  bool unit_pending;
+
+  __device__ __forceinline__ void init(const GroupedParams& p, int cluster, int nclusters) {
+    c = cluster;
+    P = nclusters;
+    next_dp = cluster;
+    unit_pending = p.split_tiles > 0 && cluster < p.split_tiles * p.splits;
+  }
+  __device__ __forceinline__ bool next(const GroupedParams& p, GItem& it) {
+    if (unit_pending) {
+      unit_pending = false;
+      it.tile = p.total_tiles - p.split_tiles + c / p.splits;
+      it.g = locate(p, it.tile, it.mt, it.nt);
+      const int kbn = p.groups[it.g].kb_total, piece = c % p.splits;
+      it.kb0 = static_cast<int>(static_cast<long long>(piece) * kbn / p.splits);
+      it.kb1 = static_cast<int>(static_cast<long long>(piece + 1) * kbn / p.splits);
+      it.unit = c;
+      return true;
+    }
+    if (next_dp < p.total_tiles - p.split_tiles) {
+      it.tile = next_dp;
+      it.g = locate(p, it.tile, it.mt, it.nt);
+      it.kb0 = 0;
+      it.kb1 = p.groups[it.g].kb_total;
+      it.unit = -1;
+      next_dp += P;
+      return true;
+    }
+    return false;
+  }
+};
+
 template <int BK, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_constant__ GroupedParams p) {
   constexpr int A_BYTES = 128 * BK * 2;
   constexpr int B_BYTES = 128 * BK * 2;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr int KSTEPS = BK / 16;
+  constexpr int SLOT = 128 * kTileN;  // floats of one CTA's partial tile
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -76,6 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
   uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  volatile int* reduce_flag = reinterpret_cast<volatile int*>(misc + 8);
 
   const uint32_t warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();
@@ -113,18 +161,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
     long long issued = 0;
     int last_g = -1;
     bool ok = true;
-    for (long long t = cluster; ok && t < p.total_tiles; t += nclusters) {
-      int mt, nt;
-      const int g = locate(p, t, mt, nt);
-      const GroupDesc* d = p.groups + g;
-      if (g != last_g && elect_one()) {
+    GIter wi;
+    wi.init(p, cluster, nclusters);
+    GItem it;
+    while (ok && wi.next(p, it)) {
+      const GroupDesc* d = p.groups + it.g;
+      if (it.g != last_g && elect_one()) {
         tensormap_acquire(&d->tm_a);
         tensormap_acquire(&d->tm_b);
       }
-      last_g = g;
-      const int a_row = mt * 256 + static_cast<int>(rank) * 128;
-      const int b_row = nt * kTileN + static_cast<int>(rank) * 128;
-      for (int kb = 0; kb < d->kb_total; ++kb) {
+      last_g = it.g;
+      const int a_row = it.mt * 256 + static_cast<int>(rank) * 128;
+      const int b_row = it.nt * kTileN + static_cast<int>(rank) * 128;
+      for (int kb = it.kb0; kb < it.kb1; ++kb) {
         const bool w = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         const uint32_t sa = smem_base + stage * STAGE_BYTES;
@@ -154,15 +203,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
     uint32_t phase = 0;
     int local = 0;
     bool ok = true;
-    for (long long t = cluster; ok && t < p.total_tiles; t += nclusters) {
-      int mt, nt;
-      const int kbn = p.groups[locate(p, t, mt, nt)].kb_total;
+    GIter wi;
+    wi.init(p, cluster, nclusters);
+    GItem it;
+    while (ok && wi.next(p, it)) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, limit))) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * kTileN;
-      for (int kb = 0; kb < kbn; ++kb) {
+      for (int kb = it.kb0; kb < it.kb1; ++kb) {
         if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, abort_flag, limit))) { ok = false; break; }
         tc_fence_after();
         const uint32_t sa = smem_base + stage * STAGE_BYTES;
@@ -171,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
 #pragma unroll
           for (int k = 0; k < KSTEPS; ++k) {
             umma_f16_pair(d_tmem, operand_desc<128, BK>(sa, p.a_mn_major, k),
-                          operand_desc<128, BK>(sb, p.b_mn_major, k), p.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                          operand_desc<128, BK>(sb, p.b_mn_major, k), p.idesc, (kb > it.kb0 || k > 0) ? 1u : 0u);
           }
           umma_commit_pair(empty_bar(stage), 0x3);
         }
@@ -192,18 +242,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
     const int q = warp & 3;
     const int r_local = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const int epi_tid = threadIdx.x - kEpiWarp0 * 32;
     int local = 0;
     bool dead = false;
-    for (long long t = cluster; t < p.total_tiles; t += nclusters) {
-      int mt, nt;
-      const GroupDesc* d = p.groups + locate(p, t, mt, nt);
+    GIter wi;
+    wi.init(p, cluster, nclusters);
+    GItem it;
+    while (wi.next(p, it)) {
+      const GroupDesc* d = p.groups + it.g;
       const EpiArgs e{d->M, d->N, d->bias, p.bias_dtype, p.act, d->C, p.c_dtype, d->ldc};
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!dead) dead = !mbar_wait(tfull_bar(acc), acc_phase, abort_flag, limit);
       dead = __any_sync(0xffffffffu, dead);
-      const int row = mt * 256 + static_cast<int>(rank) * 128 + r_local;
+      const int row = it.mt * 256 + static_cast<int>(rank) * 128 + r_local;
       const uint32_t tacc = tmem_base + lane_addr + acc * kTileN;
+      const bool split = it.unit >= 0;
+      float* my_slot = split ? p.slots + (static_cast<size_t>(it.unit) * 2 + rank) * SLOT : nullptr;
       if (!dead) {
         tc_fence_after();
 #pragma unroll 1
@@ -214,11 +269,41 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          epi_row32(e, row, nt * kTileN + c * 32, v);
+          if (split) slot_store<32>(my_slot, r_local, c * 32, v);
+          else epi_row32(e, row, it.nt * kTileN + c * 32, v);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+      }
+      if (split) {
+        // The last of the tile's S pieces (per rank) sums them in piece order (= K order)
+        // and runs the epilogue: deterministic, and no CTA waits for another.
+        const long long r_tail = it.tile - (p.total_tiles - p.split_tiles);
+        __threadfence();
+        named_barrier_sync(1, 128);
+        if (epi_tid == 0) {
+          const bool any_dead = *abort_flag != 0;
+          const int old = any_dead ? -1 : atomicAdd(p.counters + r_tail * 2 + rank, 1);
+          *reduce_flag = (!any_dead && old == p.splits - 1);
+        }
+        named_barrier_sync(1, 128);
+        if (*reduce_flag) {
+          __threadfence();
+#pragma unroll 1
+          for (int c = 0; c < kTileN / 32; ++c) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+#pragma unroll 1
+            for (int pc = 0; pc < p.splits; ++pc) {
+              const float* src = p.slots + ((r_tail * p.splits + pc) * 2 + rank) * static_cast<size_t>(SLOT);
+              slot_accumulate<32>(src, r_local, c * 32, v);
+            }
+            epi_row32(e, row, it.nt * kTileN + c * 32, v);
+          }
+        }
+        named_barrier_sync(1, 128);
       }
       ++local;
     }
@@ -233,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
 
 namespace {
 constexpr int kBK = 64, kStages = 6;
-constexpr int kSmem = 1024 + kStages * (2 * 128 * kBK * 2) + 8 * (2 * kStages + 5) + 16;
+constexpr int kSmem = 1024 + kStages * (2 * 128 * kBK * 2) + 8 * (2 * kStages + 5) + 16;  // + misc words
 static_assert(kSmem <= 232448, "shared memory budget");
 
 cudaError_t prepare() {

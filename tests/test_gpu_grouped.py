@@ -116,3 +116,26 @@ def test_grouped_many_small_groups(cuda_device):
         b, bd = orc_view(Bh[g])
         ref, acc = oracle.gemm(a, b, a_dtype=ad, b_dtype=bd, out_dtype=oracle.F32, want_absacc=True)
         check_tolerance(outs[g].cpu().numpy(), ref, acc, torch.float32, what=f"group {g} {M}x{N}x{K}")
+
+
+def test_grouped_split_tail_few_tiles(cuda_device):
+    """Three single-tile groups with K = 4096 leave most clusters idle, so each tile is
+    split along K into pieces summed in fixed order: checked against the oracle and
+    bit-identical across calls."""
+    shapes = [(256, 256, 4096), (200, 136, 4096), (64, 256, 4096)]
+    As, Bs, Ah, Bh = [], [], [], []
+    for g, (M, N, K) in enumerate(shapes):
+        a = to_dtype(synth.normal(44, 2 * g, (M, K)), torch.bfloat16)
+        b = to_dtype(synth.normal(44, 2 * g + 1, (K, N), 0.02), torch.bfloat16)
+        Ah.append(a); Bh.append(b); As.append(a.cuda()); Bs.append(b.cuda())
+    o1 = sg.gemm_bf16_grouped(As, Bs, out_dtype=torch.float32)
+    cfg = sg.last_config()
+    o2 = sg.gemm_bf16_grouped(As, Bs, out_dtype=torch.float32)
+    assert sg.check() == sg.OK
+    assert "splits=" in cfg and "splits=0" not in cfg, cfg
+    for g in range(len(shapes)):
+        a, ad = orc_view(Ah[g])
+        b, bd = orc_view(Bh[g])
+        ref, acc = oracle.gemm(a, b, a_dtype=ad, b_dtype=bd, out_dtype=oracle.F32, want_absacc=True)
+        check_tolerance(o1[g].cpu().numpy(), ref, acc, torch.float32, what=f"group {g}")
+        assert torch.equal(o1[g], o2[g])
