@@ -6,7 +6,9 @@
 //  - skinny M (the thin-and-tall LM-head / decode shape of "为什么我们要死磕GEMM",
 //    kwkr.cn, sections 2.2 and 7.2): swap-AB, the weight supplies the 128 MMA rows
 //    and the few tokens are the MMA N (16..64), so the tensor core streams the
-//    weight once; the epilogue writes the transposed accumulator.
+//    weight once; the epilogue writes the transposed accumulator. For the LM head
+//    fused with its log-softmax (same page, section 7.2) the epilogue also reduces
+//    each 128-column tile of every token row to (max, sum of exp) partials.
 //
 // Warp roles (256 threads): warp 0 = TMA producer, warp 1 = MMA issuer, warp 2 =
 // TMEM allocator, warp 3 idle, warps 4..7 = epilogue (warp w reads TMEM lanes
