@@ -17,6 +17,7 @@
 #include <vector>
 
 #include "../../include/smgemm.h"
+#include "grouped.h"
 #include "kernels.h"
 
 using namespace smg;
@@ -588,21 +589,22 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
     if (S < 2 || workspace_bytes < grouped_table_bytes(G) + grouped_split_bytes(static_cast<int>(R * S))) S = 0;
   }
   int clusters = static_cast<int>(std::min<long long>(tiles, P));
+  GroupedSplit sp{0, 0, nullptr, nullptr};
   if (S >= 2) {
     if (tiles < P) clusters = static_cast<int>(R * S);
     uint8_t* split_base = static_cast<uint8_t*>(workspace) + grouped_table_bytes(G);
-    p.split_tiles = R;
-    p.splits = S;
-    p.slots = reinterpret_cast<float*>(split_base);
-    p.counters = reinterpret_cast<int*>(split_base + static_cast<size_t>(R * S) * 2 * 128 * 256 * sizeof(float));
-    if (cudaMemsetAsync(p.counters, 0, static_cast<size_t>(R) * 2 * sizeof(int), stream) != cudaSuccess)
+    sp.split_tiles = R;
+    sp.splits = S;
+    sp.slots = reinterpret_cast<float*>(split_base);
+    sp.counters = reinterpret_cast<int*>(split_base + static_cast<size_t>(R * S) * 2 * 128 * 256 * sizeof(float));
+    if (cudaMemsetAsync(sp.counters, 0, static_cast<size_t>(R) * 2 * sizeof(int), stream) != cudaSuccess)
       return launch_status(cudaGetLastError());
   }
   std::snprintf(g_last_config, sizeof(g_last_config),
                 "path=grouped groups=%d tiles=%lld grid=%d tile=128x256 split_tiles=%lld splits=%d", G, tiles, clusters,
                 S >= 2 ? R : 0LL, S >= 2 ? S : 0);
   if (env_ll("SMGEMM_LOG", 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
-  return launch_status(launch_gemm_grouped(p, clusters, stream));
+  return launch_status(launch_gemm_grouped_split(p, sp, clusters, stream));
 }
 
 smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_t* Aq, const float* sa,

@@ -23,6 +23,7 @@
 #include <cuda_fp16.h>
 
 #include "epilogue.cuh"
+#include "grouped.h"
 #include "kernels.h"
 #include "operands.cuh"
 #include "sm100.cuh"
@@ -73,24 +74,26 @@ struct GIter {
   long long next_dp;
   bool unit_pending;
 
-  __device__ __forceinline__ void init(const GroupedParams& p, int cluster, int nclusters) {
+  __device__ __forceinline__ void init(const GroupedParams& p, const GroupedSplit& sp, int cluster,
+                                       int nclusters) {
     c = cluster;
     P = nclusters;
     next_dp = cluster;
-    unit_pending = p.split_tiles > 0 && cluster < p.split_tiles * p.splits;
+    unit_pending = sp.split_tiles > 0 && cluster < sp.split_tiles * sp.splits;
+    (void)p;
   }
-  __device__ __forceinline__ bool next(const GroupedParams& p, GItem& it) {
+  __device__ __forceinline__ bool next(const GroupedParams& p, const GroupedSplit& sp, GItem& it) {
     if (unit_pending) {
       unit_pending = false;
-      it.tile = p.total_tiles - p.split_tiles + c / p.splits;
+      it.tile = p.total_tiles - sp.split_tiles + c / sp.splits;
       it.g = locate(p, it.tile, it.mt, it.nt);
-      const int kbn = p.groups[it.g].kb_total, piece = c % p.splits;
-      it.kb0 = static_cast<int>(static_cast<long long>(piece) * kbn / p.splits);
-      it.kb1 = static_cast<int>(static_cast<long long>(piece + 1) * kbn / p.splits);
+      const int kbn = p.groups[it.g].kb_total, piece = c % sp.splits;
+      it.kb0 = static_cast<int>(static_cast<long long>(piece) * kbn / sp.splits);
+      it.kb1 = static_cast<int>(static_cast<long long>(piece + 1) * kbn / sp.splits);
       it.unit = c;
       return true;
     }
-    if (next_dp < p.total_tiles - p.split_tiles) {
+    if (next_dp < p.total_tiles - sp.split_tiles) {
       it.tile = next_dp;
       it.g = locate(p, it.tile, it.mt, it.nt);
       it.kb0 = 0;
@@ -104,7 +107,8 @@ struct GIter {
 };
 
 template <int BK, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_constant__ GroupedParams p) {
+__global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_constant__ GroupedParams p,
+                                                                   const __grid_constant__ GroupedSplit sp) {
   constexpr int A_BYTES = 128 * BK * 2;
   constexpr int B_BYTES = 128 * BK * 2;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -162,9 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
     int last_g = -1;
     bool ok = true;
     GIter wi;
-    wi.init(p, cluster, nclusters);
+    wi.init(p, sp, cluster, nclusters);
     GItem it;
-    while (ok && wi.next(p, it)) {
+    while (ok && wi.next(p, sp, it)) {
       const GroupDesc* d = p.groups + it.g;
       if (it.g != last_g && elect_one()) {
         tensormap_acquire(&d->tm_a);
@@ -204,9 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
     int local = 0;
     bool ok = true;
     GIter wi;
-    wi.init(p, cluster, nclusters);
+    wi.init(p, sp, cluster, nclusters);
     GItem it;
-    while (ok && wi.next(p, it)) {
+    while (ok && wi.next(p, sp, it)) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, limit))) break;
@@ -246,9 +250,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
     int local = 0;
     bool dead = false;
     GIter wi;
-    wi.init(p, cluster, nclusters);
+    wi.init(p, sp, cluster, nclusters);
     GItem it;
-    while (wi.next(p, it)) {
+    while (wi.next(p, sp, it)) {
       const GroupDesc* d = p.groups + it.g;
       const EpiArgs e{d->M, d->N, d->bias, p.bias_dtype, p.act, d->C, p.c_dtype, d->ldc};
       const int acc = local & 1;
@@ -258,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
       const int row = it.mt * 256 + static_cast<int>(rank) * 128 + r_local;
       const uint32_t tacc = tmem_base + lane_addr + acc * kTileN;
       const bool split = it.unit >= 0;
-      float* my_slot = split ? p.slots + (static_cast<size_t>(it.unit) * 2 + rank) * SLOT : nullptr;
+      float* my_slot = split ? sp.slots + (static_cast<size_t>(it.unit) * 2 + rank) * SLOT : nullptr;
       if (!dead) {
         tc_fence_after();
 #pragma unroll 1
@@ -279,13 +283,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
       if (split) {
         // The last of the tile's S pieces (per rank) sums them in piece order (= K order)
         // and runs the epilogue: deterministic, and no CTA waits for another.
-        const long long r_tail = it.tile - (p.total_tiles - p.split_tiles);
+        const long long r_tail = it.tile - (p.total_tiles - sp.split_tiles);
         __threadfence();
         named_barrier_sync(1, 128);
         if (epi_tid == 0) {
           const bool any_dead = *abort_flag != 0;
-          const int old = any_dead ? -1 : atomicAdd(p.counters + r_tail * 2 + rank, 1);
-          *reduce_flag = (!any_dead && old == p.splits - 1);
+          const int old = any_dead ? -1 : atomicAdd(sp.counters + r_tail * 2 + rank, 1);
+          *reduce_flag = (!any_dead && old == sp.splits - 1);
         }
         named_barrier_sync(1, 128);
         if (*reduce_flag) {
@@ -296,8 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.0f;
 #pragma unroll 1
-            for (int pc = 0; pc < p.splits; ++pc) {
-              const float* src = p.slots + ((r_tail * p.splits + pc) * 2 + rank) * static_cast<size_t>(SLOT);
+            for (int pc = 0; pc < sp.splits; ++pc) {
+              const float* src = sp.slots + ((r_tail * sp.splits + pc) * 2 + rank) * static_cast<size_t>(SLOT);
               slot_accumulate<32>(src, r_local, c * 32, v);
             }
             epi_row32(e, row, it.nt * kTileN + c * 32, v);
@@ -360,14 +364,19 @@ int grouped_max_clusters() {
 
 int grouped_bk() { return kBK; }
 
-cudaError_t launch_gemm_grouped(const GroupedParams& p, int clusters, cudaStream_t stream) {
+cudaError_t launch_gemm_grouped_split(const GroupedParams& p, const GroupedSplit& sp, int clusters,
+                                      cudaStream_t stream) {
   cudaError_t e = prepare();
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = config(clusters, stream, attr);
-  e = cudaLaunchKernelEx(&cfg, gemm_grouped_kernel<kBK, kStages>, p);
+  e = cudaLaunchKernelEx(&cfg, gemm_grouped_kernel<kBK, kStages>, p, sp);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_grouped(const GroupedParams& p, int clusters, cudaStream_t stream) {
+  return launch_gemm_grouped_split(p, GroupedSplit{0, 0, nullptr, nullptr}, clusters, stream);
 }
 
 unsigned take_error_word_grouped() { return take_error_word(); }

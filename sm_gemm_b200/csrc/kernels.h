@@ -76,10 +76,6 @@ struct GroupedParams {
   int a_mn_major, b_mn_major;
   uint32_t idesc;
   unsigned long long wait_limit_cycles;
-  long long split_tiles;    // R: the last R tiles are split along K (0: none)
-  int splits;               // S pieces per split tile
-  float* slots;             // [R * S][2 ranks][128][256] float partials
-  int* counters;            // [R][2], zeroed before the launch
 };
 
 cudaError_t launch_gemm_grouped(const GroupedParams& p, int clusters, cudaStream_t stream);
