@@ -184,3 +184,21 @@ def test_load_fp16_and_bf16_decoding():
     ref = b.to(torch.float64).numpy()
     for i in range(0, 1000, 7):
         assert oracle.load_elem(bits, oracle.BF16, i) == ref[i]
+
+
+def test_encode_exhaustive_against_torch():
+    """Every non-negative FP32 value up to 448 (all 1,138,753,537 bit patterns from +0 to
+    448.0), encoded by the oracle and by torch's independent float8_e4m3fn cast (RNE),
+    plus the sign-flipped patterns of a strided subset."""
+    top = int(np.array(448.0, dtype=np.float32).view(np.uint32))
+    step = 1 << 25
+    for lo in range(0, top + 1, step):
+        bits = np.arange(lo, min(lo + step, top + 1), dtype=np.uint32)
+        y = bits.view(np.float32)
+        ref = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        got = oracle.e4m3_encode(y)
+        bad = np.flatnonzero(got != ref)
+        assert bad.size == 0, f"{bad.size} mismatches from {y[bad[0]]!r}: {got[bad[0]]:#x} vs {ref[bad[0]]:#x}"
+    neg = -(np.arange(0, top + 1, 997, dtype=np.uint32).view(np.float32))
+    ref = torch.from_numpy(neg).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(neg), ref)
