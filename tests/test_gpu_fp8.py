@@ -136,6 +136,41 @@ def test_quant_division_edge_scales(cuda_device):
     assert np.array_equal(Q, Qr)
 
 
+def test_quant_encoder_every_fp32_value_up_to_448(cuda_device):
+    """The device E4M3 encoder on every FP32 bit pattern of magnitude <= 448, both signs
+    (2,277,507,074 values). Each 1x128 group holds 448 in its first slot, so its scale is
+    448 / 448 = 1 exactly, x / s = x, and every code must be the oracle's encoding of x
+    itself. Inputs are an enumeration of bit patterns built on the device; the codes come
+    back in chunks of 127 * 2^20 values and are checked against the oracle's encoder."""
+    assert oracle.quant_1x128(np.float32([[448.0, 1.0]]))[1][0, 0] == np.float32(1.0)
+    top = int(np.array(448.0, dtype=np.float32).view(np.uint32))
+    rows = 1 << 20
+    per = rows * 127
+    X = torch.empty((rows, 128), dtype=torch.float32, device="cuda")
+    body = torch.empty(per, dtype=torch.float32, device="cuda")
+    for sign in (0, 1):
+        for lo in range(0, top + 1, per):
+            n = min(per, top + 1 - lo)
+            bits = torch.arange(lo, lo + n, dtype=torch.int64, device="cuda")
+            if sign:
+                bits -= 1 << 31  # the int32 of the pattern with the sign bit set
+            body.zero_()
+            body[:n] = bits.to(torch.int32).view(torch.float32)
+            X[:, 0] = 448.0
+            X[:, 1:] = body.view(rows, 127)
+            Q, S = sg.quantize_fp8_blockwise(X, 1)
+            assert sg.check() == sg.OK
+            assert bool((S == 1.0).all()) and bool((Q[:, 0] == 0x7E).all())
+            got = Q[:, 1:].reshape(-1)[:n].cpu().numpy()
+            y = np.arange(lo, lo + n, dtype=np.uint32)
+            if sign:
+                y |= np.uint32(1 << 31)
+            ref = oracle.e4m3_encode(y.view(np.float32))
+            bad = np.flatnonzero(got != ref)
+            assert bad.size == 0, f"{bad.size} codes differ, first for bits {y[bad[0]]:#010x}: " \
+                f"{got[bad[0]]:#04x} vs {ref[bad[0]]:#04x}"
+
+
 def _quantised_problem(M, N, K, seed):
     A = synth.normal_with_outliers(seed, 0, (M, K))
     B = synth.normal_with_outliers(seed, 1, (K, N))

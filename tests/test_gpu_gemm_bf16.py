@@ -189,6 +189,50 @@ def test_skinny_integer_exact_with_bias_act(cuda_device, M):
     check_tolerance(got, ref, acc, torch.bfloat16, what="skinny epilogue")
 
 
+# ------------------------------------------------------------------ activation accuracy
+
+def _act_points(n=8192):
+    """n FP32 activation inputs: a dense sweep of [-20, 20] plus zeros, tiny and large
+    magnitudes (where exp overflows and tanh saturates)."""
+    special = np.float32([0.0, -0.0, 1e-30, -1e-30, 1e-6, -1e-6, 0.5, -0.5, 1.0, -1.0, 40.0, -40.0,
+                          60.0, -60.0, -87.0, -89.0, 100.0, -100.0])
+    sweep = np.linspace(-20.0, 20.0, n - special.size, dtype=np.float32)
+    return np.concatenate([special, sweep]).astype(np.float32)
+
+
+@pytest.mark.parametrize("act", ["gelu_tanh", "silu"])
+@pytest.mark.parametrize("M", [16, 128])
+@pytest.mark.parametrize("offset", [0, 1])
+def test_epilogue_activation_accuracy(cuda_device, act, M, offset):
+    """The epilogue's activation against the oracle's FP64 one, with A = 0 so that every
+    output is act(bias[n]) over 8192 FP32 inputs. The GEMM epilogues evaluate tanh with
+    tanh.approx.f32 (relative error below 2^-10.9) and exp with __expf (error 2 + 1.17|x|
+    ulp), so the stated bounds are |GeLU_dev - GeLU| <= 2^-10 |x| (the tanh error times
+    x/2, with a factor 4 of margin) and |SiLU_dev - SiLU| <= 2^-15 |SiLU| + 1e-30 (the
+    absolute floor covers exp overflow at x < -88, where the true value is below 1e-36).
+    M = 16 runs the swap-AB (skinny) epilogue, M = 128 the tile epilogue; offset = 1
+    misaligns the bias so that the scalar bias loads run instead of the 16-byte ones."""
+    x = _act_points()
+    N = x.size
+    buf = torch.zeros(N + 4, dtype=torch.float32, device="cuda")  # 256-byte aligned start
+    buf[offset:offset + N] = torch.from_numpy(x).cuda()
+    bias = buf[offset:offset + N]
+    A = torch.zeros((M, 64), dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros((N, 64), dtype=torch.bfloat16, device="cuda").t()
+    out = sg.gemm_bf16(A, B, bias=bias, act=act, out_dtype=torch.float32)
+    assert sg.check() == sg.OK
+    got = out.cpu().numpy()
+    assert (got.view(np.uint32) == got[0].view(np.uint32)).all(), "rows differ"
+    which = ORC_ACT[act]
+    ref = np.array([oracle.act(float(v), which) for v in x])
+    err = np.abs(got[0].astype(np.float64) - ref)
+    xa = np.abs(x.astype(np.float64))
+    bound = 2.0 ** -10 * xa if act == "gelu_tanh" else 2.0 ** -15 * np.abs(ref) + 1e-30
+    bad = np.flatnonzero(err > bound)
+    assert bad.size == 0, f"{act}: {bad.size} beyond the bound, first x={x[bad[0]]!r} " \
+        f"got {got[0, bad[0]]!r} ref {ref[bad[0]]!r}"
+
+
 # ------------------------------------------------------------------ degenerate shapes
 
 def test_k_zero_writes_activation_of_bias(cuda_device):
