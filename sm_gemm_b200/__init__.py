@@ -38,6 +38,8 @@ class SmgemmError(RuntimeError):
 def lib():
     """The loaded C library (built in-tree by ``python -m sm_gemm_b200.build``)."""
     global _lib
+    if _lib is not None:
+        return _lib
     with _lock:
         if _lib is None:
             if not os.path.exists(LIB_PATH):
@@ -87,19 +89,26 @@ def _torch():
     return torch
 
 
+_DTYPES: dict = {}
+
+
 def _dtype_code(dt) -> int:
-    torch = _torch()
-    return {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}[dt]
+    if not _DTYPES:
+        torch = _torch()
+        _DTYPES.update({torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16})
+    return _DTYPES[dt]
 
 
 def _layout(t, name):
     """(layout, leading dimension) of a 2-D tensor; one of its strides must be 1."""
-    if t.dim() != 2:
+    st = t.stride()
+    if len(st) != 2:
         raise ValueError(f"{name} must be 2-D")
-    if t.stride(1) == 1 and (t.shape[0] <= 1 or t.stride(0) >= t.shape[1]):
-        return ROW_MAJOR, max(t.stride(0), t.shape[1])
-    if t.stride(0) == 1:
-        return COL_MAJOR, max(t.stride(1), t.shape[0])
+    (rows, cols), (s0, s1) = t.shape, st
+    if s1 == 1 and (rows <= 1 or s0 >= cols):
+        return ROW_MAJOR, max(s0, cols)
+    if s0 == 1:
+        return COL_MAJOR, max(s1, rows)
     raise ValueError(f"{name} must have a unit stride in one dimension")
 
 
@@ -115,13 +124,27 @@ def _layout_as(t, name, want):
     raise ValueError(f"{name} cannot be read in the layout the other groups use")
 
 
+_current_stream = None
+
+
 def _stream(stream):
-    torch = _torch()
+    """The cudaStream_t handle of `stream` (a torch stream or a raw handle), or of
+    torch's current stream on the current device when None."""
+    global _current_stream
     if stream is None:
-        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+        if _current_stream is None:
+            torch = _torch()
+            torch.cuda.init()
+            getdev = getattr(torch._C, "_cuda_getDevice", None)
+            raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+            if getdev is not None and raw is not None:
+                _current_stream = lambda: raw(getdev())
+            else:
+                _current_stream = lambda: torch.cuda.current_stream().cuda_stream
+        return _current_stream()
     if hasattr(stream, "cuda_stream"):
-        return C.c_void_p(stream.cuda_stream)
-    return C.c_void_p(stream)
+        return stream.cuda_stream
+    return stream
 
 
 def _workspace(nbytes: int, device):
