@@ -14,7 +14,9 @@ Timing: W untimed warm-up steps, then K steps between CUDA events on the launchi
 stream, bracketed by a barrier and a device synchronise; the maximum over ranks is
 taken. Workloads whose operands fit in L2 rotate over enough copies that the bytes
 touched between two uses of one copy exceed L2. SM clocks and throttle reasons are
-sampled with nvidia-smi during the headline's timed region.
+sampled with nvidia-smi during the headline's timed region. After that region the
+headline also times at least 50 further calls one by one (events around each call) and
+reports their median, minimum and maximum.
 
 ``--impl reference`` times the CPU oracle (plain FP64 triple loop) on a bounded
 sample of the same workload on the host cores, as the reference arm.
@@ -159,6 +161,28 @@ def time_steps(torch, step, warmup: int, steps: int, dist=None):
     return max_over_ranks(s.elapsed_time(e), dist)
 
 
+def per_call_us(torch, step, start: int, calls: int) -> dict:
+    """Median, min and max device time (us) of `calls` further calls of step(i), each
+    bracketed by its own CUDA events on the current stream (run after the timed region,
+    so its events do not touch the headline timing)."""
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(calls + 1)]
+    step(start)  # not measured: keeps the device busy while the measured calls are queued
+    ev[0].record()
+    for i in range(calls):
+        step(start + 1 + i)
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    return call_stats([ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(calls)])
+
+
+def call_stats(us) -> dict:
+    t = sorted(us)
+    n = len(t)
+    med = t[n // 2] if n % 2 else 0.5 * (t[n // 2 - 1] + t[n // 2])
+    return {"median": round(med, 2), "min": round(t[0], 2), "max": round(t[-1], 2), "calls": n}
+
+
 def max_over_ranks(x: float, dist=None) -> float:
     """The largest of every rank's x (all ranks call it; NCCL reduces on the device,
     other backends on the host)."""
@@ -246,10 +270,12 @@ def wl_square_bf16(c: Ctx, headline: bool):
         smi_id = str(c.dev.index)
     with ClockSampler(smi_id) as clk:
         ms = c.time(step)
+    dist_us = per_call_us(torch, step, c.W + c.K, max(50, c.K))
     assert sg.check() == sg.OK
     flops = m.gemm_flops(n, n, n)
     plan = sg.last_config()
-    c.record("square_bf16_4096", ms, c.K, flops=flops, peak_tf=c.peaks["bf16_tflops"], extra={"plan": plan})
+    c.record("square_bf16_4096", ms, c.K, flops=flops, peak_tf=c.peaks["bf16_tflops"],
+             extra={"plan": plan, "per_call_us": dist_us})
     out = {"ms": ms, "flops": flops, "copies": copies, "set_bytes": set_bytes, "plan": plan,
            "clocks": clk.summary()}
     if not headline:

@@ -53,3 +53,8 @@ def test_max_over_ranks_and_aggregate(world):
 def test_single_process_passthrough():
     assert bench.max_over_ranks(1.25, None) == 1.25
     assert bench.whole_job_tflops(1e12, 4, 1, 2.0) == pytest.approx(2000.0)
+
+
+def test_call_stats_median_min_max():
+    assert bench.call_stats([3.0, 1.0, 2.0]) == {"median": 2.0, "min": 1.0, "max": 3.0, "calls": 3}
+    assert bench.call_stats([4.0, 1.0, 2.0, 3.0]) == {"median": 2.5, "min": 1.0, "max": 4.0, "calls": 4}
