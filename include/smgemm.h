@@ -116,10 +116,16 @@ smgemm_status gemm_bf16_noalloc(int64_t M, int64_t N, int64_t K,
  *              gemm_bf16. Groups with M or N = 0 are skipped; K = 0 writes act(bias).
  *   workspace  device, at least smgemm_grouped_workspace_size(G) bytes: the host writes
  *              the groups' TMA descriptors and sizes there (an asynchronous copy on
- *              `stream`, from pageable memory) before the launch; calls that can overlap
- *              on the GPU must not share it.
- * Every group is validated before anything is enqueued; errors as in gemm_bf16. Each
- * output tile is one unit of work (no split-K); results are deterministic.
+ *              `stream`, from pageable memory) before the launch; the rest holds the
+ *              partial tiles of a split last wave. Calls that can overlap on the GPU
+ *              must not share it. A smaller workspace that still holds the table is
+ *              accepted; the last wave is then not split.
+ * Every group is validated before anything is enqueued; errors as in gemm_bf16. Tiles
+ * of 256 x 256 run one per CTA pair; when the tiles do not fill a whole last wave, the
+ * R tiles of that wave are each split along K into S = min(P / R, KB / 8) pieces (P
+ * co-resident pairs, KB the smallest K-block count among those tiles) that run side
+ * by side; the last piece to finish sums the partials in piece order, so results are
+ * deterministic run to run.
  */
 size_t smgemm_grouped_workspace_size(int G);
 smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const int64_t* K,
