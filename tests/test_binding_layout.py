@@ -39,3 +39,70 @@ def test_layout_as_reads_single_rows_and_columns_in_either_layout():
     assert sg._layout_as(dense_col, "c", sg.COL_MAJOR) == (sg.COL_MAJOR, 64)  # unused pitch: >= rows
     with pytest.raises(ValueError):
         sg._layout_as(torch.zeros(4, 8), "x", sg.COL_MAJOR)    # a true row-major matrix
+
+
+class _RecordingLib:
+    """Stands in for the C library: records the arguments of gemm_bf16_grouped."""
+
+    def __init__(self):
+        self.calls = []
+
+    def smgemm_grouped_workspace_size(self, G):
+        return 4096
+
+    def gemm_bf16_grouped(self, *args):
+        self.calls.append(args)
+        return sg.OK
+
+
+def _grouped_args(monkeypatch, *a, **kw):
+    rec = _RecordingLib()
+    monkeypatch.setattr(sg, "_lib", rec)
+    monkeypatch.setattr(sg, "_stream", lambda s: 0)
+    res = sg.gemm_bf16_grouped(*a, **kw)
+    (args,) = rec.calls
+    (G, Ms, Ns, Ks, pA, adt, lay_a, ldas, pB, lay_b, ldbs, pbias, bdt, act, pC, cdt, ldcs, ws, wsb, st) = args
+    as_list = lambda arr: [arr[i] for i in range(G)]
+    return res, dict(G=G, M=as_list(Ms), N=as_list(Ns), K=as_list(Ks), A=as_list(pA), adt=adt, lay_a=lay_a,
+                     lda=as_list(ldas), B=as_list(pB), lay_b=lay_b, ldb=as_list(ldbs),
+                     bias=None if pbias is None else as_list(pbias), bdt=bdt, act=act, C=as_list(pC), cdt=cdt,
+                     ldc=as_list(ldcs), ws=ws, wsb=wsb)
+
+
+def test_grouped_marshalling_padded_views(monkeypatch):
+    """Sizes, pitches, pointers, dtypes and the shared layouts handed to the C ABI."""
+    bf = torch.bfloat16
+    As = [torch.zeros(3, 72, dtype=bf)[:, :64], torch.zeros(5, 136, dtype=bf)[:, :128]]   # row-major, padded
+    Bs = [torch.zeros(40, 64, dtype=bf)[:, :64].t()[:, :24], torch.zeros(16, 136, dtype=bf)[:, :128].t()]  # col
+    biases = [torch.zeros(24, dtype=torch.float32), None]
+    outs = [torch.zeros(3, 32, dtype=torch.float32)[:, :24], torch.zeros(5, 16, dtype=torch.float32)]
+    ws = torch.zeros(8192, dtype=torch.uint8)
+    res, d = _grouped_args(monkeypatch, As, Bs, biases=biases, act="silu", outs=outs, workspace=ws)
+    assert res == outs
+    assert (d["G"], d["M"], d["N"], d["K"]) == (2, [3, 5], [24, 16], [64, 128])
+    assert (d["lay_a"], d["lda"]) == (sg.ROW_MAJOR, [72, 136])
+    assert (d["lay_b"], d["ldb"]) == (sg.COL_MAJOR, [64, 136])
+    assert d["ldc"] == [32, 16]
+    assert d["A"] == [t.data_ptr() for t in As] and d["B"] == [t.data_ptr() for t in Bs]
+    assert d["C"] == [t.data_ptr() for t in outs]
+    assert d["bias"] == [biases[0].data_ptr(), None] and d["bdt"] == sg.F32
+    assert (d["adt"], d["cdt"], d["act"]) == (sg.BF16, sg.F32, sg.ACTS["silu"])
+    assert (d["ws"], d["wsb"]) == (ws.data_ptr(), 8192)
+
+
+def test_grouped_marshalling_single_rows_and_allocated_outputs(monkeypatch):
+    """A one-row A takes the layout of the other groups (column-major here); outputs
+    are allocated with the requested type when not given; no biases."""
+    h = torch.float16
+    a0 = torch.zeros(64, 8, dtype=h)[:, :1].t()            # one row [1, 64], column pitch 8
+    a1 = torch.zeros(96, 48, dtype=h)[:, :40].t()          # [40, 96] column-major, pitch 48
+    As = [a0, a1]
+    Bs = [torch.zeros(64, 8, dtype=h), torch.zeros(96, 16, dtype=h)]
+    with pytest.raises(ValueError):                        # K of group 1 does not match its B
+        _grouped_args(monkeypatch, [a0, torch.zeros(48, 40, dtype=h)], Bs)
+    res, d = _grouped_args(monkeypatch, As, Bs, out_dtype=torch.bfloat16, workspace=torch.zeros(16, dtype=torch.uint8))
+    assert [tuple(r.shape) for r in res] == [(1, 8), (40, 16)] and all(r.dtype == torch.bfloat16 for r in res)
+    assert d["lay_a"] == sg.COL_MAJOR and d["lda"] == [8, 48]
+    assert d["lay_b"] == sg.ROW_MAJOR and d["ldb"] == [8, 16]
+    assert d["bias"] is None and d["bdt"] == 0 and d["cdt"] == sg.BF16 and d["adt"] == sg.F16
+    assert d["K"] == [64, 96] and d["M"] == [1, 40] and d["N"] == [8, 16]
