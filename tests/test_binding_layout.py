@@ -51,7 +51,14 @@ class _RecordingLib:
         return 4096
 
     def gemm_bf16_grouped(self, *args):
-        self.calls.append(args)
+        # The host arrays are only valid during the call (as for the library, which
+        # copies what it needs before returning): decode them now.
+        (G, Ms, Ns, Ks, pA, adt, lay_a, ldas, pB, lay_b, ldbs, pbias, bdt, act, pC, cdt, ldcs, ws, wsb, st) = args
+        as_list = lambda arr: [arr[i] for i in range(G)]
+        self.calls.append(dict(G=G, M=as_list(Ms), N=as_list(Ns), K=as_list(Ks), A=as_list(pA), adt=adt,
+                               lay_a=lay_a, lda=as_list(ldas), B=as_list(pB), lay_b=lay_b, ldb=as_list(ldbs),
+                               bias=None if pbias is None else as_list(pbias), bdt=bdt, act=act, C=as_list(pC),
+                               cdt=cdt, ldc=as_list(ldcs), ws=ws, wsb=wsb))
         return sg.OK
 
 
@@ -60,13 +67,8 @@ def _grouped_args(monkeypatch, *a, **kw):
     monkeypatch.setattr(sg, "_lib", rec)
     monkeypatch.setattr(sg, "_stream", lambda s: 0)
     res = sg.gemm_bf16_grouped(*a, **kw)
-    (args,) = rec.calls
-    (G, Ms, Ns, Ks, pA, adt, lay_a, ldas, pB, lay_b, ldbs, pbias, bdt, act, pC, cdt, ldcs, ws, wsb, st) = args
-    as_list = lambda arr: [arr[i] for i in range(G)]
-    return res, dict(G=G, M=as_list(Ms), N=as_list(Ns), K=as_list(Ks), A=as_list(pA), adt=adt, lay_a=lay_a,
-                     lda=as_list(ldas), B=as_list(pB), lay_b=lay_b, ldb=as_list(ldbs),
-                     bias=None if pbias is None else as_list(pbias), bdt=bdt, act=act, C=as_list(pC), cdt=cdt,
-                     ldc=as_list(ldcs), ws=ws, wsb=wsb)
+    (d,) = rec.calls
+    return res, d
 
 
 def test_grouped_marshalling_padded_views(monkeypatch):
