@@ -27,6 +27,7 @@ ACTS = {"none": 0, None: 0, "gelu_tanh": 1, "gelu": 1, "silu": 2}
 _lock = threading.Lock()
 _lib = None
 _ws_cache: dict = {}
+_ws_retired: list = []
 
 
 class SmgemmError(RuntimeError):
@@ -147,14 +148,23 @@ def _stream(stream):
     return stream
 
 
-def _workspace(nbytes: int, device):
+def _workspace(nbytes: int, device, stream_handle):
+    """A cached workspace of at least nbytes for calls on (device, stream). Calls on one
+    stream run in order and share it; calls on different streams, which may overlap,
+    get different ones. A workspace that is outgrown is kept alive (in _ws_retired),
+    since kernels already queued may still use it; sizes at least double, so the kept
+    ones total less than the live one."""
     if nbytes == 0:
         return None, 0
     torch = _torch()
-    key = (device.index if device.index is not None else torch.cuda.current_device())
+    key = (device.index if device.index is not None else torch.cuda.current_device(),
+           int(getattr(stream_handle, "value", stream_handle) or 0))
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < nbytes:
-        ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        if ws is not None:
+            _ws_retired.append(ws)
+        size = max(nbytes, 1 << 20, 0 if ws is None else 2 * ws.numel())
+        ws = torch.empty(size, dtype=torch.uint8, device=device)
         _ws_cache[key] = ws
     return ws, ws.numel()
 
@@ -185,13 +195,14 @@ def gemm_bf16(A, B, *, bias=None, act="none", out=None, out_dtype=None, workspac
     if out.stride(1) != 1:
         raise ValueError("out must be row-major")
     ldc = max(out.stride(0), N)
+    sh = _stream(stream)
     ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
-        _workspace(workspace_size(M, N, K, 0), A.device)
+        _workspace(workspace_size(M, N, K, 0), A.device, sh)
     st = lib().gemm_bf16(M, N, K, A.data_ptr(), _dtype_code(A.dtype), la, lda, B.data_ptr(), lb, ldb,
                          None if bias is None else bias.data_ptr(),
                          _dtype_code(bias.dtype) if bias is not None else 0, ACTS[act],
                          out.data_ptr(), _dtype_code(out.dtype), ldc,
-                         None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+                         None if ws is None else ws.data_ptr(), wsb, sh)
     _check(st, "gemm_bf16")
     return out
 
@@ -214,13 +225,14 @@ def gemm_bf16_fp8out(A, B, *, bias=None, act="none", Q=None, scales=None, worksp
     if Q.stride(1) != 1:
         raise ValueError("Q must be row-major")
     ldc = max(Q.stride(0), N)
+    sh = _stream(stream)
     ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
-        _workspace(workspace_size(M, N, K, 0), A.device)
+        _workspace(workspace_size(M, N, K, 0), A.device, sh)
     st = lib().gemm_bf16_fp8out(M, N, K, A.data_ptr(), _dtype_code(A.dtype), la, lda, B.data_ptr(), lb, ldb,
                                 None if bias is None else bias.data_ptr(),
                                 _dtype_code(bias.dtype) if bias is not None else 0, ACTS[act],
                                 Q.data_ptr(), ldc, scales.data_ptr(), None if ws is None else ws.data_ptr(), wsb,
-                                _stream(stream))
+                                sh)
     _check(st, "gemm_bf16_fp8out")
     return Q, scales
 
@@ -240,12 +252,13 @@ def gemm_bf16_logsoftmax(A, B, *, bias=None, out=None, workspace=None, stream=No
     if out.dtype != torch.float32 or out.stride(1) != 1:
         raise ValueError("out must be row-major float32")
     ldc = max(out.stride(0), N)
+    sh = _stream(stream)
     ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
-        _workspace(int(lib().smgemm_logsoftmax_workspace_size(M, N, K)), A.device)
+        _workspace(int(lib().smgemm_logsoftmax_workspace_size(M, N, K)), A.device, sh)
     st = lib().gemm_bf16_logsoftmax(M, N, K, A.data_ptr(), _dtype_code(A.dtype), la, lda, B.data_ptr(), lb, ldb,
                                     None if bias is None else bias.data_ptr(),
                                     _dtype_code(bias.dtype) if bias is not None else 0,
-                                    out.data_ptr(), ldc, None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+                                    out.data_ptr(), ldc, None if ws is None else ws.data_ptr(), wsb, sh)
     _check(st, "gemm_bf16_logsoftmax")
     return out
 
@@ -282,13 +295,14 @@ def gemm_bf16_grouped(As, Bs, *, biases=None, act="none", outs=None, out_dtype=N
     arr = lambda xs: (C.c_int64 * G)(*xs)
     ptrs = lambda ts: (C.c_void_p * G)(*[None if t is None else t.data_ptr() for t in ts])
     nbytes = int(lib().smgemm_grouped_workspace_size(G))
-    ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(nbytes, As[0].device)
+    sh = _stream(stream)
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(nbytes, As[0].device, sh)
     bias_dt = next((_dtype_code(b.dtype) for b in (biases or []) if b is not None), 0)
     st = lib().gemm_bf16_grouped(G, arr(Ms), arr(Ns), arr(Ks), ptrs(As), _dtype_code(As[0].dtype), lay_a,
                                  arr(ldas), ptrs(Bs), lay_b, arr(ldbs),
                                  None if biases is None else ptrs(biases), bias_dt, ACTS[act],
                                  ptrs(res), _dtype_code(res[0].dtype), arr(ldcs),
-                                 None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+                                 None if ws is None else ws.data_ptr(), wsb, sh)
     _check(st, "gemm_bf16_grouped")
     return res
 
@@ -308,13 +322,14 @@ def gemm_fp8_blockscaled(Aq, sa, Bq, sb, *, bias=None, act="none", out=None, out
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=Aq.device)
     ldc = max(out.stride(0), N)
+    sh = _stream(stream)
     ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
-        _workspace(workspace_size(M, N, K, 1), Aq.device)
+        _workspace(workspace_size(M, N, K, 1), Aq.device, sh)
     st = lib().gemm_fp8_blockscaled(M, N, K, Aq.data_ptr(), sa.data_ptr(), Bq.data_ptr(), sb.data_ptr(),
                                     None if bias is None else bias.data_ptr(),
                                     _dtype_code(bias.dtype) if bias is not None else 0, ACTS[act],
                                     out.data_ptr(), _dtype_code(out.dtype), ldc,
-                                    None if ws is None else ws.data_ptr(), wsb, _stream(stream))
+                                    None if ws is None else ws.data_ptr(), wsb, sh)
     _check(st, "gemm_fp8_blockscaled")
     return out
 

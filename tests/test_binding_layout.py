@@ -108,3 +108,21 @@ def test_grouped_marshalling_single_rows_and_allocated_outputs(monkeypatch):
     assert d["lay_b"] == sg.ROW_MAJOR and d["ldb"] == [8, 16]
     assert d["bias"] is None and d["bdt"] == 0 and d["cdt"] == sg.BF16 and d["adt"] == sg.F16
     assert d["K"] == [64, 96] and d["M"] == [1, 40] and d["N"] == [8, 16]
+
+
+def test_workspace_cache_per_stream_and_growth(monkeypatch):
+    """Cached workspaces: shared by calls on one stream, distinct per stream (calls on
+    different streams may overlap), and an outgrown one is kept alive, not freed."""
+    import ctypes
+    monkeypatch.setattr(sg, "_ws_cache", {})
+    monkeypatch.setattr(sg, "_ws_retired", [])
+    dev = torch.device("cpu", 0)
+    assert sg._workspace(0, dev, 0) == (None, 0)
+    w1, n1 = sg._workspace(1000, dev, 0)
+    assert n1 == w1.numel() >= 1 << 20
+    assert sg._workspace(5000, dev, 0)[0] is w1                 # same stream: reused
+    w2, _ = sg._workspace(1000, dev, 0x1234)                      # another stream: its own
+    assert w2 is not w1
+    assert sg._workspace(1000, dev, ctypes.c_void_p(0x1234))[0] is w2
+    w3, n3 = sg._workspace(n1 + 1, dev, 0)                        # outgrown: at least doubled
+    assert w3 is not w1 and n3 >= 2 * n1 and sg._ws_retired == [w1]
