@@ -43,3 +43,15 @@ def test_workload_shapes():
     assert f["b1"].shape == (32,)
     l1, l2 = synth.lm_head(m=2, d_model=8, vocab=40), synth.lm_head(m=3, d_model=8, vocab=40)
     assert (l1["W"] == l2["W"]).all()           # one weight shared by every M
+
+
+def test_splitmix64_reference_sequence():
+    """The counter-based stream equals the published sequential generator: output i of
+    stream `key` is the finaliser of key + (i + 1) * gamma, so key = 1234567 must give
+    the generator's check values for that initial state (tests/golden)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "splitmix64_state_1234567.txt")
+    want = [int(l) for l in open(path) if l.strip() and not l.startswith("#")]
+    got = synth._bits(1234567, 0, len(want))
+    assert [int(v) for v in got] == want
+    assert [int(v) for v in synth._bits(1234567, 2, 3)] == want[2:]   # any counter range alone
