@@ -76,6 +76,12 @@ def _brute_force_encode(y: np.ndarray) -> np.ndarray:
     return out
 
 
+def test_nearest_search_agrees_with_brute_force():
+    y = np.abs(_structured_floats())
+    y = y[y <= 448.0]
+    assert (_nearest_code_sorted(y.astype(np.float64)) == _brute_force_encode(y)).all()
+
+
 def test_encode_brute_force_structured():
     y = _structured_floats()
     y = y[np.abs(y) < 1e6]
@@ -186,12 +192,24 @@ def test_load_fp16_and_bf16_decoding():
         assert oracle.load_elem(bits, oracle.BF16, i) == ref[i]
 
 
+def _nearest_code_sorted(a: np.ndarray) -> np.ndarray:
+    """Code of the E4M3 value nearest to each magnitude a in [0, 448], ties to the even
+    code, by bisection over the 127 ascending non-negative finite values (the same
+    definition as _brute_force_encode, fast enough for a billion inputs)."""
+    vals = _table()[:127]
+    i = np.minimum(np.searchsorted(vals, a, side="left"), 126)   # vals[i - 1] < a <= vals[i]
+    lo = np.maximum(i - 1, 0)
+    d_lo, d_hi = a - vals[lo], vals[i] - a                       # exact in double
+    return np.where(d_hi < d_lo, i, np.where(d_lo < d_hi, lo, np.where(i % 2 == 0, i, lo))).astype(np.uint8)
+
+
 def test_encode_exhaustive_against_torch():
     """Every non-negative FP32 value up to 448 (all 1,138,753,537 bit patterns from +0 to
-    448.0), encoded by the oracle and by torch's independent float8_e4m3fn cast (RNE),
-    plus the sign-flipped patterns of a strided subset."""
+    448.0), encoded by the oracle, by torch's independent float8_e4m3fn cast (RNE) and by
+    a nearest-value search with ties to even; plus the sign-flipped patterns of a
+    strided subset."""
     top = int(np.array(448.0, dtype=np.float32).view(np.uint32))
-    step = 1 << 25
+    step = 1 << 24
     for lo in range(0, top + 1, step):
         bits = np.arange(lo, min(lo + step, top + 1), dtype=np.uint32)
         y = bits.view(np.float32)
@@ -199,6 +217,9 @@ def test_encode_exhaustive_against_torch():
         got = oracle.e4m3_encode(y)
         bad = np.flatnonzero(got != ref)
         assert bad.size == 0, f"{bad.size} mismatches from {y[bad[0]]!r}: {got[bad[0]]:#x} vs {ref[bad[0]]:#x}"
+        near = _nearest_code_sorted(y.astype(np.float64))
+        bad = np.flatnonzero(got != near)
+        assert bad.size == 0, f"{bad.size} off the nearest code from {y[bad[0]]!r}: {got[bad[0]]:#x} vs {near[bad[0]]:#x}"
     neg = -(np.arange(0, top + 1, 997, dtype=np.uint32).view(np.float32))
     ref = torch.from_numpy(neg).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.array_equal(oracle.e4m3_encode(neg), ref)
