@@ -1,8 +1,11 @@
 """Python binding of the smgemm C-ABI (libsmgemm.so, built for sm_100a).
 
 Argument marshalling only: torch tensors give device pointers, leading dimensions
-and the current CUDA stream; every computation runs in the library's kernels. There
-is no fallback: if the library is missing or a call fails, an exception is raised.
+and the current CUDA stream; every computation runs in the library's kernels. Before a
+call, every tensor is checked to be on the call's CUDA device with the type and shape
+the sizes imply (ValueError otherwise), since the kernels dereference what they are
+given. There is no fallback: if the library is missing or a call fails, an exception
+is raised.
 
     import sm_gemm_b200 as sg
     C = sg.gemm_bf16(A, B, bias=b, act="gelu_tanh", out_dtype=torch.bfloat16)
@@ -97,7 +100,65 @@ def _dtype_code(dt) -> int:
     if not _DTYPES:
         torch = _torch()
         _DTYPES.update({torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16})
-    return _DTYPES[dt]
+    code = _DTYPES.get(dt)
+    if code is None:
+        raise ValueError(f"unsupported dtype {dt} (float32, bfloat16 or float16)")
+    return code
+
+
+# Host-side checks of every tensor a call hands to the library: the kernels dereference
+# the pointers they are given, so a host tensor, a tensor on another GPU, or one smaller
+# than the sizes say must be refused here rather than read or written out of bounds.
+
+def _need(ok: bool, msg: str):
+    if not ok:
+        raise ValueError(msg)
+
+
+def _device(*ts):
+    """CUDA device index shared by the given tensors (None entries are skipped)."""
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        _need(t.is_cuda, "every tensor of a call must be on a CUDA device")
+        d = t.get_device()
+        _need(dev is None or d == dev, "all tensors of a call must be on one CUDA device")
+        dev = d
+    return dev
+
+
+def _current_device():
+    return _torch().cuda.current_device()
+
+
+def _shape(t, want, name):
+    _need(tuple(t.shape) == tuple(want), f"{name} must have shape {tuple(want)}, not {tuple(t.shape)}")
+
+
+def _dense(t, name):
+    _need(t.is_contiguous(), f"{name} must be contiguous")
+
+
+def _vector(t, n, name):
+    """A bias: 1-D, unit stride, at least n elements."""
+    _need(t.dim() == 1 and t.shape[0] >= n and (t.shape[0] <= 1 or t.stride(0) == 1),
+          f"{name} must be a unit-stride vector of at least {n} elements")
+    _dtype_code(t.dtype)
+
+
+def _out_matrix(t, M, N, name, dtypes=None):
+    _shape(t, (M, N), name)
+    _need(t.dim() == 2 and (t.stride(1) == 1 or N <= 1), f"{name} must be row-major")
+    if dtypes is not None:
+        _need(t.dtype in dtypes, f"{name} must be one of {dtypes}")
+    else:
+        _dtype_code(t.dtype)
+
+
+def _ws_bytes(workspace):
+    _dense(workspace, "workspace")
+    return workspace.numel() * workspace.element_size()
 
 
 def _layout(t, name):
@@ -183,6 +244,11 @@ def gemm_bf16(A, B, *, bias=None, act="none", out=None, out_dtype=None, workspac
 
     ``out`` (row-major [M,N]) is allocated when not given; ``out_dtype`` defaults to
     A's dtype. Returns ``out``."""
+    dev = _device(A, B, bias, out, workspace)
+    if dev != _current_device():
+        with _torch().cuda.device(dev):
+            return gemm_bf16(A, B, bias=bias, act=act, out=out, out_dtype=out_dtype, workspace=workspace,
+                             stream=stream)
     torch = _torch()
     M, K = A.shape
     K2, N = B.shape
@@ -190,13 +256,14 @@ def gemm_bf16(A, B, *, bias=None, act="none", out=None, out_dtype=None, workspac
         raise ValueError("A and B must agree in K and dtype")
     la, lda = _layout(A, "A")
     lb, ldb = _layout(B, "B")
+    if bias is not None:
+        _vector(bias, N, "bias")
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype or A.dtype, device=A.device)
-    if out.stride(1) != 1:
-        raise ValueError("out must be row-major")
+    _out_matrix(out, M, N, "out")
     ldc = max(out.stride(0), N)
     sh = _stream(stream)
-    ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
+    ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else \
         _workspace(workspace_size(M, N, K, 0), A.device, sh)
     st = lib().gemm_bf16(M, N, K, A.data_ptr(), _dtype_code(A.dtype), la, lda, B.data_ptr(), lb, ldb,
                          None if bias is None else bias.data_ptr(),
@@ -211,6 +278,11 @@ def gemm_bf16_fp8out(A, B, *, bias=None, act="none", Q=None, scales=None, worksp
     """act(A @ B + bias) quantised to E4M3 with one FP32 scale per 1x128 row group:
     returns (codes uint8 [M, N], scales float32 [ceil(N/128), M]), the A operand of
     gemm_fp8_blockscaled."""
+    dev = _device(A, B, bias, Q, scales, workspace)
+    if dev != _current_device():
+        with _torch().cuda.device(dev):
+            return gemm_bf16_fp8out(A, B, bias=bias, act=act, Q=Q, scales=scales, workspace=workspace,
+                                    stream=stream)
     torch = _torch()
     M, K = A.shape
     K2, N = B.shape
@@ -218,15 +290,19 @@ def gemm_bf16_fp8out(A, B, *, bias=None, act="none", Q=None, scales=None, worksp
         raise ValueError("A and B must agree in K and dtype")
     la, lda = _layout(A, "A")
     lb, ldb = _layout(B, "B")
+    if bias is not None:
+        _vector(bias, N, "bias")
     if Q is None:
         Q = torch.empty((M, -(-N // 16) * 16), dtype=torch.uint8, device=A.device)[:, :N]
     if scales is None:
         scales = torch.empty((-(-N // 128), M), dtype=torch.float32, device=A.device)
-    if Q.stride(1) != 1:
-        raise ValueError("Q must be row-major")
+    _out_matrix(Q, M, N, "Q", (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8)))
+    _shape(scales, (-(-N // 128), M), "scales")
+    _dense(scales, "scales")
+    _need(scales.dtype == torch.float32, "scales must be float32")
     ldc = max(Q.stride(0), N)
     sh = _stream(stream)
-    ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
+    ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else \
         _workspace(workspace_size(M, N, K, 0), A.device, sh)
     st = lib().gemm_bf16_fp8out(M, N, K, A.data_ptr(), _dtype_code(A.dtype), la, lda, B.data_ptr(), lb, ldb,
                                 None if bias is None else bias.data_ptr(),
@@ -240,6 +316,10 @@ def gemm_bf16_fp8out(A, B, *, bias=None, act="none", Q=None, scales=None, worksp
 def gemm_bf16_logsoftmax(A, B, *, bias=None, out=None, workspace=None, stream=None):
     """log_softmax(A @ B + bias) over each row, FP32 [M, N] (the LM head and its
     log-softmax, fused). A, B, bias as in gemm_bf16; ``out`` is allocated if not given."""
+    dev = _device(A, B, bias, out, workspace)
+    if dev != _current_device():
+        with _torch().cuda.device(dev):
+            return gemm_bf16_logsoftmax(A, B, bias=bias, out=out, workspace=workspace, stream=stream)
     torch = _torch()
     M, K = A.shape
     K2, N = B.shape
@@ -247,13 +327,14 @@ def gemm_bf16_logsoftmax(A, B, *, bias=None, out=None, workspace=None, stream=No
         raise ValueError("A and B must agree in K and dtype")
     la, lda = _layout(A, "A")
     lb, ldb = _layout(B, "B")
+    if bias is not None:
+        _vector(bias, N, "bias")
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=A.device)
-    if out.dtype != torch.float32 or out.stride(1) != 1:
-        raise ValueError("out must be row-major float32")
+    _out_matrix(out, M, N, "out", (torch.float32,))
     ldc = max(out.stride(0), N)
     sh = _stream(stream)
-    ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
+    ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else \
         _workspace(int(lib().smgemm_logsoftmax_workspace_size(M, N, K)), A.device, sh)
     st = lib().gemm_bf16_logsoftmax(M, N, K, A.data_ptr(), _dtype_code(A.dtype), la, lda, B.data_ptr(), lb, ldb,
                                     None if bias is None else bias.data_ptr(),
@@ -268,12 +349,17 @@ def gemm_bf16_grouped(As, Bs, *, biases=None, act="none", outs=None, out_dtype=N
     """C_g = act(A_g @ B_g + bias_g) for every group g in one launch. All A_g share one
     layout and dtype, all B_g one layout; sizes may differ. ``outs`` (row-major) are
     allocated when not given. Returns the list of outputs."""
-    torch = _torch()
     G = len(As)
     if len(Bs) != G or (biases is not None and len(biases) != G) or (outs is not None and len(outs) != G):
         raise ValueError("As, Bs, biases and outs must have one entry per group")
     if G == 0:
         return []
+    dev = _device(*As, *Bs, *(biases or ()), *(outs or ()), workspace)
+    if dev != _current_device():
+        with _torch().cuda.device(dev):
+            return gemm_bf16_grouped(As, Bs, biases=biases, act=act, outs=outs, out_dtype=out_dtype,
+                                     workspace=workspace, stream=stream)
+    torch = _torch()
     Ms, Ns, Ks, ldas, ldbs, ldcs = [], [], [], [], [], []
     # The shared layouts: those of the first group whose operand is not a single row or column.
     lay_a = next((_layout(A, "A")[0] for A in As if min(A.shape) > 1), ROW_MAJOR)
@@ -286,9 +372,11 @@ def gemm_bf16_grouped(As, Bs, *, biases=None, act="none", outs=None, out_dtype=N
             raise ValueError(f"group {g}: A and B must agree in K and dtype")
         _, lda = _layout_as(A, f"A[{g}]", lay_a)
         _, ldb = _layout_as(B, f"B[{g}]", lay_b)
+        if biases is not None and biases[g] is not None:
+            _vector(biases[g], N, f"biases[{g}]")
         out = outs[g] if outs is not None else torch.empty((M, N), dtype=out_dtype or A.dtype, device=A.device)
-        if out.stride(1) != 1:
-            raise ValueError("outputs must be row-major")
+        _out_matrix(out, M, N, f"outs[{g}]")
+        _need(out.dtype == (outs[0].dtype if outs is not None else out.dtype), "outputs must share one dtype")
         res.append(out)
         Ms.append(M); Ns.append(N); Ks.append(K); ldas.append(lda); ldbs.append(ldb)
         ldcs.append(max(out.stride(0), N))
@@ -296,8 +384,9 @@ def gemm_bf16_grouped(As, Bs, *, biases=None, act="none", outs=None, out_dtype=N
     ptrs = lambda ts: (C.c_void_p * G)(*[None if t is None else t.data_ptr() for t in ts])
     nbytes = int(lib().smgemm_grouped_workspace_size(G))
     sh = _stream(stream)
-    ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(nbytes, As[0].device, sh)
+    ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else _workspace(nbytes, As[0].device, sh)
     bias_dt = next((_dtype_code(b.dtype) for b in (biases or []) if b is not None), 0)
+    _need(all(b is None or _dtype_code(b.dtype) == bias_dt for b in (biases or [])), "biases must share one dtype")
     st = lib().gemm_bf16_grouped(G, arr(Ms), arr(Ns), arr(Ks), ptrs(As), _dtype_code(As[0].dtype), lay_a,
                                  arr(ldas), ptrs(Bs), lay_b, arr(ldbs),
                                  None if biases is None else ptrs(biases), bias_dt, ACTS[act],
@@ -311,6 +400,11 @@ def gemm_fp8_blockscaled(Aq, sa, Bq, sb, *, bias=None, act="none", out=None, out
                          workspace=None, stream=None):
     """C = act(sum_kb sa*sb*(Aq @ Bq^T)_kb + bias) from E4M3 codes Aq[M,K], Bq[N,K] (uint8 or
     float8_e4m3fn, K contiguous) and FP32 scales sa[KB,M], sb[KB,NB]."""
+    dev = _device(Aq, sa, Bq, sb, bias, out, workspace)
+    if dev != _current_device():
+        with _torch().cuda.device(dev):
+            return gemm_fp8_blockscaled(Aq, sa, Bq, sb, bias=bias, act=act, out=out, out_dtype=out_dtype,
+                                        workspace=workspace, stream=stream)
     torch = _torch()
     M, K = Aq.shape
     N, K2 = Bq.shape
@@ -319,11 +413,19 @@ def gemm_fp8_blockscaled(Aq, sa, Bq, sb, *, bias=None, act="none", out=None, out
     for t, n in ((Aq, "Aq"), (Bq, "Bq"), (sa, "sa"), (sb, "sb")):
         if not t.is_contiguous():
             raise ValueError(f"{n} must be contiguous")
+    codes = (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8))
+    _need(Aq.dtype in codes and Bq.dtype in codes, "Aq and Bq must be uint8 or float8_e4m3fn codes")
+    _need(sa.dtype == torch.float32 and sb.dtype == torch.float32, "sa and sb must be float32")
+    _shape(sa, (-(-K // 128), M), "sa")
+    _shape(sb, (-(-K // 128), -(-N // 128)), "sb")
+    if bias is not None:
+        _vector(bias, N, "bias")
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=Aq.device)
+    _out_matrix(out, M, N, "out")
     ldc = max(out.stride(0), N)
     sh = _stream(stream)
-    ws, wsb = (workspace, workspace.numel()) if workspace is not None else \
+    ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else \
         _workspace(workspace_size(M, N, K, 1), Aq.device, sh)
     st = lib().gemm_fp8_blockscaled(M, N, K, Aq.data_ptr(), sa.data_ptr(), Bq.data_ptr(), sb.data_ptr(),
                                     None if bias is None else bias.data_ptr(),
@@ -338,7 +440,12 @@ def quantize_fp8_blockwise(X, group_rows: int = 1, *, Q=None, scales=None, strea
     """FP32 X[rows, cols] -> (codes uint8, scales float32). group_rows=1: 1x128 groups,
     codes [rows, cols], scales [ceil(cols/128), rows]. group_rows=128: 128x128 blocks of
     the weight X[K, N], codes written transposed [N, K], scales [ceil(K/128), ceil(N/128)]."""
+    dev = _device(X, Q, scales)
+    if dev != _current_device():
+        with _torch().cuda.device(dev):
+            return quantize_fp8_blockwise(X, group_rows, Q=Q, scales=scales, stream=stream)
     torch = _torch()
+    _need(X.dtype == torch.float32, "X must be float32")
     rows, cols = X.shape
     lx, ldx = _layout(X, "X")
     if group_rows == 1:
@@ -349,6 +456,12 @@ def quantize_fp8_blockwise(X, group_rows: int = 1, *, Q=None, scales=None, strea
         Q = torch.empty(qshape, dtype=torch.uint8, device=X.device)
     if scales is None:
         scales = torch.empty(sshape, dtype=torch.float32, device=X.device)
+    _shape(Q, qshape, "Q")
+    _dense(Q, "Q")
+    _need(Q.dtype in (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8)), "Q must hold uint8 codes")
+    _shape(scales, sshape, "scales")
+    _dense(scales, "scales")
+    _need(scales.dtype == torch.float32, "scales must be float32")
     st = lib().quantize_fp8_blockwise(X.data_ptr(), rows, cols, lx, ldx, group_rows, Q.data_ptr(),
                                       scales.data_ptr(), _stream(stream))
     _check(st, "quantize_fp8_blockwise")

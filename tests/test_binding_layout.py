@@ -62,10 +62,18 @@ class _RecordingLib:
         return sg.OK
 
 
-def _grouped_args(monkeypatch, *a, **kw):
-    rec = _RecordingLib()
+def _host_only(monkeypatch, rec):
+    """Route the binding to a stand-in library and accept CPU tensors (the device check
+    is tested on its own below)."""
     monkeypatch.setattr(sg, "_lib", rec)
     monkeypatch.setattr(sg, "_stream", lambda s: 0)
+    monkeypatch.setattr(sg, "_device", lambda *ts: None)
+    monkeypatch.setattr(sg, "_current_device", lambda: None)
+
+
+def _grouped_args(monkeypatch, *a, **kw):
+    rec = _RecordingLib()
+    _host_only(monkeypatch, rec)
     res = sg.gemm_bf16_grouped(*a, **kw)
     (d,) = rec.calls
     return res, d
@@ -126,3 +134,82 @@ def test_workspace_cache_per_stream_and_growth(monkeypatch):
     assert sg._workspace(1000, dev, ctypes.c_void_p(0x1234))[0] is w2
     w3, n3 = sg._workspace(n1 + 1, dev, 0)                        # outgrown: at least doubled
     assert w3 is not w1 and n3 >= 2 * n1 and sg._ws_retired == [w1]
+
+
+class _FakeTensor:
+    def __init__(self, cuda, dev):
+        self.is_cuda, self._dev = cuda, dev
+
+    def get_device(self):
+        return self._dev
+
+
+def test_device_check():
+    """Pointers of host tensors or of another GPU's tensors would be dereferenced by the
+    kernels: the binding refuses them before calling the library."""
+    a, b, other = _FakeTensor(True, 0), _FakeTensor(True, 0), _FakeTensor(True, 1)
+    assert sg._device(a, None, b) == 0
+    assert sg._device(None) is None
+    with pytest.raises(ValueError):
+        sg._device(a, _FakeTensor(False, -1))
+    with pytest.raises(ValueError):
+        sg._device(a, other)
+    with pytest.raises(ValueError):
+        sg._device(torch.zeros(2, 2))                       # a real host tensor
+
+
+class _CountingLib:
+    """Stand-in library that counts calls; the size queries return a small workspace."""
+
+    def __init__(self):
+        self.calls = 0
+
+    def __getattr__(self, name):
+        if name.endswith("workspace_size"):
+            return lambda *a: 0
+        def call(*a):
+            self.calls += 1
+            return sg.OK
+        return call
+
+
+def test_shape_and_dtype_checks_refuse_before_the_library(monkeypatch):
+    """Tensors smaller than the sizes say, or of the wrong type, never reach the library
+    (the kernels would read or write past them)."""
+    rec = _CountingLib()
+    _host_only(monkeypatch, rec)
+    bf = torch.bfloat16
+    A, B = torch.zeros(8, 16, dtype=bf), torch.zeros(16, 24, dtype=bf)
+    bad_calls = [
+        lambda: sg.gemm_bf16(A, B, bias=torch.zeros(23, dtype=bf)),                       # bias too short
+        lambda: sg.gemm_bf16(A, B, bias=torch.zeros(48, dtype=bf)[::2]),                  # bias strided
+        lambda: sg.gemm_bf16(A, B, out=torch.zeros(8, 23, dtype=bf)),                     # out too small
+        lambda: sg.gemm_bf16(A, B, out=torch.zeros(8, 24, dtype=torch.int32)),            # out type
+        lambda: sg.gemm_bf16(A, B, bias=torch.zeros(24, dtype=torch.int64)),              # bias type
+        lambda: sg.gemm_bf16_fp8out(A, B, scales=torch.zeros(1, 7)),                      # scales shape
+        lambda: sg.gemm_bf16_fp8out(A, B, Q=torch.zeros(8, 24)),                          # codes type
+        lambda: sg.gemm_bf16_logsoftmax(A, B, out=torch.zeros(8, 24, dtype=bf)),          # not float32
+        lambda: sg.quantize_fp8_blockwise(torch.zeros(4, 256, dtype=bf)),                 # X type
+        lambda: sg.quantize_fp8_blockwise(torch.zeros(4, 256), Q=torch.zeros(4, 255, dtype=torch.uint8)),
+        lambda: sg.quantize_fp8_blockwise(torch.zeros(4, 256), scales=torch.zeros(2, 3)),
+        lambda: sg.gemm_fp8_blockscaled(torch.zeros(8, 256, dtype=torch.uint8), torch.zeros(1, 8),
+                                        torch.zeros(24, 256, dtype=torch.uint8), torch.zeros(2, 1)),  # sa shape
+        lambda: sg.gemm_fp8_blockscaled(torch.zeros(8, 256, dtype=torch.uint8), torch.zeros(2, 8, dtype=bf),
+                                        torch.zeros(24, 256, dtype=torch.uint8), torch.zeros(2, 1)),  # sa type
+        lambda: sg.gemm_bf16_grouped([A], [B], outs=[torch.zeros(8, 20, dtype=bf)]),       # group output
+        lambda: sg.gemm_bf16_grouped([A, A], [B, B], biases=[torch.zeros(24), torch.zeros(24, dtype=bf)]),
+    ]
+    for i, f in enumerate(bad_calls):
+        with pytest.raises(ValueError):
+            f()
+        assert rec.calls == 0, f"call {i} reached the library"
+    # the well-formed versions do reach it
+    sg.gemm_bf16(A, B, bias=torch.zeros(24, dtype=bf), out=torch.zeros(8, 24))
+    sg.gemm_bf16_fp8out(A, B)
+    sg.gemm_bf16_logsoftmax(A, B)
+    sg.quantize_fp8_blockwise(torch.zeros(4, 256))
+    sg.quantize_fp8_blockwise(torch.zeros(256, 4), 128)
+    sg.gemm_fp8_blockscaled(torch.zeros(8, 256, dtype=torch.uint8), torch.zeros(2, 8),
+                            torch.zeros(24, 256, dtype=torch.uint8), torch.zeros(2, 1))
+    sg.gemm_bf16_grouped([A, A], [B, B], biases=[torch.zeros(24), None])
+    assert rec.calls == 7
