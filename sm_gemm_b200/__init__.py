@@ -156,6 +156,15 @@ def _out_matrix(t, M, N, name, dtypes=None):
         _dtype_code(t.dtype)
 
 
+def _ldc(out, M, N):
+    """Row pitch of an output. A single row's pitch is never used to address anything,
+    so it is rounded up to 16 elements (16-byte aligned for every output type) instead
+    of failing the library's pitch-alignment check (a one-token LM head with an odd
+    vocabulary size)."""
+    ld = max(out.stride(0), N)
+    return -(-ld // 16) * 16 if M == 1 else ld
+
+
 def _ws_bytes(workspace):
     _dense(workspace, "workspace")
     return workspace.numel() * workspace.element_size()
@@ -261,7 +270,7 @@ def gemm_bf16(A, B, *, bias=None, act="none", out=None, out_dtype=None, workspac
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype or A.dtype, device=A.device)
     _out_matrix(out, M, N, "out")
-    ldc = max(out.stride(0), N)
+    ldc = _ldc(out, M, N)
     sh = _stream(stream)
     ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else \
         _workspace(workspace_size(M, N, K, 0), A.device, sh)
@@ -300,7 +309,7 @@ def gemm_bf16_fp8out(A, B, *, bias=None, act="none", Q=None, scales=None, worksp
     _shape(scales, (-(-N // 128), M), "scales")
     _dense(scales, "scales")
     _need(scales.dtype == torch.float32, "scales must be float32")
-    ldc = max(Q.stride(0), N)
+    ldc = _ldc(Q, M, N)
     sh = _stream(stream)
     ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else \
         _workspace(workspace_size(M, N, K, 0), A.device, sh)
@@ -332,7 +341,7 @@ def gemm_bf16_logsoftmax(A, B, *, bias=None, out=None, workspace=None, stream=No
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=A.device)
     _out_matrix(out, M, N, "out", (torch.float32,))
-    ldc = max(out.stride(0), N)
+    ldc = _ldc(out, M, N)
     sh = _stream(stream)
     ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else \
         _workspace(int(lib().smgemm_logsoftmax_workspace_size(M, N, K)), A.device, sh)
@@ -379,7 +388,7 @@ def gemm_bf16_grouped(As, Bs, *, biases=None, act="none", outs=None, out_dtype=N
         _need(out.dtype == (outs[0].dtype if outs is not None else out.dtype), "outputs must share one dtype")
         res.append(out)
         Ms.append(M); Ns.append(N); Ks.append(K); ldas.append(lda); ldbs.append(ldb)
-        ldcs.append(max(out.stride(0), N))
+        ldcs.append(_ldc(out, M, N))
     arr = lambda xs: (C.c_int64 * G)(*xs)
     ptrs = lambda ts: (C.c_void_p * G)(*[None if t is None else t.data_ptr() for t in ts])
     nbytes = int(lib().smgemm_grouped_workspace_size(G))
@@ -423,7 +432,7 @@ def gemm_fp8_blockscaled(Aq, sa, Bq, sb, *, bias=None, act="none", out=None, out
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=Aq.device)
     _out_matrix(out, M, N, "out")
-    ldc = max(out.stride(0), N)
+    ldc = _ldc(out, M, N)
     sh = _stream(stream)
     ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else \
         _workspace(workspace_size(M, N, K, 1), Aq.device, sh)

@@ -213,3 +213,21 @@ def test_shape_and_dtype_checks_refuse_before_the_library(monkeypatch):
                             torch.zeros(24, 256, dtype=torch.uint8), torch.zeros(2, 1))
     sg.gemm_bf16_grouped([A, A], [B, B], biases=[torch.zeros(24), None])
     assert rec.calls == 7
+
+
+def test_single_row_output_pitch_is_rounded(monkeypatch):
+    """A one-row output's pitch addresses nothing, so an odd width (a one-token LM head
+    over an odd vocabulary) gets a 16-element pitch instead of an alignment error;
+    outputs of several rows keep their real pitch."""
+    seen = []
+
+    class Lib(_CountingLib):
+        def gemm_bf16(self, *a):
+            seen.append(a[15])
+            return sg.OK
+
+    _host_only(monkeypatch, Lib())
+    bf = torch.bfloat16
+    sg.gemm_bf16(torch.zeros(1, 16, dtype=bf), torch.zeros(16, 50257, dtype=bf), out_dtype=torch.float32)
+    sg.gemm_bf16(torch.zeros(2, 16, dtype=bf), torch.zeros(16, 24, dtype=bf))
+    assert seen == [50272, 24]
