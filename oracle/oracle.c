@@ -101,17 +101,29 @@ void orc_round_array(const double* x, int64_t n, int dtype, double* out) {
 
 /* ---------------------------------------------------------------- activations (double) */
 
+/* sigmoid(z) = 1 / (1 + e^-z), written so that no step overflows or cancels: for z < 0
+ * it is e^z / (1 + e^z) with e^z <= 1. */
+static double orc_sigmoid(double z) {
+  if (z >= 0.0) return 1.0 / (1.0 + exp(-z));
+  const double e = exp(z);
+  return e / (1.0 + e);
+}
+
 double orc_act(double x, int act) {
   switch (act) {
     case ORC_ACT_NONE: return x;
     case ORC_ACT_GELU_TANH: {
-      /* GeLU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) */
+      /* GeLU, tanh form: 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3).
+       * Since 1 + tanh(u) = 2 / (1 + e^(-2u)), this is x * sigmoid(2u); it is evaluated
+       * in that form because 1 + tanh(u) cancels to nothing in double once u < -19
+       * (x < -7), where the true value is still far above the smallest output values. */
       const double c = sqrt(2.0 / M_PI);
-      return 0.5 * x * (1.0 + tanh(c * (x + 0.044715 * x * x * x)));
+      const double u = c * (x + 0.044715 * x * x * x);
+      return x * orc_sigmoid(2.0 * u);
     }
     case ORC_ACT_SILU:
       /* SiLU (Swish-1): x * sigmoid(x) = x / (1 + e^-x) */
-      return x / (1.0 + exp(-x));
+      return x * orc_sigmoid(x);
     default: return NAN;
   }
 }

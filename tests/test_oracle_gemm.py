@@ -137,6 +137,50 @@ def test_activations_against_torch():
     assert math.isclose(oracle.act(40.0, oracle.ACT_SILU), 40.0, rel_tol=1e-15)
 
 
+def _gelu_tanh_decimal(x: float) -> "Decimal":
+    """0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3), in 200-digit decimal
+    arithmetic with tanh(u) = (e^(2u) - 1) / (e^(2u) + 1): the definition as written,
+    accurate even where 1 + tanh(u) is below 1e-100."""
+    from decimal import Decimal, localcontext
+    with localcontext() as ctx:
+        ctx.prec, ctx.Emax, ctx.Emin = 200, 10 ** 9, -10 ** 9
+        xd = Decimal(x)
+        pi = Decimal("3.14159265358979323846264338327950288419716939937510582097494459230781640628620899863")
+        c = (Decimal(2) / pi).sqrt()
+        u = c * (xd + Decimal("0.044715") * xd * xd * xd)
+        e = (2 * u).exp()
+        return Decimal("0.5") * xd * (1 + (e - 1) / (e + 1))
+
+
+def _silu_decimal(x: float) -> "Decimal":
+    from decimal import Decimal, localcontext
+    with localcontext() as ctx:
+        ctx.prec, ctx.Emax, ctx.Emin = 200, 10 ** 9, -10 ** 9
+        xd = Decimal(x)
+        return xd / (1 + (-xd).exp())
+
+
+def test_activations_against_high_precision():
+    """GeLU (tanh form) and SiLU over [-15, 15] and a few large magnitudes, against the
+    definitions evaluated in 200-digit decimal arithmetic: relative error at most 1e-13
+    everywhere, including the negative tails where the values are tiny (GeLU(-12) is
+    about 1e-53) and any cancellation in 1 + tanh(u) would show."""
+    from decimal import Decimal
+    xs = [float(v) for v in np.linspace(-15, 15, 1201)] + [-40.0, -80.0, -300.0, 1e-20, -1e-20, 37.5, 500.0]
+    for x in xs:
+        for which, ref_fn in ((oracle.ACT_GELU_TANH, _gelu_tanh_decimal), (oracle.ACT_SILU, _silu_decimal)):
+            got = oracle.act(x, which)
+            ref = ref_fn(x)
+            if ref == 0:
+                assert got == 0.0
+                continue
+            if abs(ref) < Decimal("1e-300"):        # below the normal double range: compare absolutely
+                assert abs(Decimal(got) - ref) < Decimal("1e-310"), (which, x, got, ref)
+                continue
+            rel = abs((Decimal(got) - ref) / ref)
+            assert rel < Decimal("1e-13"), (which, x, got, float(ref), float(rel))
+
+
 def test_bias_then_activation_then_one_cast():
     K = 16
     A = np.zeros((3, K), dtype=np.float16)
