@@ -24,32 +24,67 @@ struct EpiArgs {
   float* scales;       // E4M3 output only: [ceil(N/128)][M] group scales
 };
 
-// Activations in FP32. The GEMM epilogues use the hardware tanh.approx.f32 (maximum
-// relative error about 2^-11, some 16x below half a bf16 ulp) and the fast exponential
-// __expf: the GeLU/SiLU arithmetic then stays a few instructions per element, so the
-// epilogue warps keep pace with the tensor cores. act_apply_precise uses the libm
-// functions (tanhf, expf) for the K == 0 fill, which has no GEMM to hide behind.
-__device__ __forceinline__ float tanh_approx(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
+// Activations. Both are x * sigmoid(z): SiLU with z = x, and the tanh-form GeLU with
+// z = 2u, u = sqrt(2/pi) (x + 0.044715 x^3), because 0.5 x (1 + tanh(u)) = x / (1 + e^(-2u)).
+// The sigmoid is taken as 1 / (1 + e) for z >= 0 and e / (1 + e) for z < 0, with
+// e = e^(-|z|) <= 1: nothing overflows and nothing cancels, so the result keeps its
+// relative accuracy far out in the negative tail, where 1 + tanh(u) would round to
+// nothing (x < -5 in FP32).
+//
+// 16-bit and FP8 outputs use the FP32 form below: e^(-a) = 2^(-a log2 e) on the
+// special-function unit (ex2.approx.f32, results down to the subnormal range kept) and
+// an approximate reciprocal of 1 + e in [1, 2]. Its relative error is below 2^-16 for
+// every input (the rounding of a log2 e, |a| log2 e <= 150, is the largest term),
+// against the 2^-8 (BF16) and 2^-11 (FP16) spacing of the outputs, and the GeLU/SiLU
+// arithmetic stays a dozen instructions per element, so the epilogue warps keep pace
+// with the tensor cores. FP32 outputs add the bias and evaluate the activation in
+// double precision (libm exp) and round once, so they are within one FP32 ulp of the
+// exact value even where the accumulator contributes nothing.
+__device__ __forceinline__ float exp2_sfu(float y) {
+  float r;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(r) : "f"(y));
+  return r;
+}
+
+__device__ __forceinline__ float rcp_sfu(float d) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
+  return r;
+}
+
+// x * sigmoid(z) in FP32. Below 2^-120, e = 2^t is formed as 2^(t + 64) * 2^-64, so the
+// final multiply (IEEE, subnormals kept) rounds it into the subnormal range correctly
+// whatever the special-function unit does with subnormal results.
+__device__ __forceinline__ float x_sigmoid_f32(float x, float z) {
+  const float t = -fabsf(z) * 1.4426950408889634f;  // log2(e)
+  const bool tiny = t < -120.0f;
+  float e = exp2_sfu(tiny ? t + 64.0f : t);
+  if (tiny) e *= 5.421010862427522e-20f;           // 2^-64
+  const float r = rcp_sfu(1.0f + e);
+  return z >= 0.0f ? x * r : (x * e) * r;
 }
 
 __device__ __forceinline__ float act_apply(float x, int act) {
-  if (act == 1) {  // GeLU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
-    const float c = 0.7978845608028654f;  // sqrt(2/pi)
-    return 0.5f * x * (1.0f + tanh_approx(c * (x + 0.044715f * x * x * x)));
+  if (act == 1) {
+    const float u = 0.7978845608028654f * (x + 0.044715f * x * x * x);  // sqrt(2/pi) (x + 0.044715 x^3)
+    return x_sigmoid_f32(x, 2.0f * u);
   }
-  if (act == 2) return x / (1.0f + __expf(-x));  // SiLU: x * sigmoid(x)
+  if (act == 2) return x_sigmoid_f32(x, x);
   return x;
 }
 
-__device__ __forceinline__ float act_apply_precise(float x, int act) {
+__device__ __forceinline__ double x_sigmoid_f64(double x, double z) {
+  const double e = exp(-fabs(z));
+  const double r = 1.0 / (1.0 + e);
+  return z >= 0.0 ? x * r : (x * e) * r;
+}
+
+__device__ __forceinline__ double act_apply_f64(double x, int act) {
   if (act == 1) {
-    const float c = 0.7978845608028654f;
-    return 0.5f * x * (1.0f + tanhf(c * (x + 0.044715f * x * x * x)));
+    const double u = 0.79788456080286535588 * (x + 0.044715 * x * x * x);
+    return x_sigmoid_f64(x, 2.0 * u);
   }
-  if (act == 2) return x / (1.0f + expf(-x));
+  if (act == 2) return x_sigmoid_f64(x, x);
   return x;
 }
 
@@ -104,7 +139,26 @@ __device__ __forceinline__ void add_bias32_vec(const EpiArgs& e, int col0, float
   }
 }
 
+// FP32 output with an activation: bias add and activation in double, one rounding.
+// The loop is not unrolled (one copy of the double-precision code) and always works
+// on v[0], rotating the array by one after each element, so v stays in registers.
+__device__ __forceinline__ void epi_bias_act32_f64(const EpiArgs& e, int col0, float (&v)[32]) {
+#pragma unroll 1
+  for (int j = 0; j < 32; ++j) {
+    double x = static_cast<double>(v[0]);
+    if (e.bias != nullptr && col0 + j < e.N) x += static_cast<double>(load_bias(e.bias, e.bias_dtype, col0 + j));
+    const float y = __double2float_rn(act_apply_f64(x, e.act));
+#pragma unroll
+    for (int k = 0; k < 31; ++k) v[k] = v[k + 1];
+    v[31] = y;
+  }
+}
+
 __device__ __forceinline__ void epi_bias_act32(const EpiArgs& e, int col0, float (&v)[32]) {
+  if (e.act != 0 && e.c_dtype == 0) {
+    epi_bias_act32_f64(e, col0, v);
+    return;
+  }
   if (e.bias != nullptr) {
     const int esz = e.bias_dtype == 0 ? 4 : 2;
     const bool aligned = ((reinterpret_cast<uintptr_t>(e.bias) + static_cast<uintptr_t>(col0) * esz) & 15u) == 0;
@@ -237,6 +291,23 @@ template <int CNT>
 __device__ __forceinline__ void epi_col(const EpiArgs& e, int col, int row0, const float* v) {
   if (col >= e.N) return;
   const float b = e.bias != nullptr ? load_bias(e.bias, e.bias_dtype, col) : 0.0f;
+  if (e.act != 0 && e.c_dtype == 0) {
+    // FP32 output with an activation: in double, one element per iteration from w[0]
+    // with the copy rotated after each (w stays in registers; see epi_bias_act32_f64).
+    float w[CNT];
+#pragma unroll
+    for (int j = 0; j < CNT; ++j) w[j] = v[j];
+#pragma unroll 1
+    for (int j = 0; j < CNT; ++j) {
+      const int row = row0 + j;
+      if (row < e.M)
+        static_cast<float*>(e.C)[static_cast<long long>(row) * e.ldc + col] =
+            __double2float_rn(act_apply_f64(static_cast<double>(w[0]) + static_cast<double>(b), e.act));
+#pragma unroll
+      for (int k = 0; k + 1 < CNT; ++k) w[k] = w[k + 1];
+    }
+    return;
+  }
 #pragma unroll
   for (int j = 0; j < CNT; ++j) {
     const int row = row0 + j;

@@ -356,8 +356,13 @@ __global__ void fill_epilogue_kernel(int M, int N, const void* bias, int bias_dt
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long r = i / N, c = i - r * N;
-    const float b = bias != nullptr ? load_bias(bias, bias_dtype, static_cast<int>(c)) : 0.0f;
-    store_one(C, c_dtype, r * ldc + c, act_apply_precise(b, act));
+    // act(bias) in double, rounded once to the output type.
+    const double b = bias != nullptr ? static_cast<double>(load_bias(bias, bias_dtype, static_cast<int>(c))) : 0.0;
+    const double y = act_apply_f64(b, act);
+    const long long off = r * ldc + c;
+    if (c_dtype == 0) static_cast<float*>(C)[off] = __double2float_rn(y);
+    else if (c_dtype == 1) static_cast<__nv_bfloat16*>(C)[off] = __double2bfloat16(y);
+    else static_cast<__half*>(C)[off] = __double2half(y);
   }
 }
 
