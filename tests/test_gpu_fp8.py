@@ -13,7 +13,7 @@ import torch
 import oracle
 import sm_gemm_b200 as sg
 import synth
-from _parity import check_tolerance
+from _parity import TORCH_TO_ORC, check_tolerance, orc_view
 
 pytestmark = pytest.mark.gpu
 
@@ -255,3 +255,70 @@ def test_quantise_then_gemm_end_to_end_on_gpu(cuda_device):
     assert np.array_equal(qa.cpu().numpy(), qa_r) and np.array_equal(qb.cpu().numpy(), qb_r)
     ref, acc = oracle.gemm_fp8(qa_r, sa_r, qb_r, sb_r, out_dtype=oracle.BF16, want_absacc=True)
     check_tolerance(out.float().cpu().numpy(), ref, acc, torch.bfloat16, what="quant+gemm")
+
+
+# ------------------------------------------------------------------ partial last scale group (K % 128 != 0)
+
+@pytest.mark.parametrize("K", [144, 400, 4112])
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_fp8_ragged_k_quantise_then_gemm(cuda_device, monkeypatch, K, pair):
+    """K not a multiple of 128: the last 1x128 group of every A row and the last
+    128 x 128 block row of B hold K mod 128 elements, their scales come from those
+    elements only, and the codes past K are never read (TMA zero fill). Both
+    quantisations run on the GPU and must equal the oracle's bit for bit; the GEMM is
+    then checked against the oracle on the same operands, on the CTA-pair (pair=1) and
+    the one-SM (pair=0) kernels."""
+    monkeypatch.setenv("SMGEMM_PAIR", pair)
+    M, N = 300, 260
+    A = synth.normal_with_outliers(81, K, (M, K))
+    B = synth.normal_with_outliers(82, K, (K, N))
+    qa, sa = sg.quantize_fp8_blockwise(torch.from_numpy(A).cuda(), 1)
+    qb, sb = sg.quantize_fp8_blockwise(torch.from_numpy(B).cuda(), 128)
+    assert sg.check() == sg.OK
+    qa_r, sa_r = oracle.quant_1x128(A)
+    qb_r, sb_r = oracle.quant_128x128(B)
+    assert np.array_equal(qa.cpu().numpy(), qa_r) and np.array_equal(sa.cpu().numpy().view(np.uint32),
+                                                                     sa_r.view(np.uint32))
+    assert np.array_equal(qb.cpu().numpy(), qb_r) and np.array_equal(sb.cpu().numpy().view(np.uint32),
+                                                                     sb_r.view(np.uint32))
+    out = torch.empty((M, -(-N // 8) * 8), dtype=torch.bfloat16, device="cuda")[:, :N]   # 16-byte row pitch
+    sg.gemm_fp8_blockscaled(qa, sa, qb, sb, out=out)
+    assert sg.check() == sg.OK
+    ref, acc = oracle.gemm_fp8(qa_r, sa_r, qb_r, sb_r, out_dtype=oracle.BF16, want_absacc=True)
+    check_tolerance(out.float().cpu().numpy(), ref, acc, torch.bfloat16, what=f"ragged K={K} pair={pair}")
+
+
+@pytest.mark.parametrize("K", [144, 400, 4112])
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_fp8_ragged_k_integer_codes_exact(cuda_device, monkeypatch, K, pair):
+    """Integer codes with unit scales and a partial last K-block: every partial sum is
+    exact, so the output equals the oracle's bit for bit; a code read past K (instead of
+    the zero fill) or a dropped partial block would change it."""
+    monkeypatch.setenv("SMGEMM_PAIR", pair)
+    rs = np.random.RandomState(K)
+    M, N = 260, 300
+    qa = oracle.e4m3_encode(rs.randint(-8, 9, (M, K)).astype(np.float32))
+    qb = oracle.e4m3_encode(rs.randint(-8, 9, (N, K)).astype(np.float32))
+    kb = -(-K // 128)
+    sa = np.ones((kb, M), np.float32)
+    sb = np.ones((kb, -(-N // 128)), np.float32)
+    # rows are K apart, so bytes past K in a row are the next row's (non-zero) codes:
+    # only the tensor map's bounds keep them out of the last K-block
+    got = _run_fp8(qa, sa, qb, sb, out_dt=torch.float32)
+    ref = oracle.gemm_fp8(qa, sa, qb, sb, out_dtype=oracle.F32)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("out_dt", [torch.float16, torch.float32])
+@pytest.mark.parametrize("bias_dt", [torch.float32, torch.float16])
+@pytest.mark.parametrize("pair", ["1", "0"])
+def test_fp8_gemm_output_and_bias_types(cuda_device, monkeypatch, out_dt, bias_dt, pair):
+    """F16 and F32 outputs with F32 and F16 bias (and SiLU) on both FP8 kernels."""
+    monkeypatch.setenv("SMGEMM_PAIR", pair)
+    qa, sa, qb, sb = _quantised_problem(200, 300, 400, seed=83)
+    bias = torch.from_numpy(synth.normal(83, 5, (300,), 0.5)).to(bias_dt)
+    got = _run_fp8(qa, sa, qb, sb, out_dt=out_dt, bias=bias, act="silu")
+    bb, bd = orc_view(bias)
+    ref, acc = oracle.gemm_fp8(qa, sa, qb, sb, bias=bb, bias_dtype=bd, act=oracle.ACT_SILU,
+                               out_dtype=TORCH_TO_ORC[out_dt], want_absacc=True)
+    check_tolerance(got, ref, acc, out_dt, what=f"fp8 out={out_dt} bias={bias_dt}")
