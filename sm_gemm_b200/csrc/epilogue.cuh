@@ -286,6 +286,58 @@ __device__ __forceinline__ void epi_group_fp8_regs(const EpiArgs& e, int row, in
   e.scales[static_cast<long long>(col0 / 128) * e.M + row] = sc;
 }
 
+// FP8 output in two passes over a 1x128 group of one row, 32 columns at a time, so the
+// code stays one loop body per pass (the group is not held in registers): pass 1 loads
+// each raw chunk (load(c, v): c = 0..3), applies bias and activation, folds the chunk
+// into the group's amax and hands it back (keep(c, v), e.g. a store to TMEM, which then
+// serves the chunk to pass 2); pass 2 fetches the finished chunk again (again(c, v)),
+// divides by the group scale and stores the codes. Same encoding as epi_group_fp8_regs.
+template <class Load, class Keep, class Again>
+__device__ __forceinline__ void epi_group_fp8_2pass(const EpiArgs& e, int row, int col0, Load load, Keep keep,
+                                                    Again again) {
+  const bool full = col0 + 128 <= e.N;
+  float amax = 0.0f;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    float v[32];
+    load(c, v);
+    if (e.bias != nullptr || e.act != 0) epi_bias_act32(e, col0 + 32 * c, v);
+    if (full) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + 32 * c + j < e.N) amax = fmaxf(amax, fabsf(v[j]));
+    }
+    keep(c, v);
+  }
+  const float sc = group_scale(amax);
+  const bool fast = markstein_ok(sc);
+  const MarksteinDiv md = markstein_div(sc);
+  const bool live = row < e.M && col0 < e.N;
+  uint8_t* dst = static_cast<uint8_t*>(e.C) + static_cast<long long>(row) * e.ldc + col0;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    float v[32];
+    again(c, v);
+    uint32_t w[8];
+    if (fast) encode32(md, v, w);
+    else encode32(ExactDiv{sc}, v, w);
+    if (!live) continue;
+    if (full) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+      d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + 32 * c + j < e.N) dst[32 * c + j] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
+    }
+  }
+  if (live) e.scales[static_cast<long long>(col0 / 128) * e.M + row] = sc;
+}
+
 // CNT consecutive output rows row0.. of one column (transposed accumulator tiles).
 template <int CNT>
 __device__ __forceinline__ void epi_col(const EpiArgs& e, int col, int row0, const float* v) {

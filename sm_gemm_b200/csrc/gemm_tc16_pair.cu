@@ -16,8 +16,11 @@
 //  Both run their loops on the whole warp, so descriptors and coordinates stay in
 //  warp-uniform registers, and one elected lane issues.
 //  warp 2   TMEM allocator (cta_group::2, 512 columns = two 256-column accumulators).
-//  warps 4-7 epilogue: each CTA drains its own 128 rows; they release the accumulator
-//           to the rank-0 MMA issuer with a cluster-scope arrive.
+//  warps 4-11 epilogue: each CTA drains its own 128 rows; warp w reads TMEM lanes
+//           32*(w%4).. and the 128 columns 128*((w-4)/4).. of the tile, so two warps on
+//           each SM sub-partition share the work and the epilogue of the CTA's last
+//           tile (which nothing overlaps) takes half as long as with one. They release
+//           the accumulator to the rank-0 MMA issuer with a cluster-scope arrive.
 // Stream-K partial tiles are kept per (cluster, slot, rank) and reduced per rank.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -30,8 +33,11 @@
 namespace smg {
 
 namespace {
-constexpr int kThreads = 256;
 constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 32 * kEpiWarp0 + kEpiThreads;
+constexpr int kEpiCols = 128;  // tile columns per epilogue warp
 constexpr int kTileN = 256;  // columns of the pair tile (128 per CTA for B, all 256 in each TMEM)
 constexpr int kTcols = 512;
 }  // namespace
@@ -72,7 +78,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 8);
+      mbar_init(tempty_bar(b), 2 * kEpiWarps);  // every epilogue warp of both CTAs
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -180,9 +186,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;
+    const int cq = (warp - kEpiWarp0) >> 2;  // which 128-column half of the tile
     const int r_local = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     const int epi_tid = threadIdx.x - kEpiWarp0 * 32;
+    const int c_base = cq * kEpiCols;        // first tile column of this warp
     constexpr int SLOT = 128 * kTileN;
     int local = 0;
     WorkIter it;
@@ -197,30 +205,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       int mt, nt;
       tile_coords(s, seg.tile, mt, nt);
       const int row = mt * 256 + static_cast<int>(rank) * 128 + r_local;
-      const uint32_t tacc = tmem_base + lane_addr + acc * kTileN;
+      const uint32_t tacc = tmem_base + lane_addr + acc * kTileN + c_base;
+      const int col0 = nt * kTileN + c_base;
       const bool whole = (seg.kb0 == 0 && seg.kb1 == s.kb_total);
       float* my_slot = p.slots + ((static_cast<size_t>(cluster) * 2 + seg.slot) * 2 + rank) * SLOT;
       if (!dead) {
         tc_fence_after();
         if constexpr (FP8OUT) {
-          // Each 128-column half of the tile is one 1x128 group of the row, read from
-          // TMEM once into registers (stream-K partials go to the slots unchanged).
-#pragma unroll 1
-          for (int gq = 0; gq < kTileN / 128; ++gq) {
-            float g[128];
+          // This warp's 128 columns are one 1x128 group of each row: two passes over
+          // TMEM, the activated values written back in place between them.
+          auto load = [&](int c, float (&v)[32]) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32_sync(tacc + c * 32, r);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          };
+          if (whole) {
+            auto keep = [&](int c, const float (&v)[32]) {
               uint32_t r[32];
-              tmem_ld_32x32b_x32_sync(tacc + gq * 128 + c * 32, r);
 #pragma unroll
-              for (int j = 0; j < 32; ++j) g[32 * c + j] = __uint_as_float(r[j]);
+              for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(v[j]);
+              tmem_st_32x32b_x32(tacc + c * 32, r);
+            };
+            // The stores of pass 1 complete before pass 2 reads the columns back.
+            auto again = [&](int c, float (&v)[32]) {
+              if (c == 0) tmem_st_wait();
+              load(c, v);
+            };
+            epi_group_fp8_2pass(p.e, row, col0, load, keep, again);
+          } else {
+#pragma unroll 1
+            for (int c = 0; c < kEpiCols / 32; ++c) {
+              float v[32];
+              load(c, v);
+              slot_store<32>(my_slot, r_local, c_base + c * 32, v);
             }
-            if (whole) epi_group_fp8_regs(p.e, row, nt * kTileN + gq * 128, g);
-            else slot_store<128>(my_slot, r_local, gq * 128, g);
           }
         } else {
 #pragma unroll 1
-          for (int c = 0; c < kTileN / 32; ++c) {
+          for (int c = 0; c < kEpiCols / 32; ++c) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(tacc + c * 32, r);
             tmem_ld_wait();
@@ -228,9 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
             if (whole) {
-              epi_row32(p.e, row, nt * kTileN + c * 32, v);
+              epi_row32(p.e, row, col0 + c * 32, v);
             } else {
-              slot_store<32>(my_slot, r_local, c * 32, v);
+              slot_store<32>(my_slot, r_local, c_base + c * 32, v);
             }
           }
         }
@@ -242,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!whole) {
         const long long t_sk = seg.tile - s.dp_tiles;
         __threadfence();
-        named_barrier_sync(1, 128);
+        named_barrier_sync(1, kEpiThreads);
         if (epi_tid == 0) {
           const int c_lo = sk_owner(s, t_sk * s.kb_total);
           const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
@@ -252,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int old = any_dead ? -1 : atomicAdd(p.counters + t_sk * 2 + rank, 1);
           *reduce_flag = (!any_dead && old == n - 1);
         }
-        named_barrier_sync(1, 128);
+        named_barrier_sync(1, kEpiThreads);
         if (*reduce_flag) {
           __threadfence();
           const int c_lo = sk_owner(s, t_sk * s.kb_total);
@@ -269,23 +292,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           };
           if constexpr (FP8OUT) {
-#pragma unroll 1
-            for (int gq = 0; gq < kTileN / 128; ++gq) {
-              float g[128];
-#pragma unroll
-              for (int c = 0; c < 4; ++c) reduce32(gq * 128 + c * 32, *reinterpret_cast<float(*)[32]>(g + 32 * c));
-              epi_group_fp8_regs(p.e, row, nt * kTileN + gq * 128, g);
-            }
+            // No TMEM to keep the activated chunks in: pass 2 sums the partials again
+            // and re-applies bias and activation (the same arithmetic, the same values).
+            auto load = [&](int c, float (&v)[32]) { reduce32(c_base + c * 32, v); };
+            auto keep = [&](int, const float (&)[32]) {};
+            auto again = [&](int c, float (&v)[32]) {
+              reduce32(c_base + c * 32, v);
+              if (p.e.bias != nullptr || p.e.act != 0) epi_bias_act32(p.e, col0 + 32 * c, v);
+            };
+            epi_group_fp8_2pass(p.e, row, col0, load, keep, again);
           } else {
 #pragma unroll 1
-            for (int c = 0; c < kTileN / 32; ++c) {
+            for (int c = 0; c < kEpiCols / 32; ++c) {
               float v[32];
-              reduce32(c * 32, v);
-              epi_row32(p.e, row, nt * kTileN + c * 32, v);
+              reduce32(c_base + c * 32, v);
+              epi_row32(p.e, row, col0 + c * 32, v);
             }
           }
         }
-        named_barrier_sync(1, 128);
+        named_barrier_sync(1, kEpiThreads);
       }
       ++local;
     }
