@@ -472,13 +472,39 @@ def wl_lm_head(c: Ctx, ms_list=(1, 4, 16, 64)):
              extra={"plan": sg.last_config()})
 
 
+def wl_lm_head_vocab_parallel(c: Ctx, mm: int = 16):
+    """The LM head (M = 16, V = 128256) with its row log-softmax, its vocabulary split over
+    the ranks (each streams only its slice of W): GEMM with (max, sum exp) partials on the
+    slice, all-gather of the partials (NCCL), merge and subtract. Strong scaling: the whole
+    job is one LM head whatever the rank count; GB/s counts the whole head's bytes."""
+    torch, sg, m = c.torch, c.sg, c.metrics
+    from sm_gemm_b200 import vocab_parallel as vp
+    V, K = 128256, 4096
+    rank = c.dist.get_rank() if c.dist is not None else 0
+    c0, c1 = vp.shard_columns(V, c.world, rank)
+    d = c.synth.lm_head(m=mm)
+    Xl = c.t(d["X"])
+    Ws = c.t(np.ascontiguousarray(d["W"][:, c0:c1]))
+    del d
+    Cl = torch.empty((mm, c1 - c0), dtype=torch.float32, device=c.dev)
+    ws = torch.empty(max(sg.workspace_size(mm, max(c1 - c0, 1), K), 16), dtype=torch.uint8, device=c.dev)
+    # our kernels per step: the skinny GEMM (its epilogue forms the partials), the lse merge
+    # and the subtract; the all-gather is NCCL's and the padding of short slices torch's
+    ms = c.time(lambda i: vp.lm_head_log_softmax(Xl, Ws, V, dist=c.dist, out=Cl, workspace=ws),
+                launches_per_step=3)
+    c.record(f"lm_head_logsoftmax_vocab_parallel_m{mm}", ms, c.K, flops=m.gemm_flops(mm, V, K),
+             nbytes=m.gemm_bytes(mm, V, K, "bf16", "bf16", "f32") + 2 * mm * V * 4,
+             extra={"ranks": c.world, "slice_columns": c1 - c0, "scaling": "strong",
+                    "exchange": "all-gather of per-tile (max, sum exp) pairs" if c.world > 1 else "none"})
+
+
 def run_gpu(args, rank: int, world: int, dist):
     c = Ctx(args, world, dist)
     if args.only is not None and args.only != "square_bf16":
         {"tiny_fp16": lambda: wl_tiny_fp16(c), "ffn": lambda: wl_ffn(c),
          "fp8": lambda: wl_fp8(c, quant=False), "quant": lambda: wl_fp8(c, gemm=False),
          "ffn_bwd": lambda: wl_ffn_backward(c), "grouped": lambda: wl_grouped(c),
-         "lm_head": lambda: wl_lm_head(c)}[args.only]()
+         "lm_head": lambda: wl_lm_head(c), "lm_head_vp": lambda: wl_lm_head_vocab_parallel(c)}[args.only]()
         assert c.sg.check() == c.sg.OK
         return {"only": args.only, "steps": c.K, "warmup": c.W, "gpu_launches": c.launches, "configs": c.results}
 
@@ -490,6 +516,7 @@ def run_gpu(args, rank: int, world: int, dist):
         wl_grouped(c)
         wl_fp8(c)
         wl_lm_head(c)
+        wl_lm_head_vocab_parallel(c)
     assert c.sg.check() == c.sg.OK
     peaks = c.peaks
     per_launch_s = h["ms"] / c.K / 1e3
@@ -590,6 +617,25 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- main
 
+def launch_ranks(n: int) -> int:
+    """`--gpus n` without a launcher: start n ranks of this same command, one per GPU, with
+    torch.distributed.run on this node (rendezvous on 127.0.0.1), and return their exit
+    status. Refuses (status 2) when fewer than n GPUs are visible: it never times fewer
+    GPUs than asked for."""
+    import socket
+    import torch
+    have = torch.cuda.device_count()
+    if have < n:
+        print(f"bench.py: --gpus {n} but only {have} GPU(s) visible", file=sys.stderr)
+        return 2
+    with socket.socket() as sck:
+        sck.bind(("127.0.0.1", 0))
+        port = sck.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -598,15 +644,21 @@ def main():
     ap.add_argument("--impl", default="smgemm", choices=["smgemm", "reference"])
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--only", default=None,
-                    choices=["square_bf16", "tiny_fp16", "ffn", "ffn_bwd", "grouped", "fp8", "quant", "lm_head"],
+                    choices=["square_bf16", "tiny_fp16", "ffn", "ffn_bwd", "grouped", "fp8", "quant", "lm_head",
+                             "lm_head_vp"],
                     help="time one workload and print its line (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
+    if args.impl != "reference" and args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_ranks(args.gpus))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.impl != "reference" and world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        sys.exit(2)
 
     if args.impl == "reference":
         if rank == 0:

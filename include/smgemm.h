@@ -94,8 +94,11 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K,
  *   returns SMGEMM_ERR_WORKSPACE before enqueueing anything. The library allocates nothing.
  *   All calls share the array and it keeps the previous call's contents (each call
  *   clears what must start at zero); calls that can overlap on the GPU race on it.
- *   The first call on each device resolves the array's device address; make that
- *   first call before any stream capture.
+ *   The first call on each device resolves the array's device address; under CUDA's
+ *   default lazy module loading it also loads the library's device code there and
+ *   reserves the array (milliseconds, may synchronise), so make it during warm-up,
+ *   outside any latency-critical loop and before any stream capture. After
+ *   cudaDeviceReset the next call resolves the address again in the new context.
  */
 #define SMGEMM_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 smgemm_status gemm_bf16_noalloc(int64_t M, int64_t N, int64_t K,
@@ -114,13 +117,16 @@ smgemm_status gemm_bf16_noalloc(int64_t M, int64_t N, int64_t K,
  *              (nullable) device pointers.
  *   ab_dtype, layout_a, layout_b, bias_dtype, act, c_dtype: shared by all groups, as in
  *              gemm_bf16. Groups with M or N = 0 are skipped; K = 0 writes act(bias).
- *   workspace  device, at least smgemm_grouped_workspace_size(G) bytes: the host writes
+ *   workspace  device, 16-byte aligned (else SMGEMM_ERR_ALIGNMENT), at least
+ *              smgemm_grouped_workspace_size(G) bytes: the host writes
  *              the groups' TMA descriptors and sizes there (an asynchronous copy on
  *              `stream`, from pageable memory) before the launch; the rest holds the
  *              partial tiles of a split last wave. Calls that can overlap on the GPU
  *              must not share it. A smaller workspace that still holds the table is
  *              accepted; the last wave is then not split.
- * Every group is validated before anything is enqueued; errors as in gemm_bf16. Tiles
+ * Every group is validated, and every TMA descriptor encoded, before anything is
+ * enqueued; the descriptor table is copied first, then groups with K = 0 are filled,
+ * then the GEMM launches. Errors as in gemm_bf16. Tiles
  * of 256 x 256 run one per CTA pair; when the tiles do not fill a whole last wave, the
  * R tiles of that wave are each split along K into S = min(P / R, KB / 8) pieces (P
  * co-resident pairs, KB the smallest K-block count among those tiles) that run side
@@ -175,6 +181,38 @@ smgemm_status gemm_bf16_logsoftmax(int64_t M, int64_t N, int64_t K,
                                    const void* bias, smgemm_dtype bias_dtype,
                                    float* C, int64_t ldc,
                                    void* workspace, size_t workspace_bytes, smgemm_stream_t stream);
+
+/*
+ * Vocabulary-parallel LM head: the log-softmax of gemm_bf16_logsoftmax split in two steps,
+ * so that each GPU can hold only its slice of the vocabulary (the columns of W) and the
+ * ranks exchange nothing but the small per-row partials between the steps (the LM head is
+ * the memory-bound "thin and tall" GEMM of "为什么我们要死磕GEMM" (kwkr.cn), sections 2.2
+ * and 7.2; splitting its columns multiplies the HBM bandwidth that streams W).
+ *
+ * gemm_bf16_lse_partials: z = A[M,K] * B[K,N] + bias[N] in FP32, written to C (row-major,
+ *   ldc >= N, 16-byte aligned rows), and for every 128-column tile t < ceil(N/128) and row
+ *   m the pair part[2*(t*M + m) + 0/1] = (max of the tile's z, sum of exp(z - max)).
+ *   A, B, bias, layouts, lda, ldb: as in gemm_bf16 (no activation). part: device float
+ *   [ceil(N/128)][M][2], 16-byte aligned. workspace: smgemm_workspace_size(M,N,K,0) bytes.
+ *   On the skinny path the GEMM epilogue forms the pairs; otherwise a light pass over C does.
+ *
+ * logsoftmax_apply_partials: lse[m] = log sum over every column of exp(z), merged from
+ *   n_parts pairs part[2*(p*M + m) + 0/1], p < n_parts (for example every rank's partials,
+ *   gathered one rank after another; a pair (-inf, 0) is neutral), with the rule
+ *   (m1, s1) + (m2, s2) = (m, s1 e^(m1-m) + s2 e^(m2-m)), m = max(m1, m2), in a fixed order
+ *   (deterministic); then C[m, n] -= lse[m] for n < N (this rank's slice; N may be 0).
+ *   C: device float, ldc >= N, 16-byte aligned. part: device, 8-byte aligned. lse: device
+ *   float [M], written. n_parts >= 1.
+ * Errors as in gemm_bf16.
+ */
+smgemm_status gemm_bf16_lse_partials(int64_t M, int64_t N, int64_t K,
+                                     const void* A, smgemm_dtype ab_dtype, smgemm_layout layout_a, int64_t lda,
+                                     const void* B, smgemm_layout layout_b, int64_t ldb,
+                                     const void* bias, smgemm_dtype bias_dtype,
+                                     float* C, int64_t ldc, float* part,
+                                     void* workspace, size_t workspace_bytes, smgemm_stream_t stream);
+smgemm_status logsoftmax_apply_partials(float* C, int64_t ldc, int64_t M, int64_t N,
+                                        const float* part, int64_t n_parts, float* lse, smgemm_stream_t stream);
 
 /*
  * gemm_fp8_blockscaled: C[i,j] = cast_c( act( sum_kb sa[kb,i] * sb[kb, j/128] *

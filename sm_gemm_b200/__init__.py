@@ -80,6 +80,10 @@ def lib():
             L.smgemm_logsoftmax_workspace_size.restype = SZ
             L.gemm_bf16_fp8out.argtypes = [I64, I64, I64, P, I, I, I64, P, I, I64, P, I, I, P, I64, P, P, SZ, P]
             L.gemm_bf16_fp8out.restype = I
+            L.gemm_bf16_lse_partials.argtypes = [I64, I64, I64, P, I, I, I64, P, I, I64, P, I, P, I64, P, P, SZ, P]
+            L.gemm_bf16_lse_partials.restype = I
+            L.logsoftmax_apply_partials.argtypes = [P, I64, I64, I64, P, I64, P, P]
+            L.logsoftmax_apply_partials.restype = I
             _lib = L
     return _lib
 
@@ -128,30 +132,46 @@ def _device(*ts):
     return dev
 
 
-def _current_device():
-    return _torch().cuda.current_device()
+_getdev = None
 
+
+def _current_device():
+    """Index of the current CUDA device (torch's raw getter once torch is initialised)."""
+    global _getdev
+    if _getdev is None:
+        torch = _torch()
+        torch.cuda.init()
+        _getdev = getattr(torch._C, "_cuda_getDevice", None) or torch.cuda.current_device
+    return _getdev()
+
+
+# The checks below build their error messages only when a check fails: they run on
+# every call, and formatting a message costs as much as the check itself.
 
 def _shape(t, want, name):
-    _need(tuple(t.shape) == tuple(want), f"{name} must have shape {tuple(want)}, not {tuple(t.shape)}")
+    if tuple(t.shape) != tuple(want):
+        raise ValueError(f"{name} must have shape {tuple(want)}, not {tuple(t.shape)}")
 
 
 def _dense(t, name):
-    _need(t.is_contiguous(), f"{name} must be contiguous")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
 
 
 def _vector(t, n, name):
     """A bias: 1-D, unit stride, at least n elements."""
-    _need(t.dim() == 1 and t.shape[0] >= n and (t.shape[0] <= 1 or t.stride(0) == 1),
-          f"{name} must be a unit-stride vector of at least {n} elements")
+    if not (t.dim() == 1 and t.shape[0] >= n and (t.shape[0] <= 1 or t.stride(0) == 1)):
+        raise ValueError(f"{name} must be a unit-stride vector of at least {n} elements")
     _dtype_code(t.dtype)
 
 
 def _out_matrix(t, M, N, name, dtypes=None):
     _shape(t, (M, N), name)
-    _need(t.dim() == 2 and (t.stride(1) == 1 or N <= 1), f"{name} must be row-major")
+    if not (t.dim() == 2 and (t.stride(1) == 1 or N <= 1)):
+        raise ValueError(f"{name} must be row-major")
     if dtypes is not None:
-        _need(t.dtype in dtypes, f"{name} must be one of {dtypes}")
+        if t.dtype not in dtypes:
+            raise ValueError(f"{name} must be one of {dtypes}")
     else:
         _dtype_code(t.dtype)
 
@@ -351,6 +371,68 @@ def gemm_bf16_logsoftmax(A, B, *, bias=None, out=None, workspace=None, stream=No
                                     out.data_ptr(), ldc, None if ws is None else ws.data_ptr(), wsb, sh)
     _check(st, "gemm_bf16_logsoftmax")
     return out
+
+
+def gemm_bf16_lse_partials(A, B, *, bias=None, out=None, part=None, workspace=None, stream=None):
+    """Logits z = A @ B + bias (FP32 [M, N]) and, per 128-column tile t and row m, the pair
+    (max z, sum exp(z - max)) in part[t, m] (float32 [ceil(N/128), M, 2]): the first step of
+    a vocabulary-parallel log-softmax. Returns (out, part)."""
+    dev = _device(A, B, bias, out, part, workspace)
+    if dev != _current_device():
+        with _torch().cuda.device(dev):
+            return gemm_bf16_lse_partials(A, B, bias=bias, out=out, part=part, workspace=workspace, stream=stream)
+    torch = _torch()
+    M, K = A.shape
+    K2, N = B.shape
+    if K != K2 or A.dtype != B.dtype:
+        raise ValueError("A and B must agree in K and dtype")
+    la, lda = _layout(A, "A")
+    lb, ldb = _layout(B, "B")
+    if bias is not None:
+        _vector(bias, N, "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    _out_matrix(out, M, N, "out", (torch.float32,))
+    if part is None:
+        part = torch.empty((-(-N // 128), M, 2), dtype=torch.float32, device=A.device)
+    _shape(part, (-(-N // 128), M, 2), "part")
+    _dense(part, "part")
+    _need(part.dtype == torch.float32, "part must be float32")
+    ldc = _ldc(out, M, N)
+    sh = _stream(stream)
+    ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else \
+        _workspace(workspace_size(M, N, K, 0), A.device, sh)
+    st = lib().gemm_bf16_lse_partials(M, N, K, A.data_ptr(), _dtype_code(A.dtype), la, lda, B.data_ptr(), lb, ldb,
+                                      None if bias is None else bias.data_ptr(),
+                                      _dtype_code(bias.dtype) if bias is not None else 0,
+                                      out.data_ptr(), ldc, part.data_ptr(), None if ws is None else ws.data_ptr(),
+                                      wsb, sh)
+    _check(st, "gemm_bf16_lse_partials")
+    return out, part
+
+
+def logsoftmax_apply_partials(C, part, *, lse=None, stream=None):
+    """lse[m] merged from every pair part[p, m] (float32 [P, M, 2], e.g. all ranks' partials
+    stacked), then C[m, n] -= lse[m] in place (C: FP32 [M, N], N may be 0). Returns lse."""
+    dev = _device(C, part, lse)
+    if dev != _current_device():
+        with _torch().cuda.device(dev):
+            return logsoftmax_apply_partials(C, part, lse=lse, stream=stream)
+    torch = _torch()
+    M, N = C.shape
+    _need(part.dim() == 3 and part.shape[1] == M and part.shape[2] == 2, "part must be [P, M, 2]")
+    _dense(part, "part")
+    _need(part.dtype == torch.float32 and part.shape[0] >= 1, "part must be float32 with P >= 1")
+    if lse is None:
+        lse = torch.empty((M,), dtype=torch.float32, device=C.device)
+    _vector(lse, M, "lse")
+    _need(lse.dtype == torch.float32 and lse.is_contiguous(), "lse must be a contiguous float32 vector")
+    _out_matrix(C, M, N, "C", (torch.float32,))
+    ldc = _ldc(C, M, N)
+    st = lib().logsoftmax_apply_partials(C.data_ptr(), ldc, M, N, part.data_ptr(), part.shape[0], lse.data_ptr(),
+                                         _stream(stream))
+    _check(st, "logsoftmax_apply_partials")
+    return lse
 
 
 def gemm_bf16_grouped(As, Bs, *, biases=None, act="none", outs=None, out_dtype=None, workspace=None,

@@ -160,18 +160,58 @@ Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, siz
 
 // ------------------------------------------------------------------ TMA maps
 
+// A tensor map is a pure function of its arguments (it holds the global address, not a
+// handle to the allocation), so encoded maps are kept per host thread, keyed by every
+// argument, and a call on the same operand as a recent call reuses its map instead of
+// encoding it again (the shape -> descriptor cache of the DeepGEMM kernel-library
+// walkthrough (zwxr.cn), section 4.3). A stale entry for memory freed and reallocated at
+// the same address is still exactly the map an encode would produce.
+struct MapKey {
+  const void* base;
+  uint64_t inner, outer, stride;
+  uint32_t box_inner, box_outer;
+  int dt, swizzle;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && inner == o.inner && outer == o.outer && stride == o.stride &&
+           box_inner == o.box_inner && box_outer == o.box_outer && dt == o.dt && swizzle == o.swizzle;
+  }
+};
+
+struct MapCache {
+  static constexpr int kEntries = 32;
+  MapKey key[kEntries];
+  CUtensorMap map[kEntries];
+  bool used[kEntries] = {};
+  int next = 0;
+};
+
 bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
                uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+  thread_local MapCache cache;
+  const MapKey k{base, inner, outer, row_stride_bytes, box_inner, box_outer, static_cast<int>(dt),
+                 static_cast<int>(swizzle)};
+  for (int i = 0; i < MapCache::kEntries; ++i) {
+    if (cache.used[i] && cache.key[i] == k) {
+      *map = cache.map[i];
+      return true;
+    }
+  }
   PFN_encodeTiled fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_stride_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int slot = cache.next;
+  cache.next = (cache.next + 1) % MapCache::kEntries;
+  cache.key[slot] = k;
+  cache.map[slot] = *map;
+  cache.used[slot] = true;
+  return true;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -468,6 +508,43 @@ smgemm_status gemm_bf16_logsoftmax(int64_t M, int64_t N, int64_t K, const void* 
                                                stream));
 }
 
+smgemm_status gemm_bf16_lse_partials(int64_t M, int64_t N, int64_t K, const void* A, smgemm_dtype ab_dtype,
+                                     smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b,
+                                     int64_t ldb, const void* bias, smgemm_dtype bias_dtype, float* C, int64_t ldc,
+                                     float* part, void* workspace, size_t workspace_bytes, smgemm_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (M < 0 || N < 0 || K < 0) return SMGEMM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return SMGEMM_OK;
+  if (part == nullptr) return SMGEMM_ERR_INVALID_ARG;
+  if (!aligned16(part)) return SMGEMM_ERR_ALIGNMENT;
+  bool used = false;
+  smgemm_status st = gemm16_impl(M, N, K, A, ab_dtype, layout_a, lda, B, layout_b, ldb, bias, bias_dtype,
+                                 SMGEMM_ACT_NONE, C, SMGEMM_F32, ldc, workspace, workspace_bytes, stream,
+                                 reinterpret_cast<float2*>(part), &used);
+  if (st != SMGEMM_OK || used) return st;
+  // Large-tile path (or K = 0): the partials come from the logits just written.
+  return launch_status(launch_lse_tile_partials(C, ldc, static_cast<int>(M), static_cast<int>(N),
+                                                reinterpret_cast<float2*>(part), stream));
+}
+
+smgemm_status logsoftmax_apply_partials(float* C, int64_t ldc, int64_t M, int64_t N, const float* part,
+                                        int64_t n_parts, float* lse, smgemm_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (M < 0 || N < 0 || n_parts < 0 || !fits_int(M) || !fits_int(N) || !fits_int(n_parts))
+    return SMGEMM_ERR_INVALID_ARG;
+  if (M == 0) return SMGEMM_OK;
+  if (part == nullptr || lse == nullptr || n_parts == 0 || (N > 0 && (C == nullptr || ldc < N)))
+    return SMGEMM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(part) & 7u) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (N > 0 && !aligned16(C)))
+    return SMGEMM_ERR_ALIGNMENT;
+  DevInfo d;
+  if (current_device(d) != SMGEMM_OK) return SMGEMM_ERR_CUDA;
+  return launch_status(launch_log_softmax_rows(C, ldc, static_cast<int>(M), static_cast<int>(N),
+                                               reinterpret_cast<const float2*>(part), static_cast<int>(n_parts), lse,
+                                               d.sms, stream));
+}
+
 // Group table, then (when the device is known) room for splitting a ragged last wave:
 // one 2 x 128 x 256-float partial per cluster and two counters per split tile.
 size_t grouped_table_bytes(int G) { return (static_cast<size_t>(G) * sizeof(GroupDesc) + 64 + 255) / 256 * 256; }
@@ -512,6 +589,8 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
     }
   }
   if (workspace == nullptr || workspace_bytes < grouped_table_bytes(G)) return SMGEMM_ERR_WORKSPACE;
+  // The split-wave partials are read and written as float4 at workspace + table bytes.
+  if (!aligned16(workspace)) return SMGEMM_ERR_ALIGNMENT;
   DevInfo d;
   if (current_device(d) != SMGEMM_OK) return SMGEMM_ERR_CUDA;
   const CUtensorMapDataType dt =
@@ -521,6 +600,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   const bool b_mn = (layout_b == SMGEMM_ROW_MAJOR);
   const int bk = grouped_bk();
   std::vector<GroupDesc> table(static_cast<size_t>(G));
+  std::vector<int> fills;  // groups with K = 0: filled with act(bias) after the table is enqueued
   long long tiles = 0;
   for (int g = 0; g < G; ++g) {
     GroupDesc& e = table[static_cast<size_t>(g)];
@@ -533,9 +613,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
     e.bias = bias != nullptr ? bias[g] : nullptr;
     if (M[g] == 0 || N[g] == 0) continue;
     if (K[g] == 0) {  // no products: the output is act(bias) (or act(0))
-      smgemm_status st = launch_status(launch_fill_epilogue(e.M, e.N, e.bias, bias_dtype, act, C[g], c_dtype,
-                                                            ldc[g], stream));
-      if (st != SMGEMM_OK) return st;
+      fills.push_back(g);
       continue;
     }
     bool ok;
@@ -549,14 +627,21 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
     e.kb_total = static_cast<int>((K[g] + bk - 1) / bk);
     tiles += static_cast<long long>(e.m_tiles) * e.n_tiles;
   }
-  if (tiles == 0) return SMGEMM_OK;
+  const int clusters_max = tiles > 0 ? grouped_max_clusters() : 0;
+  if (tiles > 0 && clusters_max <= 0) return SMGEMM_ERR_CUDA;
   GroupDesc* dev_table = reinterpret_cast<GroupDesc*>((reinterpret_cast<uintptr_t>(workspace) + 63) & ~uintptr_t(63));
-  // Pageable source: the copy has consumed `table` by the time the call returns.
-  if (cudaMemcpyAsync(dev_table, table.data(), table.size() * sizeof(GroupDesc), cudaMemcpyHostToDevice, stream) !=
-      cudaSuccess)
+  // Pageable source: the copy has consumed `table` by the time the call returns. It is
+  // the first thing enqueued, so a failure here leaves every output untouched.
+  if (tiles > 0 && cudaMemcpyAsync(dev_table, table.data(), table.size() * sizeof(GroupDesc),
+                                   cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return launch_status(cudaGetLastError());
-  const int clusters_max = grouped_max_clusters();
-  if (clusters_max <= 0) return SMGEMM_ERR_CUDA;
+  for (int g : fills) {
+    const GroupDesc& e = table[static_cast<size_t>(g)];
+    smgemm_status st =
+        launch_status(launch_fill_epilogue(e.M, e.N, e.bias, bias_dtype, act, C[g], c_dtype, ldc[g], stream));
+    if (st != SMGEMM_OK) return st;
+  }
+  if (tiles == 0) return SMGEMM_OK;
   GroupedParams p{};
   p.groups = dev_table;
   p.G = G;

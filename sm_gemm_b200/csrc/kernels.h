@@ -53,6 +53,8 @@ int tc16_pair_bk();
 // C[m, n] -= lse[m].
 cudaError_t launch_log_softmax_rows(float* C, long long ldc, int M, int N, const float2* part, int n_tiles,
                                     float* lse, int sms, cudaStream_t stream);
+// Per-128-column-tile (max, sum of exp) partials of an FP32 [M, N] logit matrix, part[t * M + m].
+cudaError_t launch_lse_tile_partials(const float* C, long long ldc, int M, int N, float2* part, cudaStream_t stream);
 
 // Grouped GEMM (gemm_grouped.cu): one record per group in device memory, 64-byte
 // aligned (the TMA descriptors must be). tile0 = index of the group's first tile in the

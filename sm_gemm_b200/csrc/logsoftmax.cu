@@ -96,15 +96,47 @@ __global__ void __launch_bounds__(256) subtract_lse_kernel(float* __restrict__ C
   }
 }
 
+// One warp per (128-column tile t, row m) of an FP32 logit matrix: the tile's max logit and
+// sum of exp(logit - max), written to part[t * M + m] as on the swap-AB GEMM's epilogue
+// (columns past N contribute nothing; a tile with none gives the identity (-inf, 0)).
+__global__ void __launch_bounds__(256) lse_tile_partials_kernel(const float* __restrict__ C, long long ldc, int M,
+                                                                int N, int n_tiles, float2* __restrict__ part) {
+  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<long long>(M) * n_tiles) return;
+  const int t = static_cast<int>(w / M), m = static_cast<int>(w - static_cast<long long>(t) * M);
+  const float* row = C + static_cast<long long>(m) * ldc;
+  MaxSum v{-INFINITY, 0.0f};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int n = t * 128 + 32 * j + lane;
+    if (n < N) v = merge(v, MaxSum{row[n], 1.0f});
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    MaxSum u{__shfl_xor_sync(0xffffffffu, v.m, o), __shfl_xor_sync(0xffffffffu, v.s, o)};
+    v = merge(v, u);
+  }
+  if (lane == 0) part[static_cast<long long>(t) * M + m] = v.s > 0.0f ? make_float2(v.m, v.s) : make_float2(-INFINITY, 0.0f);
+}
+
 }  // namespace
+
+cudaError_t launch_lse_tile_partials(const float* C, long long ldc, int M, int N, float2* part, cudaStream_t stream) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  const int n_tiles = (N + 127) / 128;
+  const long long warps = static_cast<long long>(M) * n_tiles;
+  lse_tile_partials_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(C, ldc, M, N, n_tiles, part);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_log_softmax_rows(float* C, long long ldc, int M, int N, const float2* part, int n_tiles,
                                     float* lse, int sms, cudaStream_t stream) {
-  if (M <= 0 || N <= 0) return cudaSuccess;
+  if (M <= 0 || (part == nullptr && N <= 0)) return cudaSuccess;
   if (part != nullptr) lse_from_partials_kernel<<<M, 256, 0, stream>>>(part, n_tiles, M, lse);
   else lse_from_logits_kernel<<<M, 256, 0, stream>>>(C, ldc, N, lse);
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || N <= 0) return e;
   const long long work = static_cast<long long>(M) * N / 4;
   const long long want = (work + 255) / 256;
   const long long cap = 4LL * (sms > 0 ? sms : 1);

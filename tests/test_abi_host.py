@@ -187,6 +187,8 @@ def test_grouped_argument_errors():
     assert _grouped(good, ptr=FAKE + 2) == sg.ERR_ALIGNMENT
     assert _grouped(good, wsb=16) == sg.ERR_WORKSPACE
     assert _grouped(good, ws=None) == sg.ERR_WORKSPACE
+    assert _grouped(good, ws=FAKE + 4) == sg.ERR_ALIGNMENT       # split partials are float4
+    assert _grouped(good, ws=FAKE + 8) == sg.ERR_ALIGNMENT
     assert _grouped([(0, 256, 256), (256, 0, 64)]) == sg.ERR_CUDA  # valid: needs a device
     assert _grouped(good) == sg.ERR_CUDA
 

@@ -84,3 +84,28 @@ def test_reference_arm_json_line():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2")
     r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=root, env=env)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_gpus_n_without_enough_gpus_refuses():
+    """`bench.py --gpus 2` started without a launcher starts its own ranks, one per GPU;
+    with fewer GPUs visible than asked for it exits with status 2 and times nothing
+    (it never reports fewer GPUs than requested)."""
+    import subprocess
+    import sys
+    import torch
+    if torch.cuda.device_count() >= 2:
+        pytest.skip("two GPUs are visible: the launch would run")
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, bench.__file__, "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 2
+    assert "GPU(s) visible" in r.stderr and r.stdout.strip() == ""
+
+
+def test_world_size_must_match_gpus():
+    import subprocess
+    import sys
+    env = dict(os.environ, WORLD_SIZE="3", RANK="0")
+    r = subprocess.run([sys.executable, bench.__file__, "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 2 and "WORLD_SIZE=3" in r.stderr

@@ -139,3 +139,25 @@ def test_grouped_split_tail_few_tiles(cuda_device):
         ref, acc = oracle.gemm(a, b, a_dtype=ad, b_dtype=bd, out_dtype=oracle.F32, want_absacc=True)
         check_tolerance(o1[g].cpu().numpy(), ref, acc, torch.float32, what=f"group {g}")
         assert torch.equal(o1[g], o2[g])
+
+
+def test_grouped_misaligned_workspace_is_rejected_before_any_launch(cuda_device):
+    """A workspace that is not 16-byte aligned is refused with SMGEMM_ERR_ALIGNMENT before
+    anything is enqueued: neither the GEMM groups nor a K = 0 group (filled with act(bias)
+    on valid calls) touch their outputs."""
+    shapes = [(256, 256, 1024), (64, 128, 0)]
+    As = [torch.ones((M, K), dtype=torch.bfloat16, device="cuda") for M, N, K in shapes]
+    Bs = [torch.ones((K, N), dtype=torch.bfloat16, device="cuda") for M, N, K in shapes]
+    outs = [torch.full((M, N), 7.0, dtype=torch.float32, device="cuda") for M, N, K in shapes]
+    nbytes = int(sg.lib().smgemm_grouped_workspace_size(len(shapes)))
+    ws = torch.zeros(nbytes + 64, dtype=torch.uint8, device="cuda")[4:]
+    assert ws.data_ptr() % 16 == 4
+    with pytest.raises(sg.SmgemmError) as ei:
+        sg.gemm_bf16_grouped(As, Bs, outs=outs, workspace=ws)
+    assert ei.value.status == sg.ERR_ALIGNMENT
+    assert sg.check() == sg.OK
+    for o in outs:
+        assert bool((o == 7.0).all())
+    sg.gemm_bf16_grouped(As, Bs, outs=outs, workspace=torch.zeros(nbytes, dtype=torch.uint8, device="cuda"))
+    assert sg.check() == sg.OK
+    assert bool((outs[0] == 1024.0).all()) and bool((outs[1] == 0.0).all())

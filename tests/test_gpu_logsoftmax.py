@@ -82,3 +82,62 @@ def test_logsoftmax_k0_is_log_softmax_of_bias(cuda_device):
     assert sg.check() == sg.OK
     ref, _ = oracle.log_softmax_rows(np.tile(b.numpy().astype(np.float64), (M, 1)))
     assert np.allclose(out.cpu().numpy(), ref, rtol=0, atol=1e-5)
+
+
+# ------------------------------------------------------------------ vocabulary split (two-step API)
+
+@pytest.mark.parametrize("M,layout", [(5, "row"), (16, "row"), (64, "row"), (200, "row"), (16, "col")])
+@pytest.mark.parametrize("slices", [1, 3])
+def test_lse_partials_over_vocabulary_slices(cuda_device, M, layout, slices):
+    """The vocabulary-parallel steps on one GPU: the columns of W are split into slices
+    (tile-aligned, as the ranks of a vocabulary-parallel LM head hold them), each slice
+    runs gemm_bf16_lse_partials on its own, the partials of all slices are stacked in
+    slice order, and logsoftmax_apply_partials on each slice must give that slice of the
+    whole row's log-softmax (same bound as the fused call). Rows M <= 64 with row-major X
+    take the skinny kernel, whose epilogue forms the partials; the others the light pass
+    over the logits."""
+    from sm_gemm_b200 import vocab_parallel as vp
+    N, K = 1000, 264
+    X = to_dtype(synth.normal(54, M, (M, K)), torch.bfloat16)
+    W = to_dtype(synth.normal(54, 1, (K, N), 0.2), torch.bfloat16)
+    b = to_dtype(synth.normal(54, 2, (N,), 0.5), torch.float32)
+    Xd = X.cuda() if layout == "row" else X.t().contiguous().cuda().t()
+    outs, parts = [], []
+    for r in range(slices):
+        c0, c1 = vp.shard_columns(N, slices, r)
+        Ws = W[:, c0:c1].contiguous().cuda()
+        out = torch.empty((M, -(-(c1 - c0) // 4) * 4), dtype=torch.float32, device="cuda")[:, :c1 - c0]
+        o, p = sg.gemm_bf16_lse_partials(Xd, Ws, bias=b[c0:c1].contiguous().cuda(), out=out)
+        assert sg.check() == sg.OK
+        outs.append((c0, c1, o))
+        parts.append(p)
+    every = torch.cat(parts, dim=0)
+    full = torch.empty((M, N), dtype=torch.float32)
+    lses = []
+    for c0, c1, o in outs:
+        lses.append(sg.logsoftmax_apply_partials(o, every).cpu())
+        assert sg.check() == sg.OK
+        full[:, c0:c1] = o.cpu()
+    for l in lses[1:]:
+        assert torch.equal(l, lses[0])
+    _check(full, X, W, b)
+
+
+def test_apply_partials_neutral_pairs_and_empty_slice(cuda_device):
+    """Pairs (-inf, 0) (the padding of a short slice) change nothing, and a slice with no
+    columns still receives the row's lse."""
+    M, N, K = 4, 320, 128   # 2.5 tiles; W's row pitch (640 bytes) meets the 16-byte rule
+    X = to_dtype(synth.normal(55, 0, (M, K)), torch.bfloat16).cuda()
+    W = to_dtype(synth.normal(55, 1, (K, N), 0.2), torch.bfloat16).cuda()
+    o, p = sg.gemm_bf16_lse_partials(X, W)
+    pad = torch.zeros((2, M, 2), dtype=torch.float32, device="cuda")
+    pad[:, :, 0] = float("-inf")
+    ref = o.clone()
+    lse_ref = sg.logsoftmax_apply_partials(ref, p)
+    lse_pad = sg.logsoftmax_apply_partials(o, torch.cat([pad[:1], p, pad[1:]], dim=0))
+    empty = torch.empty((M, 0), dtype=torch.float32, device="cuda")
+    lse_empty = sg.logsoftmax_apply_partials(empty, p)
+    assert sg.check() == sg.OK
+    # neutral pairs change nothing but the pairing order of the merge tree (last-bit rounding)
+    assert torch.allclose(lse_pad, lse_ref, rtol=0, atol=1e-5) and torch.allclose(o, ref, rtol=0, atol=1e-5)
+    assert torch.equal(lse_empty, lse_ref)
