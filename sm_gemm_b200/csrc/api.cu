@@ -16,6 +16,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/smgemm.h"
 #include "grouped.h"
 #include "kernels.h"
@@ -23,6 +25,15 @@
 using namespace smg;
 
 namespace {
+
+// One NVTX range per entry-point call, named after the entry point, so a profiler's
+// timeline shows which library call enqueued which kernels (the profiling practice of
+// "为什么我们要死磕GEMM" (kwkr.cn), section 7.1). Without an attached tool a range costs
+// one predictable branch (NVTX's header-only API).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 // ------------------------------------------------------------------ driver entry point
 
@@ -98,6 +109,17 @@ SchedMode sched_mode() {
   return SchedMode::kAuto;
 }
 
+// SMGEMM_FORCE_CONFIG picks the kernel family instead of the heuristics, for tuning and
+// tests: "pair" (256 x 256 tiles on CTA pairs), "single" (one-SM large tiles), "large"
+// (no swap-AB path for small M; pair or single as usual), "pair128" (FP8: 256 x 128
+// pair tiles). Unknown or empty values leave the heuristics in charge. The older
+// switches SMGEMM_PAIR=0, SMGEMM_FORCE_LARGE=1 and SMGEMM_FP8_TN=128 mean "single",
+// "large" and "pair128".
+bool force_config_is(const char* want) {
+  const char* v = std::getenv("SMGEMM_FORCE_CONFIG");
+  return v != nullptr && std::strcmp(v, want) == 0;
+}
+
 // Tile-grid plan over T output tiles and P persistent CTAs (or CTA pairs).
 //  - auto: whole waves of tiles run data-parallel; the R = T mod P tiles of a ragged
 //    last wave are split along K into s = min(P / R, KB / 8) equal pieces that run
@@ -124,11 +146,19 @@ Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, siz
   long long max_ctas = env_ll("SMGEMM_GRID", sms);
   if (max_ctas < 1) max_ctas = 1;
   if (max_ctas > sms) max_ctas = sms;
-  const SchedMode mode = sched_mode();
+  SchedMode mode = sched_mode();
   constexpr int kMinItersPerPiece = 8;
+  // SMGEMM_SPLITK=s: 1 = every tile whole (data-parallel only); s >= 2 = every tile's K
+  // range cut into about s pieces (one stream-K range over min(P, s T) CTAs).
+  const long long splitk = env_ll("SMGEMM_SPLITK", 0);
+  if (splitk == 1) mode = SchedMode::kDP;
 
   long long dp = T, sk_iters = 0, sk_ctas = 0, grid = std::min<long long>(T, max_ctas);
-  if (mode == SchedMode::kSK) {
+  if (splitk >= 2) {
+    dp = 0;
+    sk_iters = T * kb_total;
+    grid = sk_ctas = std::min<long long>(std::min<long long>(max_ctas, T * splitk), sk_iters);
+  } else if (mode == SchedMode::kSK) {
     dp = 0;
     sk_iters = T * kb_total;
     grid = sk_ctas = std::min<long long>(max_ctas, sk_iters);
@@ -259,9 +289,11 @@ struct Gemm16Plan {
 Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms, int pair_clusters,
                        bool allow_skinny = true) {
   Gemm16Plan g;
-  const bool force_large = env_ll("SMGEMM_FORCE_LARGE", 0) != 0 || !allow_skinny;
+  const bool force_single = force_config_is("single") || env_ll("SMGEMM_PAIR", 1) == 0;
+  const bool force_large = env_ll("SMGEMM_FORCE_LARGE", 0) != 0 || !allow_skinny || force_config_is("large") ||
+                           force_config_is("pair") || force_single;
   g.skinny = (M <= 64 && layout_a == SMGEMM_ROW_MAJOR && !force_large);
-  g.pair = !g.skinny && pair_clusters > 0 && env_ll("SMGEMM_PAIR", 1) != 0;
+  g.pair = !g.skinny && pair_clusters > 0 && !force_single;
   if (g.skinny) g.v = M <= 16 ? Tc16Variant::kSkinny16 : (M <= 32 ? Tc16Variant::kSkinny32 : Tc16Variant::kSkinny64);
   else g.v = Tc16Variant::kLarge;
   g.mma_n = tc16_mma_n(g.v);
@@ -292,13 +324,13 @@ struct Fp8Plan {
   Plan pl;
 };
 
-int fp8_tile_n() { return env_ll("SMGEMM_FP8_TN", 256) == 128 ? 128 : 256; }
+int fp8_tile_n() { return (env_ll("SMGEMM_FP8_TN", 256) == 128 || force_config_is("pair128")) ? 128 : 256; }
 
 Fp8Plan plan_fp8(int64_t M, int64_t N, int64_t K, int sms, int tn, int pair_clusters) {
   Fp8Plan f;
   const int kb = static_cast<int>((K + kFp8BK - 1) / kFp8BK);
   const int group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", 8));
-  f.pair = pair_clusters > 0 && env_ll("SMGEMM_PAIR", 1) != 0;
+  f.pair = pair_clusters > 0 && env_ll("SMGEMM_PAIR", 1) != 0 && !force_config_is("single");
   f.tn = tn;
   if (f.pair) {
     f.pl = make_plan(static_cast<int>((M + 255) / 256), static_cast<int>((N + tn - 1) / tn), std::max(kb, 1),
@@ -464,6 +496,7 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_d
                         smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b, int64_t ldb,
                         const void* bias, smgemm_dtype bias_dtype, smgemm_act act, void* C, smgemm_dtype c_dtype,
                         int64_t ldc, void* workspace, size_t workspace_bytes, smgemm_stream_t stream) {
+  const NvtxRange nvtx_range("smgemm:gemm_bf16");
   return gemm16_impl(M, N, K, A, ab_dtype, layout_a, lda, B, layout_b, ldb, bias, bias_dtype, act, C, c_dtype, ldc,
                      workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr);
 }
@@ -472,6 +505,7 @@ smgemm_status gemm_bf16_fp8out(int64_t M, int64_t N, int64_t K, const void* A, s
                                smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b, int64_t ldb,
                                const void* bias, smgemm_dtype bias_dtype, smgemm_act act, uint8_t* Cq, int64_t ldc,
                                float* scales, void* workspace, size_t workspace_bytes, smgemm_stream_t stream) {
+  const NvtxRange nvtx_range("smgemm:gemm_bf16_fp8out");
   if (scales == nullptr) return SMGEMM_ERR_INVALID_ARG;
   return gemm16_impl(M, N, K, A, ab_dtype, layout_a, lda, B, layout_b, ldb, bias, bias_dtype, act, Cq, SMGEMM_E4M3,
                      ldc, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, scales);
@@ -487,6 +521,7 @@ smgemm_status gemm_bf16_logsoftmax(int64_t M, int64_t N, int64_t K, const void* 
                                    smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b,
                                    int64_t ldb, const void* bias, smgemm_dtype bias_dtype, float* C, int64_t ldc,
                                    void* workspace, size_t workspace_bytes, smgemm_stream_t stream_) {
+  const NvtxRange nvtx_range("smgemm:gemm_bf16_logsoftmax");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (M < 0 || N < 0 || K < 0) return SMGEMM_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return SMGEMM_OK;
@@ -512,6 +547,7 @@ smgemm_status gemm_bf16_lse_partials(int64_t M, int64_t N, int64_t K, const void
                                      smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b,
                                      int64_t ldb, const void* bias, smgemm_dtype bias_dtype, float* C, int64_t ldc,
                                      float* part, void* workspace, size_t workspace_bytes, smgemm_stream_t stream_) {
+  const NvtxRange nvtx_range("smgemm:gemm_bf16_lse_partials");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (M < 0 || N < 0 || K < 0) return SMGEMM_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return SMGEMM_OK;
@@ -529,6 +565,7 @@ smgemm_status gemm_bf16_lse_partials(int64_t M, int64_t N, int64_t K, const void
 
 smgemm_status logsoftmax_apply_partials(float* C, int64_t ldc, int64_t M, int64_t N, const float* part,
                                         int64_t n_parts, float* lse, smgemm_stream_t stream_) {
+  const NvtxRange nvtx_range("smgemm:logsoftmax_apply_partials");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (M < 0 || N < 0 || n_parts < 0 || !fits_int(M) || !fits_int(N) || !fits_int(n_parts))
     return SMGEMM_ERR_INVALID_ARG;
@@ -565,6 +602,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
                                 const void* const* bias, smgemm_dtype bias_dtype, smgemm_act act, void* const* C,
                                 smgemm_dtype c_dtype, const int64_t* ldc, void* workspace, size_t workspace_bytes,
                                 smgemm_stream_t stream_) {
+  const NvtxRange nvtx_range("smgemm:gemm_bf16_grouped");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (G < 0 || (G > 0 && (M == nullptr || N == nullptr || K == nullptr || A == nullptr || lda == nullptr ||
                           B == nullptr || ldb == nullptr || C == nullptr || ldc == nullptr)))
@@ -696,6 +734,7 @@ smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_
                                    const uint8_t* Bq, const float* sb, const void* bias, smgemm_dtype bias_dtype,
                                    smgemm_act act, void* C, smgemm_dtype c_dtype, int64_t ldc, void* workspace,
                                    size_t workspace_bytes, smgemm_stream_t stream_) {
+  const NvtxRange nvtx_range("smgemm:gemm_fp8_blockscaled");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!fits_int(M) || !fits_int(N) || !fits_int(K)) return SMGEMM_ERR_INVALID_ARG;
   if (!valid_out_dtype(c_dtype) || !valid_act(act)) return SMGEMM_ERR_INVALID_ARG;
@@ -743,6 +782,7 @@ smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_
 smgemm_status quantize_fp8_blockwise(const float* X, int64_t rows, int64_t cols, smgemm_layout layout_x,
                                      int64_t ldx, int group_rows, uint8_t* Q, float* scales,
                                      smgemm_stream_t stream_) {
+  const NvtxRange nvtx_range("smgemm:quantize_fp8_blockwise");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (rows < 0 || cols < 0 || !valid_layout(layout_x)) return SMGEMM_ERR_INVALID_ARG;
   if (group_rows != 1 && group_rows != 128) return SMGEMM_ERR_INVALID_ARG;

@@ -284,3 +284,28 @@ def test_schedule_small_grid_override(monkeypatch):
     monkeypatch.setenv("SMGEMM_SCHED", "dp")
     d = _check_schedule(300, 300, 3000)
     assert (d[:, 4] == 0).all()
+
+
+def test_splitk_override(monkeypatch):
+    """SMGEMM_SPLITK=1 keeps every tile whole; SMGEMM_SPLITK=s cuts each tile's K range
+    into about s pieces spread over min(P, s T) CTAs, still covering every K-block once."""
+    monkeypatch.setenv("SMGEMM_SPLITK", "1")
+    d = _check_schedule(1024, 1024, 4096)                 # 4 x 4 pair tiles: a ragged wave otherwise split
+    assert (d[:, 6] == -1).all()
+    monkeypatch.setenv("SMGEMM_SPLITK", "3")
+    d = _check_schedule(512, 512, 4096)                   # 2 x 2 pair tiles -> 12 CTAs
+    assert len(set(d[:, 0].tolist())) == 12 and (d[:, 6] >= 0).all()
+
+
+def test_force_config_override(monkeypatch):
+    """SMGEMM_FORCE_CONFIG=single runs M = 16 on one-SM 128 x 256 tiles instead of the
+    swap-AB skinny path; =pair puts it on CTA pairs (256 x 256)."""
+    M, N, K = 16, 4096, 1024
+    skinny = sg.schedule_dump(M, N, K)
+    assert len(set(skinny[:, 1].tolist())) == N // 128      # swap-AB: 128 weight columns per tile
+    monkeypatch.setenv("SMGEMM_FORCE_CONFIG", "single")
+    single = _check_schedule(M, N, K, bk=64)
+    assert len(set(single[:, 1].tolist())) == N // 256
+    monkeypatch.setenv("SMGEMM_FORCE_CONFIG", "pair")
+    pair = _check_schedule(M, N, K, bk=64, sms=74)
+    assert len(set(pair[:, 1].tolist())) == N // 256
