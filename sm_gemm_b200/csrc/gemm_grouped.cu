@@ -15,7 +15,8 @@
 //
 // Roles as in gemm_tc16_pair.cu: warp 0 TMA producer and warp 1 MMA issuer (warp-wide
 // loops, one elected lane issues; MMA on the rank-0 CTA only), warp 2 TMEM allocator,
-// warps 4-7 epilogue (each CTA drains its own 128 rows of the two TMEM accumulators).
+// warps 4-11 epilogue (each CTA drains its own 128 rows of the two TMEM accumulators;
+// warp w takes lanes 32*(w%4).. and the 128 columns 128*((w-4)/4).. of the tile).
 // When the tiles leave a ragged last wave (R = T mod P tiles for P clusters), those R
 // tiles are split along K into S pieces (R S <= P) that run side by side; each piece's
 // partial goes to a workspace slot and the last piece to finish sums them in order.
@@ -31,8 +32,11 @@
 namespace smg {
 
 namespace {
-constexpr int kThreads = 256;
 constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 32 * kEpiWarp0 + kEpiThreads;
+constexpr int kEpiCols = 128;  // tile columns per epilogue warp
 constexpr int kTileN = 256;
 constexpr int kTcols = 512;
 
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 8);
+      mbar_init(tempty_bar(b), 2 * kEpiWarps);  // every epilogue warp of both CTAs
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -247,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
     const int r_local = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     const int epi_tid = threadIdx.x - kEpiWarp0 * 32;
+    const int c_base = ((warp - kEpiWarp0) >> 2) * kEpiCols;  // this warp's first tile column
     int local = 0;
     bool dead = false;
     GIter wi;
@@ -260,21 +265,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
       if (!dead) dead = !mbar_wait(tfull_bar(acc), acc_phase, abort_flag, limit);
       dead = __any_sync(0xffffffffu, dead);
       const int row = it.mt * 256 + static_cast<int>(rank) * 128 + r_local;
-      const uint32_t tacc = tmem_base + lane_addr + acc * kTileN;
+      const uint32_t tacc = tmem_base + lane_addr + acc * kTileN + c_base;
+      const int col0 = it.nt * kTileN + c_base;
       const bool split = it.unit >= 0;
       float* my_slot = split ? sp.slots + (static_cast<size_t>(it.unit) * 2 + rank) * SLOT : nullptr;
       if (!dead) {
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < kTileN / 32; ++c) {
+        for (int c = 0; c < kEpiCols / 32; ++c) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tacc + c * 32, r);
           tmem_ld_wait();
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          if (split) slot_store<32>(my_slot, r_local, c * 32, v);
-          else epi_row32(e, row, it.nt * kTileN + c * 32, v);
+          if (split) slot_store<32>(my_slot, r_local, c_base + c * 32, v);
+          else epi_row32(e, row, col0 + c * 32, v);
         }
         tc_fence_before();
         __syncwarp();
@@ -285,29 +291,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
         // and runs the epilogue: deterministic, and no CTA waits for another.
         const long long r_tail = it.tile - (p.total_tiles - sp.split_tiles);
         __threadfence();
-        named_barrier_sync(1, 128);
+        named_barrier_sync(1, kEpiThreads);
         if (epi_tid == 0) {
           const bool any_dead = *abort_flag != 0;
           const int old = any_dead ? -1 : atomicAdd(sp.counters + r_tail * 2 + rank, 1);
           *reduce_flag = (!any_dead && old == sp.splits - 1);
         }
-        named_barrier_sync(1, 128);
+        named_barrier_sync(1, kEpiThreads);
         if (*reduce_flag) {
           __threadfence();
 #pragma unroll 1
-          for (int c = 0; c < kTileN / 32; ++c) {
+          for (int c = 0; c < kEpiCols / 32; ++c) {
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.0f;
 #pragma unroll 1
             for (int pc = 0; pc < sp.splits; ++pc) {
               const float* src = sp.slots + ((r_tail * sp.splits + pc) * 2 + rank) * static_cast<size_t>(SLOT);
-              slot_accumulate<32>(src, r_local, c * 32, v);
+              slot_accumulate<32>(src, r_local, c_base + c * 32, v);
             }
-            epi_row32(e, row, it.nt * kTileN + c * 32, v);
+            epi_row32(e, row, col0 + c * 32, v);
           }
         }
-        named_barrier_sync(1, 128);
+        named_barrier_sync(1, kEpiThreads);
       }
       ++local;
     }
