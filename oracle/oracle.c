@@ -22,10 +22,14 @@
  *    sum_{k in kb} dec(qa[i,k])*dec(qb[j,k]) + bias[j])), in double, from the same
  *    quantised operands; walkthrough section 2.4 (accumulate high, rescale).
  *
- * Readings where the pages are silent (each one is listed in the design notes):
- * an all-zero group gets scale 1.0; amax covers only the elements present in a
- * partial group; x/scale is an IEEE float division (not a reciprocal multiply);
- * rounding to zero keeps the sign (code 0x80 for negative inputs).
+ * Readings where the pages are silent: an all-zero group gets scale 1.0 (it avoids
+ * 0/0, gives all-zero codes and dequantises to exactly 0); amax covers only the
+ * elements present in a partial group, and the missing elements take no part in the
+ * GEMM; x/scale is an IEEE float division (not a reciprocal multiply), and the scale
+ * amax/448 is an FP32 division, not rounded to a power of two; rounding to zero keeps
+ * the sign (code 0x80 for negative inputs); GeLU is the tanh form with sqrt(2/pi) and
+ * 0.044715 (Hendrycks & Gimpel), SiLU is x*sigmoid(x); the bias is added to the
+ * exact sum and the activation applied before the single rounding to the output type.
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -shared -fPIC (no fast-math: every
  * float operation here is IEEE with round-to-nearest-even).
