@@ -480,8 +480,23 @@ smgemm_status gemm16_impl(int64_t M, int64_t N, int64_t K, const void* A, smgemm
   st = prepare_workspace(g.pl, workspace, workspace_bytes, stream, &p.slots, &p.counters);
   if (st != SMGEMM_OK) return st;
   if (g.pair) {
-    note_config("pair", g.pl, 256);
-    return launch_status(launch_gemm_tc16_pair(tm_a, tm_b, p, g.pl.grid, stream));
+    // C leaves through TMA tile stores (32 x 32 boxes staged in shared memory), measured
+    // slightly faster than 16-byte stores from registers (square BF16 4096^3: 97.5 vs
+    // 98.7 us); SMGEMM_EPI_STORE=direct selects the register stores.
+    CUtensorMap tm_c;
+    const CUtensorMap* pc = nullptr;
+    const char* es = std::getenv("SMGEMM_EPI_STORE");
+    if (!fp8_out && !(es != nullptr && std::strcmp(es, "direct") == 0)) {
+      const CUtensorMapDataType cdt = c_dtype == SMGEMM_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                      : c_dtype == SMGEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                               : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+      if (!encode_2d(&tm_c, cdt, C, N, M, ldc * elem_size(c_dtype), 32, 32,
+                     c_dtype == SMGEMM_F32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+        return SMGEMM_ERR_CUDA;
+      pc = &tm_c;
+    }
+    note_config(pc != nullptr ? "pair-tmastore" : "pair", g.pl, 256);
+    return launch_status(launch_gemm_tc16_pair(tm_a, tm_b, pc, p, g.pl.grid, stream));
   }
   note_config(g.skinny ? "skinny" : "large", g.pl, g.mma_n);
   return launch_status(launch_gemm_tc16(tm_a, tm_b, p, g.v, g.pl.grid, stream));
@@ -637,11 +652,17 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   const bool a_mn = (layout_a == SMGEMM_COL_MAJOR);
   const bool b_mn = (layout_b == SMGEMM_ROW_MAJOR);
   const int bk = grouped_bk();
-  std::vector<GroupDesc> table(static_cast<size_t>(G));
+  // Up to kInlineGroups records are passed with the launch (no copy); more go to the
+  // workspace through one host-to-device copy.
+  const bool inline_table = G <= kInlineGroups;
+  GroupTableInline inl;
+  std::vector<GroupDesc> heap;
+  if (!inline_table) heap.resize(static_cast<size_t>(G));
+  GroupDesc* table = inline_table ? inl.d : heap.data();
   std::vector<int> fills;  // groups with K = 0: filled with act(bias) after the table is enqueued
   long long tiles = 0;
   for (int g = 0; g < G; ++g) {
-    GroupDesc& e = table[static_cast<size_t>(g)];
+    GroupDesc& e = table[g];
     std::memset(&e, 0, sizeof(e));
     e.tile0 = tiles;
     e.M = static_cast<int>(M[g]);
@@ -670,11 +691,12 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   GroupDesc* dev_table = reinterpret_cast<GroupDesc*>((reinterpret_cast<uintptr_t>(workspace) + 63) & ~uintptr_t(63));
   // Pageable source: the copy has consumed `table` by the time the call returns. It is
   // the first thing enqueued, so a failure here leaves every output untouched.
-  if (tiles > 0 && cudaMemcpyAsync(dev_table, table.data(), table.size() * sizeof(GroupDesc),
-                                   cudaMemcpyHostToDevice, stream) != cudaSuccess)
+  if (!inline_table && tiles > 0 &&
+      cudaMemcpyAsync(dev_table, table, static_cast<size_t>(G) * sizeof(GroupDesc), cudaMemcpyHostToDevice,
+                      stream) != cudaSuccess)
     return launch_status(cudaGetLastError());
   for (int g : fills) {
-    const GroupDesc& e = table[static_cast<size_t>(g)];
+    const GroupDesc& e = table[g];
     smgemm_status st =
         launch_status(launch_fill_epilogue(e.M, e.N, e.bias, bias_dtype, act, C[g], c_dtype, ldc[g], stream));
     if (st != SMGEMM_OK) return st;
@@ -727,7 +749,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
                 "path=grouped groups=%d tiles=%lld grid=%d tile=128x256 split_tiles=%lld splits=%d", G, tiles, clusters,
                 S >= 2 ? R : 0LL, S >= 2 ? S : 0);
   if (env_ll("SMGEMM_LOG", 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
-  return launch_status(launch_gemm_grouped_split(p, sp, clusters, stream));
+  return launch_status(launch_gemm_grouped_split(p, sp, inline_table ? &inl : nullptr, clusters, stream));
 }
 
 smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_t* Aq, const float* sa,

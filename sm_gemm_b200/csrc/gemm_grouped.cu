@@ -7,11 +7,13 @@
 // group by group (grouped raster inside a group); cluster c takes tiles c, c + P, c + 2P,
 // ... over the whole list, so consecutive tiles of one group run side by side.
 //
-// Per-group data lives in a device table (GroupDesc: both TMA descriptors, sizes, output
-// and bias pointers) that the host writes into the caller's workspace before the launch.
-// Every role finds a tile's group by binary search over the groups' first-tile indices.
-// The producer issues fence.proxy.tensormap acquire on a group's descriptors before its
-// first copy from them, since the table may have been rewritten since an earlier launch.
+// Per-group data (GroupDesc: both TMA descriptors, sizes, output and bias pointers) comes
+// with the launch as a kernel parameter for up to kInlineGroups groups, else from a device
+// table that the host writes into the caller's workspace before the launch. Every role
+// finds a tile's group by binary search over the groups' first-tile indices. With the
+// device table the producer issues fence.proxy.tensormap acquire on a group's
+// descriptors before its first copy from them, since the table may have been rewritten
+// since an earlier launch.
 //
 // Roles as in gemm_tc16_pair.cu: warp 0 TMA producer and warp 1 MMA issuer (warp-wide
 // loops, one elected lane issues; MMA on the rank-0 CTA only), warp 2 TMEM allocator,
@@ -21,6 +23,7 @@
 // tiles are split along K into S pieces (R S <= P) that run side by side; each piece's
 // partial goes to a workspace slot and the last piece to finish sums them in order.
 #include <cuda_bf16.h>
+#include <type_traits>
 #include <cuda_fp16.h>
 
 #include "epilogue.cuh"
@@ -110,9 +113,14 @@ struct GIter {
   }
 };
 
-template <int BK, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_constant__ GroupedParams p,
-                                                                   const __grid_constant__ GroupedSplit sp) {
+struct NoInlineTable {};
+
+template <int BK, int STAGES, bool INLINE>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_grouped_kernel(const __grid_constant__ GroupedParams p_in, const __grid_constant__ GroupedSplit sp,
+                        const __grid_constant__ std::conditional_t<INLINE, GroupTableInline, NoInlineTable> inl) {
+  GroupedParams p = p_in;
+  if constexpr (INLINE) p.groups = inl.d;
   constexpr int A_BYTES = 128 * BK * 2;
   constexpr int B_BYTES = 128 * BK * 2;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -174,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const __grid_
     GItem it;
     while (ok && wi.next(p, sp, it)) {
       const GroupDesc* d = p.groups + it.g;
-      if (it.g != last_g && elect_one()) {
+      if (!INLINE && it.g != last_g && elect_one()) {
         tensormap_acquire(&d->tm_a);
         tensormap_acquire(&d->tm_b);
       }
@@ -332,8 +340,13 @@ constexpr int kSmem = 1024 + kStages * (2 * 128 * kBK * 2) + 8 * (2 * kStages + 
 static_assert(kSmem <= 232448, "shared memory budget");
 
 cudaError_t prepare() {
-  static cudaError_t st = cudaFuncSetAttribute(gemm_grouped_kernel<kBK, kStages>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  static cudaError_t st = [] {
+    cudaError_t e = cudaFuncSetAttribute(gemm_grouped_kernel<kBK, kStages, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(gemm_grouped_kernel<kBK, kStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kSmem);
+  }();
   return st;
 }
 
@@ -360,7 +373,7 @@ int grouped_max_clusters() {
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = config(1, nullptr, attr);
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_grouped_kernel<kBK, kStages>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_grouped_kernel<kBK, kStages, false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
@@ -370,19 +383,20 @@ int grouped_max_clusters() {
 
 int grouped_bk() { return kBK; }
 
-cudaError_t launch_gemm_grouped_split(const GroupedParams& p, const GroupedSplit& sp, int clusters,
-                                      cudaStream_t stream) {
+cudaError_t launch_gemm_grouped_split(const GroupedParams& p, const GroupedSplit& sp, const GroupTableInline* inl,
+                                      int clusters, cudaStream_t stream) {
   cudaError_t e = prepare();
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = config(clusters, stream, attr);
-  e = cudaLaunchKernelEx(&cfg, gemm_grouped_kernel<kBK, kStages>, p, sp);
+  if (inl != nullptr) e = cudaLaunchKernelEx(&cfg, gemm_grouped_kernel<kBK, kStages, true>, p, sp, *inl);
+  else e = cudaLaunchKernelEx(&cfg, gemm_grouped_kernel<kBK, kStages, false>, p, sp, NoInlineTable{});
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_grouped(const GroupedParams& p, int clusters, cudaStream_t stream) {
-  return launch_gemm_grouped_split(p, GroupedSplit{0, 0, nullptr, nullptr}, clusters, stream);
+  return launch_gemm_grouped_split(p, GroupedSplit{0, 0, nullptr, nullptr}, nullptr, clusters, stream);
 }
 
 unsigned take_error_word_grouped() { return take_error_word(); }

@@ -25,6 +25,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <cstring>
+
 #include "epilogue.cuh"
 #include "kernels.h"
 #include "operands.cuh"
@@ -42,27 +44,92 @@ constexpr int kTileN = 256;  // columns of the pair tile (128 per CTA for B, all
 constexpr int kTcols = 512;
 }  // namespace
 
-// FP8OUT: the epilogue emits E4M3 codes + 1x128 scales (c_dtype E4M3); a separate
-// instantiation, so the 16/32-bit-output kernel's code and registers are untouched.
-template <int BK, int STAGES, bool FP8OUT>
+// Output modes of the epilogue (separate instantiations, so each keeps its own code and
+// registers): kOutDirect - 16/32-bit C written from registers with 16-byte stores;
+// kOutFp8 - E4M3 codes + 1x128 scales (c_dtype E4M3); kOutTma - 16/32-bit C staged in
+// shared memory (one swizzled 32 x 32 box per epilogue warp and chunk) and written by a
+// TMA tile store through tm_c, the registers -> shared -> global write-back of the
+// Tensor-Core page ("Chunk处理完毕").
+constexpr int kOutDirect = 0, kOutFp8 = 1, kOutTma = 2;
+constexpr int kStageWarpBytes = 4096;  // TMA-store staging per epilogue warp (2 x bf16/f16 box or 1 x f32 box)
+
+// Bias, activation and cast of one 32 x 32 chunk (lane = row, v = its 32 columns), written
+// to this warp's staging buffer in the layout of a TMA box {32 columns, 32 rows} with the
+// map's swizzle (16-bit C: 64-byte rows, 64-byte swizzle; FP32 C: 128-byte rows, 128-byte
+// swizzle: the 16-byte chunk j of row r sits at j ^ ((r >> 1) & 3), resp. j ^ (r & 7),
+// so the 32 lanes' stores hit different banks), then one lane stores the box. 16-bit
+// chunks alternate between two 2 KB halves of the buffer, FP32 chunks use all 4 KB; a
+// half is rewritten only once the store that read it has finished reading.
+__device__ __forceinline__ void stage_and_store32(const EpiArgs& e, const CUtensorMap* tm_c, uint32_t buf, int c,
+                                                  uint32_t lane, int row0, int col0, float (&v)[32]) {
+  if (e.bias != nullptr || e.act != 0) epi_bias_act32(e, col0, v);
+  const bool f32 = e.c_dtype == 0;
+  const uint32_t dst = f32 ? buf : buf + (c & 1) * 2048;
+  if (lane == 0) {
+    if (f32) bulk_wait_group_read<0>();
+    else bulk_wait_group_read<1>();
+  }
+  __syncwarp();
+  const uint32_t r = lane;
+  if (f32) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t a = dst + r * 128 + 16 * (j ^ (r & 7));
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(v[4 * j]), "f"(v[4 * j + 1]),
+                   "f"(v[4 * j + 2]), "f"(v[4 * j + 3])
+                   : "memory");
+    }
+  } else {
+    const bool bf = e.c_dtype == 1;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t w[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float x0 = v[8 * j + 2 * h], x1 = v[8 * j + 2 * h + 1];
+        if (bf) {
+          __nv_bfloat162 t = __floats2bfloat162_rn(x0, x1);
+          w[h] = *reinterpret_cast<uint32_t*>(&t);
+        } else {
+          __half2 t = __floats2half2_rn(x0, x1);
+          w[h] = *reinterpret_cast<uint32_t*>(&t);
+        }
+      }
+      const uint32_t a = dst + r * 64 + 16 * (j ^ ((r >> 1) & 3));
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                   : "memory");
+    }
+  }
+  fence_proxy_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm_c, dst, col0, row0);
+    bulk_commit_group();
+  }
+}
+
+template <int BK, int STAGES, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc16_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                          const Tc16Params p) {
+                          const __grid_constant__ CUtensorMap tm_c, const Tc16Params p) {
+  constexpr bool FP8OUT = OUT == kOutFp8;
   constexpr int A_BYTES = 128 * BK * 2;
   constexpr int B_BYTES = 128 * BK * 2;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr int KSTEPS = BK / 16;
+  constexpr int STAGING = OUT == kOutTma ? kEpiWarps * kStageWarpBytes : 0;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
-  const uint32_t bar_base = smem_base + STAGES * STAGE_BYTES;
+  const uint32_t staging = smem_base + STAGES * STAGE_BYTES;  // 1024-byte aligned
+  const uint32_t bar_base = smem_base + STAGES * STAGE_BYTES + STAGING;
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
   auto tfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
   const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
-  uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5);
+  uint8_t* misc = smem_gen + STAGES * STAGE_BYTES + STAGING + 8 * (2 * STAGES + 5);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   volatile int* reduce_flag = reinterpret_cast<volatile int*>(misc + 8);
@@ -87,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    if (OUT == kOutTma) tma_prefetch_desc(&tm_c);
   }
   if (warp == 2) {
     tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTcols);
@@ -251,7 +319,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
             if (whole) {
-              epi_row32(p.e, row, col0 + c * 32, v);
+              if constexpr (OUT == kOutTma) {
+                stage_and_store32(p.e, &tm_c, staging + (warp - kEpiWarp0) * kStageWarpBytes, c, lane,
+                                  mt * 256 + static_cast<int>(rank) * 128 + q * 32, col0 + c * 32, v);
+              } else {
+                epi_row32(p.e, row, col0 + c * 32, v);
+              }
             } else {
               slot_store<32>(my_slot, r_local, c_base + c * 32, v);
             }
@@ -314,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++local;
     }
+    if (OUT == kOutTma && lane == 0) bulk_wait_group<0>();  // this warp's tile stores have landed
   }
 
   tc_fence_before();
@@ -325,16 +399,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 namespace {
 constexpr int kPairBK = 64, kPairStages = 6;
-constexpr int kPairSmem = 1024 + kPairStages * (2 * 128 * kPairBK * 2) + 8 * (2 * kPairStages + 5) + 16;
-static_assert(kPairSmem <= 232448, "shared memory budget");
+template <int OUT>
+constexpr int pair_smem() {
+  return 1024 + kPairStages * (2 * 128 * kPairBK * 2) + (OUT == kOutTma ? kEpiWarps * kStageWarpBytes : 0) +
+         8 * (2 * kPairStages + 5) + 16;
+}
+static_assert(pair_smem<kOutTma>() <= 232448, "shared memory budget");
 
-template <bool FP8OUT>
+template <int OUT>
 cudaError_t prepare_pair_kernel() {
-  static cudaError_t st = cudaFuncSetAttribute(gemm_tc16_pair_kernel<kPairBK, kPairStages, FP8OUT>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+  static cudaError_t st = cudaFuncSetAttribute(gemm_tc16_pair_kernel<kPairBK, kPairStages, OUT>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, pair_smem<OUT>());
   return st;
 }
 
+template <int OUT>
 cudaLaunchConfig_t pair_config(int clusters, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -343,7 +422,7 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t stream, cudaLaunchAttr
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kPairSmem;
+  cfg.dynamicSmemBytes = pair_smem<OUT>();
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -351,31 +430,49 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t stream, cudaLaunchAttr
 }
 }  // namespace
 
+namespace {
+template <int OUT>
+int max_clusters_of() {
+  if (prepare_pair_kernel<OUT>() != cudaSuccess) return 0;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pair_config<OUT>(1, nullptr, attr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc16_pair_kernel<kPairBK, kPairStages, OUT>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  return n;
+}
+}  // namespace
+
 int tc16_pair_max_clusters() {
   static int cached = -1;
   if (cached >= 0) return cached;
-  if (prepare_pair_kernel<false>() != cudaSuccess || prepare_pair_kernel<true>() != cudaSuccess) return 0;
-  cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_config(1, nullptr, attr);
-  int n = 0, n8 = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc16_pair_kernel<kPairBK, kPairStages, false>, &cfg) != cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&n8, gemm_tc16_pair_kernel<kPairBK, kPairStages, true>, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    n = n8 = 0;
-  }
-  cached = n < n8 ? n : n8;
+  const int a = max_clusters_of<kOutDirect>(), b = max_clusters_of<kOutFp8>(), c = max_clusters_of<kOutTma>();
+  cached = a < b ? (a < c ? a : c) : (b < c ? b : c);
   return cached;
 }
 
-cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Tc16Params& p,
-                                  int clusters, cudaStream_t stream) {
-  const bool fp8 = p.e.c_dtype == kE4M3;
-  cudaError_t e = fp8 ? prepare_pair_kernel<true>() : prepare_pair_kernel<false>();
+cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap* tm_c,
+                                  const Tc16Params& p, int clusters, cudaStream_t stream) {
+  const int out = p.e.c_dtype == kE4M3 ? kOutFp8 : (tm_c != nullptr ? kOutTma : kOutDirect);
+  cudaError_t e = out == kOutFp8 ? prepare_pair_kernel<kOutFp8>()
+                                 : (out == kOutTma ? prepare_pair_kernel<kOutTma>() : prepare_pair_kernel<kOutDirect>());
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pair_config(clusters, stream, attr);
-  e = fp8 ? cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages, true>, tm_a, tm_b, p)
-          : cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages, false>, tm_a, tm_b, p);
+  CUtensorMap none;
+  std::memset(&none, 0, sizeof(none));
+  const CUtensorMap& mc = tm_c != nullptr ? *tm_c : none;
+  if (out == kOutFp8) {
+    cudaLaunchConfig_t cfg = pair_config<kOutFp8>(clusters, stream, attr);
+    e = cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages, kOutFp8>, tm_a, tm_b, mc, p);
+  } else if (out == kOutTma) {
+    cudaLaunchConfig_t cfg = pair_config<kOutTma>(clusters, stream, attr);
+    e = cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages, kOutTma>, tm_a, tm_b, mc, p);
+  } else {
+    cudaLaunchConfig_t cfg = pair_config<kOutDirect>(clusters, stream, attr);
+    e = cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages, kOutDirect>, tm_a, tm_b, mc, p);
+  }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -14,7 +14,16 @@ struct GroupedSplit {
   int* counters;            // [R][2], zeroed before the launch
 };
 
-cudaError_t launch_gemm_grouped_split(const GroupedParams& p, const GroupedSplit& sp, int clusters,
-                                      cudaStream_t stream);
+// Up to kInlineGroups groups travel with the launch itself, as a kernel parameter (the
+// TMA descriptors then sit in parameter space, where a launch's tensor maps normally live),
+// so a call with few groups needs no host-to-device copy of its table.
+constexpr int kInlineGroups = 16;
+struct GroupTableInline {
+  GroupDesc d[kInlineGroups];
+};
+
+// `inl` (nullable): the table as a kernel parameter (G <= kInlineGroups); else p.groups.
+cudaError_t launch_gemm_grouped_split(const GroupedParams& p, const GroupedSplit& sp, const GroupTableInline* inl,
+                                      int clusters, cudaStream_t stream);
 
 }  // namespace smg

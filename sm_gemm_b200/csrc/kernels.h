@@ -43,8 +43,10 @@ int tc16_bk(Tc16Variant v);
 
 // CTA-pair large-tile kernel (256 x 256 per cluster of 2). p.s counts clusters;
 // p.slots is [clusters][2][2 ranks][256][128] floats, p.counters [stream-K tiles][2].
-cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Tc16Params& p,
-                                  int clusters, cudaStream_t stream);
+// tm_c (nullable): a tensor map of C (box 32 x 32, 64-byte swizzle for 16-bit C, 128-byte
+// for FP32) selects the epilogue that writes C with TMA tile stores.
+cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap* tm_c,
+                                  const Tc16Params& p, int clusters, cudaStream_t stream);
 int tc16_pair_max_clusters();   // co-resident clusters of 2 on the current device (0 if unknown)
 int tc16_pair_bk();
 

@@ -327,3 +327,40 @@ def test_deterministic_run_to_run(cuda_device):
     c2 = sg.gemm_bf16(A, B, out_dtype=torch.float32)
     assert sg.check() == sg.OK
     assert torch.equal(c1, c2)
+
+
+# ------------------------------------------------------------------ TMA-store epilogue
+
+@pytest.mark.parametrize("out_dt", [torch.bfloat16, torch.float16, torch.float32])
+@pytest.mark.parametrize("M,N,K,act", [(300, 520, 136, "gelu_tanh"), (1024, 1024, 512, "none"), (257, 200, 64, "silu"),
+                                       (4096, 4096, 256, "none")])
+def test_tma_store_epilogue_matches_direct_stores(cuda_device, monkeypatch, out_dt, M, N, K, act):
+    """The pair kernel writes C through shared memory and TMA tile stores (boxes clipped
+    at the matrix edge); SMGEMM_EPI_STORE=direct selects 16-byte stores from registers.
+    The values are computed the same way in both, so the outputs must agree bit for bit,
+    and with the oracle within the contract. Rows and columns past M and N
+    (sentinel-filled padding) stay untouched."""
+    A = to_dtype(synth.normal(97, M, (M, K)), torch.bfloat16)
+    B = to_dtype(synth.normal(97, N, (K, N), 0.2), torch.bfloat16)
+    bias = to_dtype(synth.normal(97, 1, (N,), 0.5), torch.bfloat16)
+    Ad, Bd, bd = A.cuda(), B.t().contiguous().cuda().t(), bias.cuda()
+    outs = {}
+    for mode in ("direct", "tma"):
+        if mode == "direct":
+            monkeypatch.setenv("SMGEMM_EPI_STORE", "direct")
+        else:
+            monkeypatch.delenv("SMGEMM_EPI_STORE", raising=False)
+        full, view = sentinel_out(M, N, out_dt)
+        sg.gemm_bf16(Ad, Bd, bias=bd, act=act, out=view)
+        assert sg.check() == sg.OK
+        assert ("tmastore" in sg.last_config()) == (mode == "tma")
+        assert_sentinel_intact(full, M, N)
+        outs[mode] = view.clone()
+    assert torch.equal(outs["direct"], outs["tma"])
+    if M * N <= 600_000:
+        a, ad = orc_view(A)
+        b, bdt = orc_view(B)
+        bb, bbd = orc_view(bias)
+        ref, acc = oracle.gemm(a, b, a_dtype=ad, b_dtype=bdt, bias=bb, bias_dtype=bbd, act=ORC_ACT[act],
+                               out_dtype=TORCH_TO_ORC[out_dt], want_absacc=True)
+        check_tolerance(outs["tma"].float().cpu().numpy(), ref, acc, out_dt, what=f"tma store {M}x{N}x{K}")
