@@ -139,8 +139,27 @@ struct Plan {
   size_t ws_bytes() const { return counter_bytes + slot_bytes; }
 };
 
+// Schedule choices measured per shape by an offline sweep (sm_gemm_b200/tune.py, the
+// tuning-to-a-static-table practice of the DeepGEMM kernel-library walkthrough (zwxr.cn),
+// section 5.2). A listed shape takes its group_m and split-K choice from the table;
+// SMGEMM_GROUP_M and SMGEMM_SPLITK still override both.
+struct TunedConfig {
+  int kind;
+  long long M, N, K;
+  int layout_a, group_m, splitk;
+};
+constexpr TunedConfig kTuned[] = {
+#include "tuned_configs.inc"
+    {-1, 0, 0, 0, 0, 0, 0}};
+
+const TunedConfig* find_tuned(int kind, int64_t M, int64_t N, int64_t K, int layout_a) {
+  for (const TunedConfig& t : kTuned)
+    if (t.kind == kind && t.M == M && t.N == N && t.K == K && t.layout_a == layout_a) return &t;
+  return nullptr;
+}
+
 Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, size_t slot_floats,
-               int counters_per_tile = 1) {
+               int counters_per_tile = 1, long long splitk_default = 0) {
   Plan pl;
   const long long T = static_cast<long long>(m_tiles) * n_tiles;
   long long max_ctas = env_ll("SMGEMM_GRID", sms);
@@ -150,7 +169,7 @@ Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, siz
   constexpr int kMinItersPerPiece = 8;
   // SMGEMM_SPLITK=s: 1 = every tile whole (data-parallel only); s >= 2 = every tile's K
   // range cut into about s pieces (one stream-K range over min(P, s T) CTAs).
-  const long long splitk = env_ll("SMGEMM_SPLITK", 0);
+  const long long splitk = env_ll("SMGEMM_SPLITK", splitk_default);
   if (splitk == 1) mode = SchedMode::kDP;
 
   long long dp = T, sk_iters = 0, sk_ctas = 0, grid = std::min<long long>(T, max_ctas);
@@ -299,10 +318,11 @@ Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms, i
   g.mma_n = tc16_mma_n(g.v);
   g.bk = g.pair ? tc16_pair_bk() : tc16_bk(g.v);
   const int kb = static_cast<int>((K + g.bk - 1) / g.bk);
-  const int group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", 8));
+  const TunedConfig* t = g.pair ? find_tuned(0, M, N, K, layout_a) : nullptr;
+  const int group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", t != nullptr ? t->group_m : 8));
   if (g.pair) {
     g.pl = make_plan(static_cast<int>((M + 255) / 256), static_cast<int>((N + 255) / 256), std::max(kb, 1),
-                     pair_clusters, group_m, static_cast<size_t>(2) * 128 * 256, 2);
+                     pair_clusters, group_m, static_cast<size_t>(2) * 128 * 256, 2, t != nullptr ? t->splitk : 0);
     return g;
   }
   int m_tiles, n_tiles;
@@ -329,12 +349,13 @@ int fp8_tile_n() { return (env_ll("SMGEMM_FP8_TN", 256) == 128 || force_config_i
 Fp8Plan plan_fp8(int64_t M, int64_t N, int64_t K, int sms, int tn, int pair_clusters) {
   Fp8Plan f;
   const int kb = static_cast<int>((K + kFp8BK - 1) / kFp8BK);
-  const int group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", 8));
   f.pair = pair_clusters > 0 && env_ll("SMGEMM_PAIR", 1) != 0 && !force_config_is("single");
   f.tn = tn;
+  const TunedConfig* t = f.pair && tn == 256 ? find_tuned(1, M, N, K, SMGEMM_ROW_MAJOR) : nullptr;
+  const int group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", t != nullptr ? t->group_m : 8));
   if (f.pair) {
     f.pl = make_plan(static_cast<int>((M + 255) / 256), static_cast<int>((N + tn - 1) / tn), std::max(kb, 1),
-                     pair_clusters, group_m, static_cast<size_t>(2) * 128 * tn, 2);
+                     pair_clusters, group_m, static_cast<size_t>(2) * 128 * tn, 2, t != nullptr ? t->splitk : 0);
   } else {
     f.pl = make_plan(static_cast<int>((M + kFp8BM - 1) / kFp8BM), static_cast<int>((N + kFp8BN - 1) / kFp8BN),
                      std::max(kb, 1), sms, group_m, static_cast<size_t>(kFp8BM) * kFp8BN);
@@ -482,11 +503,13 @@ smgemm_status gemm16_impl(int64_t M, int64_t N, int64_t K, const void* A, smgemm
   if (g.pair) {
     // C leaves through TMA tile stores (32 x 32 boxes staged in shared memory), measured
     // slightly faster than 16-byte stores from registers (square BF16 4096^3: 97.5 vs
-    // 98.7 us); SMGEMM_EPI_STORE=direct selects the register stores.
+    // 98.7 us); SMGEMM_EPI_STORE=direct selects the register stores. Only when a row of
+    // C is a whole number of 16-byte units: a box that ends past N in a partial unit was
+    // seen to write the rest of that unit (the columns just right of C) on B200.
     CUtensorMap tm_c;
     const CUtensorMap* pc = nullptr;
     const char* es = std::getenv("SMGEMM_EPI_STORE");
-    if (!fp8_out && !(es != nullptr && std::strcmp(es, "direct") == 0)) {
+    if (!fp8_out && (N * elem_size(c_dtype)) % 16 == 0 && !(es != nullptr && std::strcmp(es, "direct") == 0)) {
       const CUtensorMapDataType cdt = c_dtype == SMGEMM_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                       : c_dtype == SMGEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                                : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
