@@ -203,16 +203,18 @@ def _layout(t, name):
     raise ValueError(f"{name} must have a unit stride in one dimension")
 
 
-def _layout_as(t, name, want):
-    """(layout, leading dimension) of a 2-D tensor read in layout `want` (grouped calls
-    share one layout): a single row or column fits either layout, and its unused
-    leading dimension is rounded up to 8 elements (16 bytes)."""
+def _layout_as(t, name, want, g=None):
+    """Leading dimension of a 2-D tensor read in layout `want` (grouped calls share one
+    layout): a single row or column fits either layout, and its unused leading
+    dimension is rounded up to 8 elements (16 bytes). `g` (a group index) is only used
+    in the error message."""
     rows, cols = t.shape
-    if want == ROW_MAJOR and (t.stride(1) == 1 or cols <= 1):
-        return ROW_MAJOR, (max(t.stride(0), cols) if rows > 1 else -(-max(cols, 1) // 8) * 8)
-    if want == COL_MAJOR and (t.stride(0) == 1 or rows <= 1):
-        return COL_MAJOR, (max(t.stride(1), rows) if cols > 1 else -(-max(rows, 1) // 8) * 8)
-    raise ValueError(f"{name} cannot be read in the layout the other groups use")
+    s0, s1 = t.stride()
+    if want == ROW_MAJOR and (s1 == 1 or cols <= 1):
+        return max(s0, cols) if rows > 1 else -(-max(cols, 1) // 8) * 8
+    if want == COL_MAJOR and (s0 == 1 or rows <= 1):
+        return max(s1, rows) if cols > 1 else -(-max(rows, 1) // 8) * 8
+    raise ValueError(f"{name}{'' if g is None else f'[{g}]'} cannot be read in the layout the other groups use")
 
 
 _current_stream = None
@@ -450,41 +452,100 @@ def gemm_bf16_grouped(As, Bs, *, biases=None, act="none", outs=None, out_dtype=N
         with _torch().cuda.device(dev):
             return gemm_bf16_grouped(As, Bs, biases=biases, act=act, outs=outs, out_dtype=out_dtype,
                                      workspace=workspace, stream=stream)
+    args, res = _grouped_marshal(As, Bs, biases, act, outs, out_dtype, workspace, _stream(stream))
+    _check(lib().gemm_bf16_grouped(*args), "gemm_bf16_grouped")
+    return res
+
+
+def _grouped_marshal(As, Bs, biases, act, outs, out_dtype, workspace, sh):
+    """Checks every group and builds gemm_bf16_grouped's arguments (stream handle `sh`
+    last); allocates missing outputs and the workspace. Returns (args, outputs). It reads
+    each tensor's shape, strides and pointer once: with many small groups (MoE experts at
+    decode sizes) this marshalling is most of a call's host time."""
+    G = len(As)
     torch = _torch()
-    Ms, Ns, Ks, ldas, ldbs, ldcs = [], [], [], [], [], []
+    adt = As[0].dtype
     # The shared layouts: those of the first group whose operand is not a single row or column.
     lay_a = next((_layout(A, "A")[0] for A in As if min(A.shape) > 1), ROW_MAJOR)
     lay_b = next((_layout(B, "B")[0] for B in Bs if min(B.shape) > 1), ROW_MAJOR)
-    res = []
-    for g, (A, B) in enumerate(zip(As, Bs)):
+    Ms, Ns, Ks, ldas, ldbs, ldcs = [0] * G, [0] * G, [0] * G, [0] * G, [0] * G, [0] * G
+    pA, pB, pC = [0] * G, [0] * G, [0] * G
+    res = outs if outs is not None else [None] * G
+    cdt = None
+    for g in range(G):
+        A, B = As[g], Bs[g]
         M, K = A.shape
         K2, N = B.shape
-        if K != K2 or A.dtype != B.dtype or A.dtype != As[0].dtype:
+        if K != K2 or A.dtype is not adt or B.dtype is not adt:
             raise ValueError(f"group {g}: A and B must agree in K and dtype")
-        _, lda = _layout_as(A, f"A[{g}]", lay_a)
-        _, ldb = _layout_as(B, f"B[{g}]", lay_b)
+        ldas[g] = _layout_as(A, "A", lay_a, g)
+        ldbs[g] = _layout_as(B, "B", lay_b, g)
         if biases is not None and biases[g] is not None:
             _vector(biases[g], N, f"biases[{g}]")
-        out = outs[g] if outs is not None else torch.empty((M, N), dtype=out_dtype or A.dtype, device=A.device)
-        _out_matrix(out, M, N, f"outs[{g}]")
-        _need(out.dtype == (outs[0].dtype if outs is not None else out.dtype), "outputs must share one dtype")
-        res.append(out)
-        Ms.append(M); Ns.append(N); Ks.append(K); ldas.append(lda); ldbs.append(ldb)
-        ldcs.append(_ldc(out, M, N))
-    arr = lambda xs: (C.c_int64 * G)(*xs)
-    ptrs = lambda ts: (C.c_void_p * G)(*[None if t is None else t.data_ptr() for t in ts])
+        out = res[g]
+        if out is None:
+            out = torch.empty((M, N), dtype=out_dtype or adt, device=A.device)
+            res[g] = out
+        oshape, ostride = out.shape, out.stride()
+        if len(oshape) != 2 or oshape[0] != M or oshape[1] != N or not (ostride[1] == 1 or N <= 1):
+            _out_matrix(out, M, N, f"outs[{g}]")          # raises the precise error
+        if cdt is None:
+            cdt = out.dtype
+            _dtype_code(cdt)
+        elif out.dtype is not cdt:
+            raise ValueError("outputs must share one dtype")
+        ld = max(ostride[0], N)
+        ldcs[g] = -(-ld // 16) * 16 if M == 1 else ld
+        Ms[g], Ns[g], Ks[g] = M, N, K
+        pA[g], pB[g], pC[g] = A.data_ptr(), B.data_ptr(), out.data_ptr()
+    I64G, PG = C.c_int64 * G, C.c_void_p * G
     nbytes = int(lib().smgemm_grouped_workspace_size(G))
-    sh = _stream(stream)
     ws, wsb = (workspace, _ws_bytes(workspace)) if workspace is not None else _workspace(nbytes, As[0].device, sh)
-    bias_dt = next((_dtype_code(b.dtype) for b in (biases or []) if b is not None), 0)
-    _need(all(b is None or _dtype_code(b.dtype) == bias_dt for b in (biases or [])), "biases must share one dtype")
-    st = lib().gemm_bf16_grouped(G, arr(Ms), arr(Ns), arr(Ks), ptrs(As), _dtype_code(As[0].dtype), lay_a,
-                                 arr(ldas), ptrs(Bs), lay_b, arr(ldbs),
-                                 None if biases is None else ptrs(biases), bias_dt, ACTS[act],
-                                 ptrs(res), _dtype_code(res[0].dtype), arr(ldcs),
-                                 None if ws is None else ws.data_ptr(), wsb, sh)
-    _check(st, "gemm_bf16_grouped")
-    return res
+    bias_dt, pbias = 0, None
+    if biases is not None:
+        bias_dt = next((_dtype_code(b.dtype) for b in biases if b is not None), 0)
+        _need(all(b is None or _dtype_code(b.dtype) == bias_dt for b in biases), "biases must share one dtype")
+        pbias = PG(*[None if b is None else b.data_ptr() for b in biases])
+    args = (G, I64G(*Ms), I64G(*Ns), I64G(*Ks), PG(*pA), _dtype_code(adt), lay_a, I64G(*ldas), PG(*pB), lay_b,
+            I64G(*ldbs), pbias, bias_dt, ACTS[act], PG(*pC), _dtype_code(cdt), I64G(*ldcs),
+            None if ws is None else ws.data_ptr(), wsb, sh)
+    return args, list(res)
+
+
+class GroupedGemm:
+    """A grouped GEMM prepared once and launched many times: the tensors are checked and
+    the argument arrays of gemm_bf16_grouped built in the constructor, so each call only
+    enqueues the launch (the host time of a call with many small groups - MoE experts at
+    decode sizes - is then the library's own, not the argument marshalling). The tensors
+    must keep their storage, shapes and strides (their contents may change) for as long
+    as the object is used; the object holds references to them.
+
+        g = GroupedGemm(As, Bs, biases=None, act="none", outs=None, out_dtype=None, workspace=None)
+        g()                # or g(stream=s); returns the outputs
+    """
+
+    def __init__(self, As, Bs, *, biases=None, act="none", outs=None, out_dtype=None, workspace=None):
+        torch = _torch()
+        G = len(As)
+        if len(Bs) != G or (biases is not None and len(biases) != G) or (outs is not None and len(outs) != G):
+            raise ValueError("As, Bs, biases and outs must have one entry per group")
+        if G == 0:
+            raise ValueError("a grouped GEMM needs at least one group")
+        self.device = _device(*As, *Bs, *(biases or ()), *(outs or ()), workspace)
+        if workspace is None:   # its own workspace: calls on different streams may overlap
+            workspace = torch.empty(max(int(lib().smgemm_grouped_workspace_size(G)), 16), dtype=torch.uint8,
+                                    device=As[0].device)
+        args, self.outs = _grouped_marshal(As, Bs, biases, act, outs, out_dtype, workspace, 0)
+        self._args = list(args)
+        self._keep = (list(As), list(Bs), list(biases or ()), workspace)
+
+    def __call__(self, stream=None):
+        if self.device != _current_device():
+            with _torch().cuda.device(self.device):
+                return self(stream)
+        self._args[-1] = _stream(stream)
+        _check(lib().gemm_bf16_grouped(*self._args), "gemm_bf16_grouped")
+        return self.outs
 
 
 def gemm_fp8_blockscaled(Aq, sa, Bq, sb, *, bias=None, act="none", out=None, out_dtype=None,

@@ -25,18 +25,18 @@ def test_layout_rejects_non_unit_strides():
 
 def test_layout_as_reads_single_rows_and_columns_in_either_layout():
     row = torch.zeros(1, 64)                                   # one row, contiguous
-    assert sg._layout_as(row, "r", sg.ROW_MAJOR) == (sg.ROW_MAJOR, 64)
+    assert sg._layout_as(row, "r", sg.ROW_MAJOR) == 64
     # read as column-major its column pitch is real (1 element); the C ABI rejects that
     # pitch (not 16 bytes), so the binding passes it on rather than inventing another
-    assert sg._layout_as(row, "r", sg.COL_MAJOR) == (sg.COL_MAJOR, 1)
+    assert sg._layout_as(row, "r", sg.COL_MAJOR) == 1
     padded_row = torch.zeros(64, 8)[:, :1].t()                 # one row, column pitch 8
-    assert sg._layout_as(padded_row, "r", sg.COL_MAJOR) == (sg.COL_MAJOR, 8)
+    assert sg._layout_as(padded_row, "r", sg.COL_MAJOR) == 8
     col = torch.zeros(64, 8)[:, :1]                            # one column of a pitch-8 buffer
-    assert sg._layout_as(col, "c", sg.ROW_MAJOR) == (sg.ROW_MAJOR, 8)
+    assert sg._layout_as(col, "c", sg.ROW_MAJOR) == 8
     with pytest.raises(ValueError):                            # its 64 elements are 8 apart
         sg._layout_as(col, "c", sg.COL_MAJOR)
     dense_col = torch.zeros(64, 1)                             # 64 consecutive elements
-    assert sg._layout_as(dense_col, "c", sg.COL_MAJOR) == (sg.COL_MAJOR, 64)  # unused pitch: >= rows
+    assert sg._layout_as(dense_col, "c", sg.COL_MAJOR) == 64  # unused pitch: >= rows
     with pytest.raises(ValueError):
         sg._layout_as(torch.zeros(4, 8), "x", sg.COL_MAJOR)    # a true row-major matrix
 
@@ -231,3 +231,22 @@ def test_single_row_output_pitch_is_rounded(monkeypatch):
     sg.gemm_bf16(torch.zeros(1, 16, dtype=bf), torch.zeros(16, 50257, dtype=bf), out_dtype=torch.float32)
     sg.gemm_bf16(torch.zeros(2, 16, dtype=bf), torch.zeros(16, 24, dtype=bf))
     assert seen == [50272, 24]
+
+
+def test_prepared_grouped_call_marshals_once(monkeypatch):
+    """GroupedGemm builds the same arguments as gemm_bf16_grouped and each call passes
+    them unchanged (only the stream handle is refreshed)."""
+    rec = _RecordingLib()
+    _host_only(monkeypatch, rec)
+    bf = torch.bfloat16
+    As = [torch.zeros(16 * (g + 1), 32, dtype=bf) for g in range(3)]
+    Bs = [torch.zeros(32, 24, dtype=bf) for _ in range(3)]
+    outs = [torch.zeros(16 * (g + 1), 24, dtype=bf) for g in range(3)]
+    ws = torch.zeros(64, dtype=torch.uint8)
+    sg.gemm_bf16_grouped(As, Bs, outs=outs, workspace=ws, act="gelu_tanh")
+    pg = sg.GroupedGemm(As, Bs, outs=outs, workspace=ws, act="gelu_tanh")
+    assert pg() is pg.outs and pg() is pg.outs
+    one_shot, *prepared = rec.calls
+    assert len(prepared) == 2
+    for d in prepared:
+        assert d == one_shot

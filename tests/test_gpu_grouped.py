@@ -161,3 +161,21 @@ def test_grouped_misaligned_workspace_is_rejected_before_any_launch(cuda_device)
     sg.gemm_bf16_grouped(As, Bs, outs=outs, workspace=torch.zeros(nbytes, dtype=torch.uint8, device="cuda"))
     assert sg.check() == sg.OK
     assert bool((outs[0] == 1024.0).all()) and bool((outs[1] == 0.0).all())
+
+
+def test_prepared_grouped_gemm_matches_one_shot_calls(cuda_device):
+    """GroupedGemm checks and marshals once; each call only launches. Two calls, with the
+    inputs' contents changed in between, equal gemm_bf16_grouped on the same tensors bit
+    for bit (the kernel reads the tensors at launch time)."""
+    shapes = [(128 * (g + 1), 512, 256) for g in range(8)]
+    As = [to_dtype(synth.normal(42, g, (M, K)), torch.bfloat16).cuda() for g, (M, N, K) in enumerate(shapes)]
+    Bs = [to_dtype(synth.normal(42, 100 + g, (K, N), 0.1), torch.bfloat16).cuda() for g, (M, N, K) in enumerate(shapes)]
+    prepared = sg.GroupedGemm(As, Bs, act="silu", out_dtype=torch.bfloat16)
+    for step in range(2):
+        got = [o.clone() for o in prepared()]
+        want = sg.gemm_bf16_grouped(As, Bs, act="silu", out_dtype=torch.bfloat16)
+        assert sg.check() == sg.OK
+        for g in range(len(shapes)):
+            assert torch.equal(got[g], want[g]), f"step {step} group {g}"
+        for A in As:
+            A.mul_(-0.5)                       # new contents, same storage
