@@ -536,7 +536,7 @@ def run_gpu(args, rank: int, world: int, dist):
                      "peak_kind": f"{peaks['source']} bf16 burst",
                      "traffic": recorded_traffic("gemm_tc16_pair", "square_bf16_4096"),
                      "algorithmic_bytes": h["set_bytes"], "algorithmic_flops": h["flops"],
-                     "kernel": "gemm_tc16_pair_kernel<64,6> (CTA pairs, 256x256 tiles)"},
+                     "kernel": "gemm_tc16_pair_kernel<64,6,kOutTma> (CTA pairs, 256x256 tiles, TMA-store epilogue)"},
         "gpu_launches": c.launches,
         "clocks": h["clocks"],
         "configs": c.results,
