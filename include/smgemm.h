@@ -69,8 +69,10 @@ typedef enum { SMGEMM_ACT_NONE = 0, SMGEMM_ACT_GELU_TANH = 1, SMGEMM_ACT_SILU = 
  *   C        device, c_dtype SMGEMM_F32 / SMGEMM_BF16 / SMGEMM_F16, row-major, ldc >= N.
  *   workspace  device scratch of at least smgemm_workspace_size(M,N,K,0) bytes,
  *            16-byte aligned (may be NULL when that size is 0). The library uses it
- *            for split-K / stream-K partial tiles; it must not be shared by calls
- *            that can overlap on the GPU.
+ *            for split-K / stream-K partial tiles and their arrival counters; its
+ *            contents on entry do not matter (no zeroing needed: the counters carry a
+ *            per-call generation). It must not be shared by calls that can overlap on
+ *            the GPU.
  * Small M (<= 64, row-major A) runs the memory-bound swap-AB path; everything else
  * the persistent tensor-core path. Results are deterministic run to run.
  */
@@ -92,8 +94,8 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K,
  *   device image; every GPU that loads the library holds it until the process exits.
  *   A call whose schedule needs more scratch than that (at most smgemm_workspace_size)
  *   returns SMGEMM_ERR_WORKSPACE before enqueueing anything. The library allocates nothing.
- *   All calls share the array and it keeps the previous call's contents (each call
- *   clears what must start at zero); calls that can overlap on the GPU race on it.
+ *   All calls share the array and it keeps the previous call's contents (nothing in it
+ *   needs clearing); calls that can overlap on the GPU race on it.
  *   The first call on each device resolves the array's device address; under CUDA's
  *   default lazy module loading it also loads the library's device code there and
  *   reserves the array (milliseconds, may synchronise), so make it during warm-up,

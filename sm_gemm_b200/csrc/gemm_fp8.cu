@@ -100,6 +100,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
   const TileSched& s = p.s;
   const uint64_t limit = p.wait_limit_cycles;
   const int M = p.e.M;
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int n = 0;
           for (int c = c_lo; c <= c_hi; ++c) n += sk_bound(s, c) < sk_bound(s, c + 1);
           const bool any_dead = *abort_flag != 0;
-          const int old = any_dead ? -1 : atomicAdd(p.counters + t_sk, 1);
+          const int old = any_dead ? -1 : counter_arrive(p.counters + t_sk, p.gen);
           *reduce_flag = (!any_dead && old == n - 1);
         }
         named_barrier_sync(1, kPromoThreads);
@@ -311,7 +313,15 @@ cudaError_t launch_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& tm_b, co
   static const cudaError_t attr =
       cudaFuncSetAttribute(gemm_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (attr != cudaSuccess) return attr;
-  gemm_fp8_kernel<<<grid, kThreads, SMEM, stream>>>(tm_a, tm_b, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute la[1];
+  add_pdl_attr(cfg, la);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_fp8_kernel, tm_a, tm_b, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

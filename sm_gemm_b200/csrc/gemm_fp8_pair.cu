@@ -129,6 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
   const TileSched& s = p.s;
   const uint64_t limit = p.wait_limit_cycles;
   if (warp < kPromoWarp0) {
@@ -329,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int n = 0;
           for (int c = c_lo; c <= c_hi; ++c) n += sk_bound(s, c) < sk_bound(s, c + 1);
           const bool any_dead = *abort_flag != 0;
-          const int old = any_dead ? -1 : atomicAdd(p.counters + t_sk * 2 + rank, 1);
+          const int old = any_dead ? -1 : counter_arrive(p.counters + t_sk * 2 + rank, p.gen);
           *reduce_flag = (!any_dead && old == n - 1);
         }
         named_barrier_sync(1, kPromoThreads);
@@ -422,8 +424,9 @@ cudaError_t launch(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Fp8Pa
                    cudaStream_t stream) {
   cudaError_t e = prepare<TN>();
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pair_config<TN>(clusters, stream, attr);
+  add_pdl_attr(cfg, attr);
   e = cudaLaunchKernelEx(&cfg, gemm_fp8_pair_kernel<TN>, tm_a, tm_b, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -168,6 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
   const uint64_t limit = p.wait_limit_cycles;
 
   if (warp == 0) {
@@ -302,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_barrier_sync(1, kEpiThreads);
         if (epi_tid == 0) {
           const bool any_dead = *abort_flag != 0;
-          const int old = any_dead ? -1 : atomicAdd(sp.counters + r_tail * 2 + rank, 1);
+          const int old = any_dead ? -1 : counter_arrive(sp.counters + r_tail * 2 + rank, sp.gen);
           *reduce_flag = (!any_dead && old == sp.splits - 1);
         }
         named_barrier_sync(1, kEpiThreads);
@@ -387,8 +389,9 @@ cudaError_t launch_gemm_grouped_split(const GroupedParams& p, const GroupedSplit
                                       int clusters, cudaStream_t stream) {
   cudaError_t e = prepare();
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = config(clusters, stream, attr);
+  add_pdl_attr(cfg, attr);
   if (inl != nullptr) e = cudaLaunchKernelEx(&cfg, gemm_grouped_kernel<kBK, kStages, true>, p, sp, *inl);
   else e = cudaLaunchKernelEx(&cfg, gemm_grouped_kernel<kBK, kStages, false>, p, sp, NoInlineTable{});
   if (e != cudaSuccess) return e;
@@ -396,7 +399,7 @@ cudaError_t launch_gemm_grouped_split(const GroupedParams& p, const GroupedSplit
 }
 
 cudaError_t launch_gemm_grouped(const GroupedParams& p, int clusters, cudaStream_t stream) {
-  return launch_gemm_grouped_split(p, GroupedSplit{0, 0, nullptr, nullptr}, nullptr, clusters, stream);
+  return launch_gemm_grouped_split(p, GroupedSplit{0, 0, nullptr, nullptr, 0}, nullptr, clusters, stream);
 }
 
 unsigned take_error_word_grouped() { return take_error_word(); }

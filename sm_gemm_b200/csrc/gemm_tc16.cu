@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
   const TileSched& s = p.s;
   const uint64_t limit = p.wait_limit_cycles;
 
@@ -278,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int n = 0;
           for (int c = c_lo; c <= c_hi; ++c) n += sk_bound(s, c) < sk_bound(s, c + 1);
           const bool any_dead = *abort_flag != 0;
-          const int old = any_dead ? -1 : atomicAdd(p.counters + t_sk, 1);
+          const int old = any_dead ? -1 : counter_arrive(p.counters + t_sk, p.gen);
           *reduce_flag = (!any_dead && old == n - 1);
         }
         named_barrier_sync(1, 128);
@@ -328,7 +330,15 @@ static cudaError_t launch_tc16(const CUtensorMap& tm_a, const CUtensorMap& tm_b,
   auto kern = gemm_tc16_kernel<MMA_N, BK, STAGES, SWAP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, SMEM, stream>>>(tm_a, tm_b, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  add_pdl_attr(cfg, attr);
+  e = cudaLaunchKernelEx(&cfg, kern, tm_a, tm_b, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -165,6 +165,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();  // both CTAs' barriers exist before any remote arrive or copy targets them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();
   const TileSched& s = p.s;
   const uint64_t limit = p.wait_limit_cycles;
 
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int n = 0;
           for (int c = c_lo; c <= c_hi; ++c) n += sk_bound(s, c) < sk_bound(s, c + 1);
           const bool any_dead = *abort_flag != 0;
-          const int old = any_dead ? -1 : atomicAdd(p.counters + t_sk * 2 + rank, 1);
+          const int old = any_dead ? -1 : counter_arrive(p.counters + t_sk * 2 + rank, p.gen);
           *reduce_flag = (!any_dead && old == n - 1);
         }
         named_barrier_sync(1, kEpiThreads);
@@ -459,18 +461,21 @@ cudaError_t launch_gemm_tc16_pair(const CUtensorMap& tm_a, const CUtensorMap& tm
   cudaError_t e = out == kOutFp8 ? prepare_pair_kernel<kOutFp8>()
                                  : (out == kOutTma ? prepare_pair_kernel<kOutTma>() : prepare_pair_kernel<kOutDirect>());
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   CUtensorMap none;
   std::memset(&none, 0, sizeof(none));
   const CUtensorMap& mc = tm_c != nullptr ? *tm_c : none;
   if (out == kOutFp8) {
     cudaLaunchConfig_t cfg = pair_config<kOutFp8>(clusters, stream, attr);
+    add_pdl_attr(cfg, attr);
     e = cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages, kOutFp8>, tm_a, tm_b, mc, p);
   } else if (out == kOutTma) {
     cudaLaunchConfig_t cfg = pair_config<kOutTma>(clusters, stream, attr);
+    add_pdl_attr(cfg, attr);
     e = cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages, kOutTma>, tm_a, tm_b, mc, p);
   } else {
     cudaLaunchConfig_t cfg = pair_config<kOutDirect>(clusters, stream, attr);
+    add_pdl_attr(cfg, attr);
     e = cudaLaunchKernelEx(&cfg, gemm_tc16_pair_kernel<kPairBK, kPairStages, kOutDirect>, tm_a, tm_b, mc, p);
   }
   if (e != cudaSuccess) return e;

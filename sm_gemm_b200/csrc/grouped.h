@@ -11,7 +11,8 @@ struct GroupedSplit {
   long long split_tiles;    // R (0: no split)
   int splits;               // S pieces per split tile
   float* slots;             // [R * S][2 ranks][128][256] float partials
-  int* counters;            // [R][2], zeroed before the launch
+  unsigned long long* counters;  // [R][2] arrival counters (counter_arrive)
+  unsigned long long gen;        // this call's counter generation
 };
 
 // Up to kInlineGroups groups travel with the launch itself, as a kernel parameter (the

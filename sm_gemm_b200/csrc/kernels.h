@@ -27,7 +27,8 @@ struct Tc16Params {
   int a_mn_major;           // MMA "A" operand tile is MN-major (else K-major)
   int b_mn_major;           // MMA "B" operand tile is MN-major (else K-major)
   float* slots;             // stream-K partial tiles: [num_ctas][2][MMA_N][128] floats
-  int* counters;            // stream-K arrival counters, one per stream-K tile, zeroed per call
+  unsigned long long* counters;  // stream-K arrival counters (counter_arrive), one per stream-K tile
+  unsigned long long gen;        // this call's counter generation
   unsigned long long wait_limit_cycles;
   // Swap-AB (skinny) kernels only, nullable: per 128-column tile of the output and per
   // token row, the tile's max logit and sum of exp(logit - max) (float2 [m_tiles][M]).
@@ -95,7 +96,8 @@ struct Fp8Params {
   const float* sb;          // [KB][NB]
   int nb_count;             // NB = ceil(N/128)
   float* slots;             // [num_ctas][2][128][128] floats
-  int* counters;
+  unsigned long long* counters;  // stream-K arrival counters (counter_arrive)
+  unsigned long long gen;        // this call's counter generation
   unsigned long long wait_limit_cycles;
 };
 

@@ -14,10 +14,11 @@
 //    library holds that array until the process exits.
 //  - A call whose schedule needs more scratch than that is rejected with
 //    SMGEMM_ERR_WORKSPACE before anything is enqueued.
-//  - All calls share the one array, and it keeps the previous call's contents; the
-//    arrival counters that must start at zero are cleared on the stream by every call.
-//    Calls that can overlap on the GPU (different streams, different host threads)
-//    race on the array and must not be issued concurrently.
+//  - All calls share the one array, and it keeps the previous call's contents; nothing
+//    in it needs clearing (the split tiles' arrival counters carry a per-call
+//    generation, so words left by an earlier call never count). Calls that can overlap
+//    on the GPU (different streams, different host threads) race on the array and must
+//    not be issued concurrently.
 //  - The first call on each device resolves the array's device address
 //    (cudaGetSymbolAddress, with that device current). Under CUDA's default lazy
 //    module loading that first call is also what loads the library's device code on

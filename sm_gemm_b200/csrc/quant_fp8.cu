@@ -168,6 +168,11 @@ __device__ __forceinline__ QRing q_ring_setup(uint8_t* smem_raw) {
     fence_barrier_init();
   }
   __syncthreads();
+  // Programmatic dependent launch: the next kernel on the stream may start its own set-up
+  // now, and this one touches global memory only once the previous kernel has finished
+  // (griddepcontrol.wait returns at once when there is none).
+  pdl_launch_dependents();
+  pdl_wait();
   return q;
 }
 
@@ -383,6 +388,21 @@ __global__ void wait_selftest_kernel(unsigned long long limit_cycles) {
 
 }  // namespace
 
+namespace {
+// Launch configuration with programmatic dependent launch (the quantisers call
+// griddepcontrol.wait before touching global memory, so they may start early).
+cudaLaunchConfig_t pdl_config(unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                              cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  add_pdl_attr(cfg, attr);
+  return cfg;
+}
+}  // namespace
+
 cudaError_t launch_quant_1x128_tma(const CUtensorMap& tm_x, long long rows, long long cols, uint8_t* Q, float* S,
                                    int sms, unsigned long long limit, cudaStream_t stream) {
   static cudaError_t attr = cudaFuncSetAttribute(quant_1x128_tma_kernel,
@@ -397,8 +417,10 @@ cudaError_t launch_quant_1x128_tma(const CUtensorMap& tm_x, long long rows, long
   const long long tiles = (rows + kQ1Rows - 1) / kQ1Rows * ((cols + 127) / 128);
   const long long cap = static_cast<long long>(per_sm > 0 ? per_sm : 1) * sms;
   const long long blocks = tiles < cap ? tiles : cap;
-  quant_1x128_tma_kernel<<<static_cast<unsigned>(blocks), kQThreads, kQ1Smem, stream>>>(tm_x, rows, cols, Q, S,
-                                                                                        limit);
+  cudaLaunchAttribute la[1];
+  const cudaLaunchConfig_t cfg = pdl_config(static_cast<unsigned>(blocks), kQThreads, kQ1Smem, stream, la);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, quant_1x128_tma_kernel, tm_x, rows, cols, Q, S, limit);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -414,17 +436,21 @@ cudaError_t launch_quant_128x128_tma(const CUtensorMap& tm_x, bool n_contig, lon
                                      float* S, int sms, unsigned long long limit, cudaStream_t stream) {
   const long long tiles = ((K + 127) / 128) * ((N + 127) / 128);
   const unsigned blocks = static_cast<unsigned>(tiles < sms ? tiles : sms);
+  cudaLaunchAttribute la[1];
+  const cudaLaunchConfig_t cfg = pdl_config(blocks, kQThreads, kQ2Smem, stream, la);
+  cudaError_t e;
   if (n_contig) {
     static cudaError_t attr = cudaFuncSetAttribute(quant_128x128_tma_kernel<true>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kQ2Smem);
     if (attr != cudaSuccess) return attr;
-    quant_128x128_tma_kernel<true><<<blocks, kQThreads, kQ2Smem, stream>>>(tm_x, K, N, Q, S, limit);
+    e = cudaLaunchKernelEx(&cfg, quant_128x128_tma_kernel<true>, tm_x, K, N, Q, S, limit);
   } else {
     static cudaError_t attr = cudaFuncSetAttribute(quant_128x128_tma_kernel<false>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kQ2Smem);
     if (attr != cudaSuccess) return attr;
-    quant_128x128_tma_kernel<false><<<blocks, kQThreads, kQ2Smem, stream>>>(tm_x, K, N, Q, S, limit);
+    e = cudaLaunchKernelEx(&cfg, quant_128x128_tma_kernel<false>, tm_x, K, N, Q, S, limit);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

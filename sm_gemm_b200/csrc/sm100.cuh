@@ -12,6 +12,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstdlib>
+
 namespace smg {
 
 // ------------------------------------------------------------------ error word
@@ -169,6 +171,31 @@ __device__ __forceinline__ void regs_dec() {
 template <uint32_t N>
 __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Kernels launched with programmatic stream serialisation may begin while the previous
+// kernel on the stream is still finishing. Each kernel lets its successor start setting up
+// (launch_dependents) and, before touching global memory, waits until the previous
+// kernel has completed and its writes are visible (wait: immediate when there is none).
+// Only set-up (barrier init, TMEM allocation, descriptor prefetch) precedes the wait.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Host side: the launch attribute, unless SMGEMM_PDL=0.
+inline bool pdl_enabled() {
+  const char* v = std::getenv("SMGEMM_PDL");
+  return !(v != nullptr && v[0] == '0');
+}
+inline void add_pdl_attr(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attrs) {
+  if (!pdl_enabled()) return;
+  attrs[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs += 1;
 }
 
 // ------------------------------------------------------------------ TMA
@@ -543,6 +570,28 @@ struct WorkIter {
     return false;
   }
 };
+
+// Arrival of one contributor on a split tile's counter. A counter word holds the call's
+// generation (upper 48 bits, a number the host draws afresh for every call, never 0) and
+// the number of this call's arrivals (lower 16 bits); a word of another generation -
+// left by an earlier call, or whatever a fresh workspace holds - counts as zero arrivals.
+// So the workspace needs no zeroing before a call (the chance that a stale word carries
+// the current generation is 2^-48). Returns the number of earlier arrivals of this call,
+// or -1 if the compare-and-swap kept failing (it cannot fail more often than there are
+// contributors; the bound only keeps the loop finite).
+__device__ __forceinline__ int counter_arrive(unsigned long long* c, unsigned long long gen) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(c);
+#pragma unroll 1
+  for (int i = 0; i < 4096; ++i) {
+    const bool same = (cur >> 16) == gen;
+    const unsigned long long want = same ? cur + 1ull : ((gen << 16) | 1ull);
+    const unsigned long long prev = atomicCAS(c, cur, want);
+    if (prev == cur) return same ? static_cast<int>(cur & 0xffffull) : 0;
+    cur = prev;
+  }
+  atomicOr(&g_error_word, kErrTimeout);  // reported by smgemm_check like an abandoned wait
+  return -1;
+}
 
 // Partial-tile slot access for the TMEM lane `r` (tile row) and N consecutive columns
 // starting at col0 (N and col0 multiples of 4): float4 units at [col/4][r], so a

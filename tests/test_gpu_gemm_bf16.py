@@ -365,3 +365,32 @@ def test_tma_store_epilogue_matches_direct_stores(cuda_device, monkeypatch, out_
         ref, acc = oracle.gemm(a, b, a_dtype=ad, b_dtype=bdt, bias=bb, bias_dtype=bbd, act=ORC_ACT[act],
                                out_dtype=TORCH_TO_ORC[out_dt], want_absacc=True)
         check_tolerance(outs["tma"].float().cpu().numpy(), ref, acc, out_dt, what=f"tma store {M}x{N}x{K}")
+
+
+# ------------------------------------------------------------------ split-tile counters need no zeroing
+
+@pytest.mark.parametrize("fill", ["zeros", "garbage", "ones"])
+def test_split_counters_need_no_zeroed_workspace(cuda_device, fill):
+    """The split tail's arrival counters carry a per-call generation, so the workspace is
+    used as found: zeros, random bytes or all-ones bytes, and the words the previous call
+    left, all give the same bits as a fresh call (4096^3 splits its ragged last wave)."""
+    M = N = K = 4096
+    A = torch.from_numpy(synth.integers(98, 0, (M, K), -3, 3)).to(torch.bfloat16).cuda()
+    B = torch.from_numpy(synth.integers(98, 1, (K, N), -3, 3)).to(torch.bfloat16).cuda()
+    plan = sg.schedule_dump(M, N, K, 0, sg.ROW_MAJOR, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert (plan[:, 6] >= 0).any()
+    nbytes = sg.workspace_size(M, N, K, 0)
+    ref = sg.gemm_bf16(A, B, out_dtype=torch.float32)
+    if fill == "zeros":
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    elif fill == "ones":
+        ws = torch.full((nbytes,), 0xFF, dtype=torch.uint8, device="cuda")
+    else:
+        ws = torch.randint(0, 256, (nbytes,), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        out = sg.gemm_bf16(A, B, out_dtype=torch.float32, workspace=ws)
+        assert sg.check() == sg.OK
+        assert torch.equal(out, ref)
+    # integer inputs: every partial sum is exact, so the split result is the exact product
+    exact = (A.double() @ B.double()).float()
+    assert torch.equal(ref, exact)
