@@ -458,15 +458,15 @@ def wl_lm_head(c: Ctx, ms_list=(1, 4, 16, 64)):
         ms = c.time(lambda i: sg.gemm_bf16(Xl, Wl, out=Cl, workspace=ws))
         c.record(f"lm_head_m{mm}", ms, c.K, flops=m.gemm_flops(mm, 128256, 4096),
                  nbytes=m.gemm_bytes(mm, 128256, 4096, "bf16", "bf16", "f32"), extra={"plan": sg.last_config()})
-    # The same LM head fused with the row log-softmax (3 launches: GEMM with per-tile
-    # max/sum partials, lse merge, in-place subtract). Bytes add the second pass's read
+    # The same LM head fused with the row log-softmax (2 launches: GEMM with per-tile
+    # max/sum partials, then the merge and in-place subtract). Bytes add the second pass's read
     # and write of the FP32 output.
     mm = 16
     Xl = c.t(c.synth.lm_head(m=mm, vocab=8)["X"])
     Cl = torch.empty((mm, 128256), dtype=torch.float32, device=c.dev)
     wsl = torch.empty(max(int(sg.lib().smgemm_logsoftmax_workspace_size(mm, 128256, 4096)), 16), dtype=torch.uint8,
                       device=c.dev)
-    ms = c.time(lambda i: sg.gemm_bf16_logsoftmax(Xl, Wl, out=Cl, workspace=wsl), launches_per_step=3)
+    ms = c.time(lambda i: sg.gemm_bf16_logsoftmax(Xl, Wl, out=Cl, workspace=wsl), launches_per_step=2)
     c.record(f"lm_head_logsoftmax_m{mm}", ms, c.K, flops=m.gemm_flops(mm, 128256, 4096),
              nbytes=m.gemm_bytes(mm, 128256, 4096, "bf16", "bf16", "f32") + 2 * mm * 128256 * 4,
              extra={"plan": sg.last_config()})
@@ -488,10 +488,10 @@ def wl_lm_head_vocab_parallel(c: Ctx, mm: int = 16):
     del d
     Cl = torch.empty((mm, c1 - c0), dtype=torch.float32, device=c.dev)
     ws = torch.empty(max(sg.workspace_size(mm, max(c1 - c0, 1), K), 16), dtype=torch.uint8, device=c.dev)
-    # our kernels per step: the skinny GEMM (its epilogue forms the partials), the lse merge
-    # and the subtract; the all-gather is NCCL's and the padding of short slices torch's
+    # our kernels per step: the skinny GEMM (its epilogue forms the partials) and the merge +
+    # subtract; the all-gather is NCCL's and the padding of short slices torch's
     ms = c.time(lambda i: vp.lm_head_log_softmax(Xl, Ws, V, dist=c.dist, out=Cl, workspace=ws),
-                launches_per_step=3)
+                launches_per_step=2)
     c.record(f"lm_head_logsoftmax_vocab_parallel_m{mm}", ms, c.K, flops=m.gemm_flops(mm, V, K),
              nbytes=m.gemm_bytes(mm, V, K, "bf16", "bf16", "f32") + 2 * mm * V * 4,
              extra={"ranks": c.world, "slice_columns": c1 - c0, "scaling": "strong",

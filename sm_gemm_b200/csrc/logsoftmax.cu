@@ -120,6 +120,45 @@ __global__ void __launch_bounds__(256) lse_tile_partials_kernel(const float* __r
   if (lane == 0) part[static_cast<long long>(t) * M + m] = v.s > 0.0f ? make_float2(v.m, v.s) : make_float2(-INFINITY, 0.0f);
 }
 
+// Merge and subtract in one launch: CTA (x, m) merges row m's partials (every CTA of the
+// row in the same fixed order, so all get the same lse bit for bit; CTA 0 stores it) and
+// subtracts it from columns [x chunk, (x + 1) chunk) of the row.
+__global__ void __launch_bounds__(256) lse_merge_subtract_kernel(const float2* __restrict__ part, int n_parts,
+                                                                 int M, float* __restrict__ C, long long ldc, int N,
+                                                                 int chunk, float* __restrict__ lse) {
+  __shared__ MaxSum sh[8];
+  __shared__ float l_sh;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int m = blockIdx.y;
+  MaxSum v{-INFINITY, 0.0f};
+  for (int t = threadIdx.x; t < n_parts; t += blockDim.x) {
+    const float2 q = part[static_cast<size_t>(t) * M + m];
+    v = merge(v, MaxSum{q.x, q.y});
+  }
+  v = block_merge(v, sh);
+  if (threadIdx.x == 0) {
+    const float l = v.s > 0.0f ? v.m + logf(v.s) : -INFINITY;
+    l_sh = l;
+    if (blockIdx.x == 0) lse[m] = l;
+  }
+  __syncthreads();
+  const float l = l_sh;
+  float* row = C + static_cast<long long>(m) * ldc;
+  const int c0 = blockIdx.x * chunk;
+  const int c1 = c0 + chunk < N ? c0 + chunk : N;
+  if ((ldc & 3) == 0 && (N & 3) == 0) {
+    float4* r4 = reinterpret_cast<float4*>(row);
+    for (int q = (c0 >> 2) + threadIdx.x; q < (c1 >> 2); q += blockDim.x) {
+      float4 x = r4[q];
+      x.x -= l; x.y -= l; x.z -= l; x.w -= l;
+      r4[q] = x;
+    }
+  } else {
+    for (int n = c0 + threadIdx.x; n < c1; n += blockDim.x) row[n] -= l;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_lse_tile_partials(const float* C, long long ldc, int M, int N, float2* part, cudaStream_t stream) {
@@ -133,6 +172,23 @@ cudaError_t launch_lse_tile_partials(const float* C, long long ldc, int M, int N
 cudaError_t launch_log_softmax_rows(float* C, long long ldc, int M, int N, const float2* part, int n_tiles,
                                     float* lse, int sms, cudaStream_t stream) {
   if (M <= 0 || (part == nullptr && N <= 0)) return cudaSuccess;
+  if (part != nullptr && N > 0 && M <= 65535) {
+    // One launch: about four CTAs per SM over the rows' column chunks (multiples of 1024).
+    const long long ctas_per_row = (4LL * (sms > 0 ? sms : 1) + M - 1) / M;
+    long long chunk = (static_cast<long long>(N) + ctas_per_row - 1) / ctas_per_row;
+    chunk = (chunk + 1023) / 1024 * 1024;
+    const unsigned gx = static_cast<unsigned>((N + chunk - 1) / chunk);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(gx, static_cast<unsigned>(M), 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    add_pdl_attr(cfg, attr);
+    const cudaError_t e =
+        cudaLaunchKernelEx(&cfg, lse_merge_subtract_kernel, part, n_tiles, M, C, ldc, N, static_cast<int>(chunk), lse);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   if (part != nullptr) lse_from_partials_kernel<<<M, 256, 0, stream>>>(part, n_tiles, M, lse);
   else lse_from_logits_kernel<<<M, 256, 0, stream>>>(C, ldc, N, lse);
   cudaError_t e = cudaGetLastError();
