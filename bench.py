@@ -26,6 +26,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import subprocess
 import sys
@@ -141,9 +142,19 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- GPU arm
 
+# About 50 us of SM cycles: enough for the host to queue a few calls ahead.
+QUEUE_AHEAD_CYCLES = 100_000
+# Shortest timed region for the per-workload lines (see Ctx.time).
+MIN_TIMED_MS = 2.0
+
+
 def time_steps(torch, step, warmup: int, steps: int, dist=None):
     """Device time of `steps` calls of step(i) after `warmup` calls: CUDA events on the
-    current stream, barrier + synchronise on both sides, max over ranks (ms total)."""
+    current stream, barrier + synchronise on both sides, max over ranks (ms total).
+
+    A short spin kernel runs before the start event: while the device is busy with it
+    the host queues the first timed calls, so the timed region starts with work queued
+    instead of with the device waiting for the first launch to come through."""
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
@@ -151,6 +162,7 @@ def time_steps(torch, step, warmup: int, steps: int, dist=None):
         dist.barrier()
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(QUEUE_AHEAD_CYCLES)
     s.record()
     for i in range(steps):
         step(warmup + i)
@@ -217,15 +229,28 @@ class Ctx:
         self.peaks = load_peaks()
         self.fp8_peak = 2.0 * self.peaks["bf16_tflops"]   # measured bf16 x nominal fp8/bf16 ratio (2)
         self.W, self.K = args.warmup, args.steps
+        self.min_ms = args.min_timed_ms if args.min_timed_ms > 0 else None
         self.world, self.dist = world, dist
         self.launches = 0
         self.results = {}
 
-    def time(self, step, launches_per_step=1, warmup=None, steps=None):
+    def time(self, step, launches_per_step=1, warmup=None, steps=None, min_ms="default"):
+        """Device time (ms) of K calls of step. With min_ms (and no explicit step
+        count), a workload whose K calls took less than min_ms is timed again over
+        enough calls to span it, and the result is scaled back to K calls: kernels of a
+        few microseconds are then not measured over a region as short as their launch
+        jitter. The headline passes min_ms=None and is timed over exactly K steps."""
         w = self.W if warmup is None else warmup
         k = self.K if steps is None else steps
+        if min_ms == "default":
+            min_ms = self.min_ms
         ms = time_steps(self.torch, step, w, k, self.dist)
         self.launches += launches_per_step * k
+        if steps is None and min_ms is not None and 0 < ms < min_ms:
+            k2 = int(math.ceil(k * min_ms / ms))
+            ms2 = time_steps(self.torch, step, 0, k2, self.dist)
+            self.launches += launches_per_step * k2
+            ms = ms2 * k / k2
         return ms
 
     def record(self, name, ms_total, steps, flops=None, nbytes=None, peak_tf=None, extra=None):
@@ -269,7 +294,7 @@ def wl_square_bf16(c: Ctx, headline: bool):
     except Exception:
         smi_id = str(c.dev.index)
     with ClockSampler(smi_id) as clk:
-        ms = c.time(step)
+        ms = c.time(step, min_ms=None)
     dist_us = per_call_us(torch, step, c.W + c.K, max(50, c.K))
     assert sg.check() == sg.OK
     flops = m.gemm_flops(n, n, n)
@@ -643,6 +668,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="smgemm", choices=["smgemm", "reference"])
     ap.add_argument("--headline-only", action="store_true")
+    ap.add_argument("--min-timed-ms", type=float, default=MIN_TIMED_MS,
+                    help="shortest timed region of a per-workload line (0: exactly --steps calls, "
+                         "for a fixed launch sequence under a profiler)")
     ap.add_argument("--only", default=None,
                     choices=["square_bf16", "tiny_fp16", "ffn", "ffn_bwd", "grouped", "fp8", "quant", "lm_head",
                              "lm_head_vp"],

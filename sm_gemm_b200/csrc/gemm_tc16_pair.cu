@@ -262,6 +262,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int epi_tid = threadIdx.x - kEpiWarp0 * 32;
     const int c_base = cq * kEpiCols;        // first tile column of this warp
     constexpr int SLOT = 128 * kTileN;
+    // TMEM chunk c (32 columns) of this warp's accumulator columns, as floats; and back.
+    auto tmem_chunk = [&](uint32_t tacc, int c, float (&v)[32]) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32_sync(tacc + c * 32, r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    };
+    auto tmem_keep = [&](uint32_t tacc, int c, const float (&v)[32]) {
+      uint32_t r[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(v[j]);
+      tmem_st_32x32b_x32(tacc + c * 32, r);
+    };
+    // This warp is done with accumulator buffer b (its TMEM reads and writes included).
+    auto release_acc = [&](int b) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(b), 0));
+    };
     int local = 0;
     WorkIter it;
     it.init(s, cluster);
@@ -282,32 +301,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!dead) {
         tc_fence_after();
         if constexpr (FP8OUT) {
-          // This warp's 128 columns are one 1x128 group of each row: two passes over
-          // TMEM, the activated values written back in place between them.
-          auto load = [&](int c, float (&v)[32]) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32_sync(tacc + c * 32, r);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          };
           if (whole) {
-            auto keep = [&](int c, const float (&v)[32]) {
-              uint32_t r[32];
-#pragma unroll
-              for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(v[j]);
-              tmem_st_32x32b_x32(tacc + c * 32, r);
-            };
-            // The stores of pass 1 complete before pass 2 reads the columns back.
-            auto again = [&](int c, float (&v)[32]) {
-              if (c == 0) tmem_st_wait();
-              load(c, v);
-            };
-            epi_group_fp8_2pass(p.e, row, col0, load, keep, again);
+            // This warp's 128 columns are one 1x128 group of each row: two passes over
+            // TMEM, the activated values written back in place between them.
+            epi_group_fp8_2pass(p.e, row, col0, [&](int c, float (&v)[32]) { tmem_chunk(tacc, c, v); },
+                                [&](int c, const float (&v)[32]) { tmem_keep(tacc, c, v); },
+                                [&](int c, float (&v)[32]) {
+                                  if (c == 0) tmem_st_wait();  // pass 1's stores have landed
+                                  tmem_chunk(tacc, c, v);
+                                });
           } else {
 #pragma unroll 1
             for (int c = 0; c < kEpiCols / 32; ++c) {
               float v[32];
-              load(c, v);
+              tmem_chunk(tacc, c, v);
               slot_store<32>(my_slot, r_local, c_base + c * 32, v);
             }
           }
@@ -332,12 +339,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+        // A stream-K piece with FP8 output keeps its accumulator buffer through the fix-up
+        // below (see there); every other tile releases it now.
+        if (whole || !FP8OUT) release_acc(acc);
       }
 
       if (!whole) {
+        // Stream-K tile: the last contributor to arrive sums the partials in K order and
+        // runs the epilogue. The fix-up's L2 traffic is slow while the other SMs stream
+        // operands, so a 16/32-bit output frees the accumulator first (the next tile's
+        // MMAs proceed meanwhile) and reads every partial from the slots. The FP8-output
+        // epilogue needs the finished values twice (group amax, then the codes): its
+        // pieces keep the buffer, and the reducer adds its own partial from TMEM and
+        // keeps pass 1's activated values there, instead of summing the slots twice.
         const long long t_sk = seg.tile - s.dp_tiles;
         __threadfence();
         named_barrier_sync(1, kEpiThreads);
@@ -353,38 +367,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_barrier_sync(1, kEpiThreads);
         if (*reduce_flag) {
           __threadfence();
-          const int c_lo = sk_owner(s, t_sk * s.kb_total);
-          const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
-          // Sum of every contributor's partial for 32 columns (CTA order = K order).
-          auto reduce32 = [&](int col, float (&v)[32]) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-#pragma unroll 1
-            for (int cc = c_lo; cc <= c_hi; ++cc) {
-              if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
-              const float* src = p.slots + ((static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * 2 + rank) * SLOT;
-              slot_accumulate<32>(src, r_local, col, v);
-            }
-          };
           if constexpr (FP8OUT) {
-            // No TMEM to keep the activated chunks in: pass 2 sums the partials again
-            // and re-applies bias and activation (the same arithmetic, the same values).
-            auto load = [&](int c, float (&v)[32]) { reduce32(c_base + c * 32, v); };
-            auto keep = [&](int, const float (&)[32]) {};
-            auto again = [&](int c, float (&v)[32]) {
-              reduce32(c_base + c * 32, v);
-              if (p.e.bias != nullptr || p.e.act != 0) epi_bias_act32(p.e, col0 + 32 * c, v);
+            // Pass 1 sums the partials in K order (this CTA's own from TMEM) and keeps
+            // the activated values in TMEM for pass 2.
+            auto reduce32 = [&](int c, float (&v)[32]) {
+              sk_tile_sum<32>(
+                  s, t_sk, cluster,
+                  [&](int cc) {
+                    return p.slots + ((static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * 2 + rank) * SLOT;
+                  },
+                  [&](float* acc_v) {
+                    float o[32];
+                    tmem_chunk(tacc, c, o);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) acc_v[j] += o[j];
+                  },
+                  r_local, c_base + c * 32, v);
             };
-            epi_group_fp8_2pass(p.e, row, col0, load, keep, again);
+            epi_group_fp8_2pass(p.e, row, col0, reduce32, [&](int c, const float (&v)[32]) { tmem_keep(tacc, c, v); },
+                                [&](int c, float (&v)[32]) {
+                                  if (c == 0) tmem_st_wait();
+                                  tmem_chunk(tacc, c, v);
+                                });
           } else {
+            const int c_lo = sk_owner(s, t_sk * s.kb_total);
+            const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
 #pragma unroll 1
             for (int c = 0; c < kEpiCols / 32; ++c) {
               float v[32];
-              reduce32(c_base + c * 32, v);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+              // Sum of every contributor's partial (CTA order = K order).
+#pragma unroll 1
+              for (int cc = c_lo; cc <= c_hi; ++cc) {
+                if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
+                const float* src = p.slots + ((static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * 2 + rank) * SLOT;
+                slot_accumulate<32>(src, r_local, c_base + c * 32, v);
+              }
               epi_row32(p.e, row, col0 + c * 32, v);
             }
           }
         }
+        if (FP8OUT && !dead) release_acc(acc);
         named_barrier_sync(1, kEpiThreads);
       }
       ++local;

@@ -544,7 +544,9 @@ struct WorkIter {
   }
   // Stream-K range first, then the data-parallel tiles: the fix-up of a split tile
   // (done by its last contributor's epilogue warps) then overlaps the MMAs of that
-  // CTA's remaining tiles instead of landing in the kernel's tail.
+  // CTA's remaining tiles instead of landing in the kernel's tail. (Measured on the
+  // 4096^3 and FFN shapes: with the pieces last instead, the fix-ups, all in the tail
+  // at once, cost 5-13 us more per call.)
   __host__ __device__ bool next(const TileSched& s, Seg& out) {
     if (sk_pos < sk_end) {
       const long long t = sk_pos / s.kb_total;
@@ -615,6 +617,68 @@ __device__ __forceinline__ void slot_accumulate(const float* slot, int r, int co
     v[4 * q + 2] += t.z;
     v[4 * q + 3] += t.w;
   }
+}
+
+// v += slot0, then v += slot1 (the same additions, in the same order, as two
+// slot_accumulate calls), with both slots' loads issued before the first add: a split
+// tile's reduction waits for one L2 round trip per pair of contributors instead of one
+// per contributor.
+template <int N>
+__device__ __forceinline__ void slot_accumulate2(const float* slot0, const float* slot1, int r, int col0, float* v) {
+  const float4* a4 = reinterpret_cast<const float4*>(slot0);
+  const float4* b4 = reinterpret_cast<const float4*>(slot1);
+  float4 a[N / 4], b[N / 4];
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) a[q] = __ldcg(a4 + ((col0 >> 2) + q) * 128 + r);
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) b[q] = __ldcg(b4 + ((col0 >> 2) + q) * 128 + r);
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) {
+    v[4 * q] += a[q].x;
+    v[4 * q + 1] += a[q].y;
+    v[4 * q + 2] += a[q].z;
+    v[4 * q + 3] += a[q].w;
+  }
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) {
+    v[4 * q] += b[q].x;
+    v[4 * q + 1] += b[q].y;
+    v[4 * q + 2] += b[q].z;
+    v[4 * q + 3] += b[q].w;
+  }
+}
+
+// Sum, in contributor (= K) order, of the N columns col0.. of the partials of stream-K
+// tile t_sk: slot_of(cc) gives contributor cc's slot, and own(v), when the calling CTA
+// `self` is a contributor whose partial is still on chip (TMEM or registers), adds that
+// partial in its place instead of reading it back. Slot loads are issued two
+// contributors at a time.
+template <int N, class SlotOf, class Own>
+__device__ __forceinline__ void sk_tile_sum(const TileSched& s, long long t_sk, int self, SlotOf slot_of, Own own,
+                                            int r, int col0, float* v) {
+#pragma unroll
+  for (int j = 0; j < N; ++j) v[j] = 0.0f;
+  const int c_lo = sk_owner(s, t_sk * s.kb_total);
+  const int c_hi = sk_owner(s, (t_sk + 1) * s.kb_total - 1);
+  const float* pend = nullptr;
+#pragma unroll 1
+  for (int cc = c_lo; cc <= c_hi; ++cc) {
+    if (!(sk_bound(s, cc) < sk_bound(s, cc + 1))) continue;
+    if (cc == self) {
+      if (pend != nullptr) slot_accumulate<N>(pend, r, col0, v);
+      pend = nullptr;
+      own(v);
+      continue;
+    }
+    const float* src = slot_of(cc);
+    if (pend == nullptr) {
+      pend = src;
+    } else {
+      slot_accumulate2<N>(pend, src, r, col0, v);
+      pend = nullptr;
+    }
+  }
+  if (pend != nullptr) slot_accumulate<N>(pend, r, col0, v);
 }
 
 // The slot a contributor CTA `c` used for stream-K tile `t_sk` (index among the
