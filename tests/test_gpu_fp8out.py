@@ -10,6 +10,8 @@ block-scaled FP8 GEMM.
   the GEMM contract (1e-3 sum|a||b|, times 1.2 for the slope of GeLU) plus one E4M3
   spacing at the value (the FP32 value may sit beside a rounding midpoint of the exact
   one), and every scale within the same relative bound of the exact amax / 448.
+- Tiles split along K (split tail, stream-K range): the same exact codes and the same
+  bounds.
 - The output feeds gemm_fp8_blockscaled; that GEMM is checked against the oracle on
   the same codes and scales."""
 import numpy as np
@@ -44,7 +46,31 @@ def test_fp8out_integer_exact(cuda_device, M, N, K):
     assert np.array_equal(Q.cpu().numpy(), Qr)
 
 
-def test_fp8out_bias_gelu_tolerance(cuda_device):
+@pytest.mark.parametrize("M,N,K,sched", [(512, 1024, 4096, "auto"), (300, 520, 1024, "sk"), (256, 256, 2048, "sk")])
+def test_fp8out_split_tiles_integer_exact(cuda_device, monkeypatch, M, N, K, sched):
+    """Tiles whose K range is cut over several CTAs: a ragged last wave split in 8 pieces
+    (auto), or one stream-K range over all CTAs (sk). The reducer sums the pieces in K
+    order with its own piece taken from TMEM, wherever it falls in that order, and keeps
+    the activated values in TMEM between the two passes; integer inputs keep every
+    partial sum exact, so codes and scales must still equal the oracle's bit for bit."""
+    monkeypatch.setenv("SMGEMM_SCHED", sched)
+    A = torch.from_numpy(synth.integers(65, 0, (M, K), -3, 3)).to(torch.bfloat16)
+    B = torch.from_numpy(synth.integers(65, 1, (K, N), -3, 3)).to(torch.bfloat16)
+    Q, S = sg.gemm_bf16_fp8out(A.cuda(), B.cuda())
+    assert sg.check() == sg.OK
+    plan = dict(kv.split("=") for kv in sg.last_config().split() if "=" in kv)
+    assert int(plan["sk_iters"]) > 0, sg.last_config()
+    a, ad = orc_view(A)
+    b, bd = orc_view(B)
+    Z = oracle.gemm(a, b, a_dtype=ad, b_dtype=bd, out_dtype=oracle.F32).astype(np.float32)
+    Qr, Sr = oracle.quant_1x128(Z)
+    assert np.array_equal(S.cpu().numpy().view(np.uint32), Sr.view(np.uint32))
+    assert np.array_equal(Q.cpu().numpy(), Qr)
+
+
+@pytest.mark.parametrize("sched", ["auto", "sk"])
+def test_fp8out_bias_gelu_tolerance(cuda_device, monkeypatch, sched):
+    monkeypatch.setenv("SMGEMM_SCHED", sched)
     M, N, K = 384, 1000, 520
     A = to_dtype(synth.normal(62, 0, (M, K)), torch.bfloat16)
     B = to_dtype(synth.normal(62, 1, (K, N), 0.05), torch.bfloat16)
