@@ -122,7 +122,9 @@ __global__ void __launch_bounds__(256) lse_tile_partials_kernel(const float* __r
 
 // Merge and subtract in one launch: CTA (x, m) merges row m's partials (every CTA of the
 // row in the same fixed order, so all get the same lse bit for bit; CTA 0 stores it) and
-// subtracts it from columns [x chunk, (x + 1) chunk) of the row.
+// subtracts it from columns [x chunk, (x + 1) chunk) of the row. Each thread issues the
+// loads of its first four float4 of the chunk before the merge, so their latency overlaps
+// it, and loads its partials four at a time.
 __global__ void __launch_bounds__(256) lse_merge_subtract_kernel(const float2* __restrict__ part, int n_parts,
                                                                  int M, float* __restrict__ C, long long ldc, int N,
                                                                  int chunk, float* __restrict__ lse) {
@@ -131,10 +133,31 @@ __global__ void __launch_bounds__(256) lse_merge_subtract_kernel(const float2* _
   pdl_launch_dependents();
   pdl_wait();
   const int m = blockIdx.y;
+  const int bd = static_cast<int>(blockDim.x);
+  float* row = C + static_cast<long long>(m) * ldc;
+  const int c0 = blockIdx.x * chunk;
+  const int c1 = c0 + chunk < N ? c0 + chunk : N;
+  const bool vec = (ldc & 3) == 0 && (N & 3) == 0;
+  float4* r4 = reinterpret_cast<float4*>(row);
+  const int q0 = (c0 >> 2) + static_cast<int>(threadIdx.x), q1 = c1 >> 2;
+  float4 x[4];
+  if (vec) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (q0 + u * bd < q1) x[u] = r4[q0 + u * bd];
+  }
+  // Partials t = threadIdx.x, + blockDim.x, ... merged in that order (identity pairs past
+  // n_parts change nothing).
   MaxSum v{-INFINITY, 0.0f};
-  for (int t = threadIdx.x; t < n_parts; t += blockDim.x) {
-    const float2 q = part[static_cast<size_t>(t) * M + m];
-    v = merge(v, MaxSum{q.x, q.y});
+  for (int t0 = static_cast<int>(threadIdx.x); t0 < n_parts; t0 += 4 * bd) {
+    float2 q[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int t = t0 + u * bd;
+      q[u] = t < n_parts ? part[static_cast<size_t>(t) * M + m] : make_float2(-INFINITY, 0.0f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v = merge(v, MaxSum{q[u].x, q[u].y});
   }
   v = block_merge(v, sh);
   if (threadIdx.x == 0) {
@@ -144,18 +167,22 @@ __global__ void __launch_bounds__(256) lse_merge_subtract_kernel(const float2* _
   }
   __syncthreads();
   const float l = l_sh;
-  float* row = C + static_cast<long long>(m) * ldc;
-  const int c0 = blockIdx.x * chunk;
-  const int c1 = c0 + chunk < N ? c0 + chunk : N;
-  if ((ldc & 3) == 0 && (N & 3) == 0) {
-    float4* r4 = reinterpret_cast<float4*>(row);
-    for (int q = (c0 >> 2) + threadIdx.x; q < (c1 >> 2); q += blockDim.x) {
-      float4 x = r4[q];
-      x.x -= l; x.y -= l; x.z -= l; x.w -= l;
-      r4[q] = x;
+  if (vec) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int q = q0 + u * bd;
+      if (q < q1) {
+        x[u].x -= l; x[u].y -= l; x[u].z -= l; x[u].w -= l;
+        r4[q] = x[u];
+      }
+    }
+    for (int q = q0 + 4 * bd; q < q1; q += bd) {
+      float4 y = r4[q];
+      y.x -= l; y.y -= l; y.z -= l; y.w -= l;
+      r4[q] = y;
     }
   } else {
-    for (int n = c0 + threadIdx.x; n < c1; n += blockDim.x) row[n] -= l;
+    for (int n = c0 + static_cast<int>(threadIdx.x); n < c1; n += bd) row[n] -= l;
   }
 }
 
