@@ -146,6 +146,10 @@ class ClockSampler:
 QUEUE_AHEAD_CYCLES = 100_000
 # Shortest timed region for the per-workload lines (see Ctx.time).
 MIN_TIMED_MS = 2.0
+# Device warm-up before the headline's own warm-up steps: ~50 ms of a spin kernel. The
+# first timed region of a process otherwise ran 0.5-3 us per call slower than the next
+# ones on the same data (measured on B200 boxes; with the spin the difference was gone).
+DEVICE_WARMUP_CYCLES = 100_000_000
 
 
 def time_steps(torch, step, warmup: int, steps: int, dist=None):
@@ -289,6 +293,8 @@ def wl_square_bf16(c: Ctx, headline: bool):
         j = i % copies
         sg.gemm_bf16(As[j], Bs[j].t(), out=Cs[j], workspace=ws)
 
+    torch.cuda._sleep(DEVICE_WARMUP_CYCLES)
+    torch.cuda.synchronize()
     try:
         smi_id = "GPU-" + str(torch.cuda.get_device_properties(c.dev).uuid)
     except Exception:
@@ -555,7 +561,8 @@ def run_gpu(args, rank: int, world: int, dist):
                    "accumulate": "fp32",
                    "l2": f"rotating {h['copies']} input/output sets ({h['copies'] * h['set_bytes'] / 2**20:.0f} MiB) "
                          f"so reuse distance exceeds L2",
-                   "parallelism": f"replicas{world}" if world > 1 else "single-gpu", "plan": h["plan"]},
+                   "parallelism": f"replicas{world}" if world > 1 else "single-gpu", "plan": h["plan"],
+                   "device_warmup": "~50 ms spin kernel before the warm-up steps"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
                      "peak_kind": f"{peaks['source']} bf16 burst",
