@@ -18,6 +18,8 @@
 #include <mutex>
 #include <vector>
 
+#include <unistd.h>  // environ
+
 #include <nvtx3/nvToolsExt.h>
 
 #include "../../include/smgemm.h"
@@ -28,14 +30,66 @@ using namespace smg;
 
 namespace {
 
-// One NVTX range per entry-point call, named after the entry point, so a profiler's
-// timeline shows which library call enqueued which kernels (the profiling practice of
-// "为什么我们要死磕GEMM" (kwkr.cn), section 7.1). Without an attached tool a range costs
-// one predictable branch (NVTX's header-only API).
-struct NvtxRange {
-  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
-  ~NvtxRange() { nvtxRangePop(); }
+// ------------------------------------------------------------------ environment switches
+
+// The SMGEMM_* switches (tuning and test overrides), read in one pass over the
+// environment when a call enters the library, instead of a separate scan of the whole
+// environment for each of the dozen switches a GEMM call consults.
+enum Knob {
+  kKnobGrid, kKnobSched, kKnobSplitK, kKnobForceConfig, kKnobPair, kKnobForceLarge, kKnobGroupM, kKnobFp8Tn,
+  kKnobLog, kKnobWaitLimitNs, kKnobEpiStore, kKnobGroupedSplit, kKnobPdl, kNumKnobs
 };
+const char* const kKnobNames[kNumKnobs] = {
+    "SMGEMM_GRID", "SMGEMM_SCHED", "SMGEMM_SPLITK", "SMGEMM_FORCE_CONFIG", "SMGEMM_PAIR", "SMGEMM_FORCE_LARGE",
+    "SMGEMM_GROUP_M", "SMGEMM_FP8_TN", "SMGEMM_LOG", "SMGEMM_WAIT_LIMIT_NS", "SMGEMM_EPI_STORE",
+    "SMGEMM_SCHED_GROUPED_SPLIT", "SMGEMM_PDL"};
+thread_local const char* g_knobs[kNumKnobs] = {};
+
+void refresh_knobs() {
+  const char* k[kNumKnobs] = {};
+  for (char** e = environ; e != nullptr && *e != nullptr; ++e) {
+    const char* s = *e;
+    if (std::strncmp(s, "SMGEMM_", 7) != 0) continue;
+    const char* eq = std::strchr(s, '=');
+    if (eq == nullptr) continue;
+    const size_t n = static_cast<size_t>(eq - s);
+    for (int i = 0; i < kNumKnobs; ++i) {
+      if (std::strlen(kKnobNames[i]) == n && std::memcmp(kKnobNames[i], s, n) == 0) {
+        k[i] = eq + 1;
+        break;
+      }
+    }
+  }
+  for (int i = 0; i < kNumKnobs; ++i) g_knobs[i] = k[i];
+}
+
+const char* knob(Knob i) { return g_knobs[i]; }
+
+// Every entry point that plans or launches work opens one: an NVTX range named after the
+// entry point, so a profiler's timeline shows which library call enqueued which kernels
+// (the profiling practice of "为什么我们要死磕GEMM" (kwkr.cn), section 7.1; without an
+// attached tool a range costs one predictable branch, NVTX's header-only API), and a
+// fresh snapshot of the SMGEMM_* switches for the call.
+struct CallScope {
+  explicit CallScope(const char* name) {
+    nvtxRangePushA(name);
+    refresh_knobs();
+  }
+  ~CallScope() { nvtxRangePop(); }
+};
+
+}  // namespace
+
+namespace smg {
+// Launch attribute switch of the kernel launchers (declared in sm100.cuh): programmatic
+// dependent launch unless SMGEMM_PDL=0 when the current call entered the library.
+bool pdl_enabled() {
+  const char* v = knob(kKnobPdl);
+  return !(v != nullptr && v[0] == '0');
+}
+}  // namespace smg
+
+namespace {
 
 // ------------------------------------------------------------------ driver entry point
 
@@ -95,8 +149,8 @@ smgemm_status current_device(DevInfo& out) {
 
 thread_local char g_last_config[256] = "none";
 
-long long env_ll(const char* name, long long dflt) {
-  const char* v = std::getenv(name);
+long long env_ll(Knob name, long long dflt) {
+  const char* v = knob(name);
   if (v == nullptr || *v == 0) return dflt;
   return std::atoll(v);
 }
@@ -104,7 +158,7 @@ long long env_ll(const char* name, long long dflt) {
 enum class SchedMode { kAuto, kDP, kSK };
 
 SchedMode sched_mode() {
-  const char* v = std::getenv("SMGEMM_SCHED");
+  const char* v = knob(kKnobSched);
   if (v == nullptr) return SchedMode::kAuto;
   if (std::strcmp(v, "dp") == 0) return SchedMode::kDP;
   if (std::strcmp(v, "sk") == 0) return SchedMode::kSK;
@@ -118,7 +172,7 @@ SchedMode sched_mode() {
 // switches SMGEMM_PAIR=0, SMGEMM_FORCE_LARGE=1 and SMGEMM_FP8_TN=128 mean "single",
 // "large" and "pair128".
 bool force_config_is(const char* want) {
-  const char* v = std::getenv("SMGEMM_FORCE_CONFIG");
+  const char* v = knob(kKnobForceConfig);
   return v != nullptr && std::strcmp(v, want) == 0;
 }
 
@@ -164,14 +218,14 @@ Plan make_plan(int m_tiles, int n_tiles, int kb_total, int sms, int group_m, siz
                int counters_per_tile = 1, long long splitk_default = 0) {
   Plan pl;
   const long long T = static_cast<long long>(m_tiles) * n_tiles;
-  long long max_ctas = env_ll("SMGEMM_GRID", sms);
+  long long max_ctas = env_ll(kKnobGrid, sms);
   if (max_ctas < 1) max_ctas = 1;
   if (max_ctas > sms) max_ctas = sms;
   SchedMode mode = sched_mode();
   constexpr int kMinItersPerPiece = 8;
   // SMGEMM_SPLITK=s: 1 = every tile whole (data-parallel only); s >= 2 = every tile's K
   // range cut into about s pieces (one stream-K range over min(P, s T) CTAs).
-  const long long splitk = env_ll("SMGEMM_SPLITK", splitk_default);
+  const long long splitk = env_ll(kKnobSplitK, splitk_default);
   if (splitk == 1) mode = SchedMode::kDP;
 
   long long dp = T, sk_iters = 0, sk_ctas = 0, grid = std::min<long long>(T, max_ctas);
@@ -311,8 +365,8 @@ struct Gemm16Plan {
 Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms, int pair_clusters,
                        bool allow_skinny = true) {
   Gemm16Plan g;
-  const bool force_single = force_config_is("single") || env_ll("SMGEMM_PAIR", 1) == 0;
-  const bool force_large = env_ll("SMGEMM_FORCE_LARGE", 0) != 0 || !allow_skinny || force_config_is("large") ||
+  const bool force_single = force_config_is("single") || env_ll(kKnobPair, 1) == 0;
+  const bool force_large = env_ll(kKnobForceLarge, 0) != 0 || !allow_skinny || force_config_is("large") ||
                            force_config_is("pair") || force_single;
   g.skinny = (M <= 64 && layout_a == SMGEMM_ROW_MAJOR && !force_large);
   g.pair = !g.skinny && pair_clusters > 0 && !force_single;
@@ -322,7 +376,7 @@ Gemm16Plan plan_gemm16(int64_t M, int64_t N, int64_t K, int layout_a, int sms, i
   g.bk = g.pair ? tc16_pair_bk() : tc16_bk(g.v);
   const int kb = static_cast<int>((K + g.bk - 1) / g.bk);
   const TunedConfig* t = g.pair ? find_tuned(0, M, N, K, layout_a) : nullptr;
-  const int group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", t != nullptr ? t->group_m : 8));
+  const int group_m = static_cast<int>(env_ll(kKnobGroupM, t != nullptr ? t->group_m : 8));
   if (g.pair) {
     g.pl = make_plan(static_cast<int>((M + 255) / 256), static_cast<int>((N + 255) / 256), std::max(kb, 1),
                      pair_clusters, group_m, static_cast<size_t>(2) * 128 * 256, 2, t != nullptr ? t->splitk : 0);
@@ -347,15 +401,15 @@ struct Fp8Plan {
   Plan pl;
 };
 
-int fp8_tile_n() { return (env_ll("SMGEMM_FP8_TN", 256) == 128 || force_config_is("pair128")) ? 128 : 256; }
+int fp8_tile_n() { return (env_ll(kKnobFp8Tn, 256) == 128 || force_config_is("pair128")) ? 128 : 256; }
 
 Fp8Plan plan_fp8(int64_t M, int64_t N, int64_t K, int sms, int tn, int pair_clusters) {
   Fp8Plan f;
   const int kb = static_cast<int>((K + kFp8BK - 1) / kFp8BK);
-  f.pair = pair_clusters > 0 && env_ll("SMGEMM_PAIR", 1) != 0 && !force_config_is("single");
+  f.pair = pair_clusters > 0 && env_ll(kKnobPair, 1) != 0 && !force_config_is("single");
   f.tn = tn;
   const TunedConfig* t = f.pair && tn == 256 ? find_tuned(1, M, N, K, SMGEMM_ROW_MAJOR) : nullptr;
-  const int group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", t != nullptr ? t->group_m : 8));
+  const int group_m = static_cast<int>(env_ll(kKnobGroupM, t != nullptr ? t->group_m : 8));
   if (f.pair) {
     f.pl = make_plan(static_cast<int>((M + 255) / 256), static_cast<int>((N + tn - 1) / tn), std::max(kb, 1),
                      pair_clusters, group_m, static_cast<size_t>(2) * 128 * tn, 2, t != nullptr ? t->splitk : 0);
@@ -405,13 +459,13 @@ void note_config(const char* path, const Plan& pl, int mma_n) {
                 "path=%s tile=128x%d tiles=%dx%d kb=%d grid=%d dp_tiles=%d sk_iters=%lld sk_ctas=%d ws=%zu", path,
                 mma_n, pl.s.m_tiles, pl.s.n_tiles, pl.s.kb_total, pl.grid, pl.s.dp_tiles, pl.s.sk_iters, pl.s.sk_ctas,
                 pl.ws_bytes());
-  if (env_ll("SMGEMM_LOG", 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
+  if (env_ll(kKnobLog, 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
 }
 
 // Limit of the kernels' bounded barrier waits, in SM cycles.
 unsigned long long wait_limit() {
   return kCyclesPerNs *
-         static_cast<unsigned long long>(env_ll("SMGEMM_WAIT_LIMIT_NS", static_cast<long long>(kWaitLimitNs)));
+         static_cast<unsigned long long>(env_ll(kKnobWaitLimitNs, static_cast<long long>(kWaitLimitNs)));
 }
 
 }  // namespace
@@ -434,6 +488,7 @@ const char* smgemm_status_string(smgemm_status st) {
 const char* smgemm_last_config(void) { return g_last_config; }
 
 size_t smgemm_workspace_size(int64_t M, int64_t N, int64_t K, int kind) {
+  refresh_knobs();  // the plan, hence the size, follows the SMGEMM_* switches
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   DevInfo d;
   if (current_device(d) != SMGEMM_OK) return 0;
@@ -533,7 +588,7 @@ smgemm_status gemm16_impl(int64_t M, int64_t N, int64_t K, const void* A, smgemm
     // seen to write the rest of that unit (the columns just right of C) on B200.
     CUtensorMap tm_c;
     const CUtensorMap* pc = nullptr;
-    const char* es = std::getenv("SMGEMM_EPI_STORE");
+    const char* es = knob(kKnobEpiStore);
     if (!fp8_out && (N * elem_size(c_dtype)) % 16 == 0 && !(es != nullptr && std::strcmp(es, "direct") == 0)) {
       const CUtensorMapDataType cdt = c_dtype == SMGEMM_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                       : c_dtype == SMGEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -559,7 +614,7 @@ smgemm_status gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, smgemm_d
                         smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b, int64_t ldb,
                         const void* bias, smgemm_dtype bias_dtype, smgemm_act act, void* C, smgemm_dtype c_dtype,
                         int64_t ldc, void* workspace, size_t workspace_bytes, smgemm_stream_t stream) {
-  const NvtxRange nvtx_range("smgemm:gemm_bf16");
+  const CallScope scope("smgemm:gemm_bf16");
   return gemm16_impl(M, N, K, A, ab_dtype, layout_a, lda, B, layout_b, ldb, bias, bias_dtype, act, C, c_dtype, ldc,
                      workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr);
 }
@@ -568,7 +623,7 @@ smgemm_status gemm_bf16_fp8out(int64_t M, int64_t N, int64_t K, const void* A, s
                                smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b, int64_t ldb,
                                const void* bias, smgemm_dtype bias_dtype, smgemm_act act, uint8_t* Cq, int64_t ldc,
                                float* scales, void* workspace, size_t workspace_bytes, smgemm_stream_t stream) {
-  const NvtxRange nvtx_range("smgemm:gemm_bf16_fp8out");
+  const CallScope scope("smgemm:gemm_bf16_fp8out");
   if (scales == nullptr) return SMGEMM_ERR_INVALID_ARG;
   return gemm16_impl(M, N, K, A, ab_dtype, layout_a, lda, B, layout_b, ldb, bias, bias_dtype, act, Cq, SMGEMM_E4M3,
                      ldc, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, scales);
@@ -584,7 +639,7 @@ smgemm_status gemm_bf16_logsoftmax(int64_t M, int64_t N, int64_t K, const void* 
                                    smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b,
                                    int64_t ldb, const void* bias, smgemm_dtype bias_dtype, float* C, int64_t ldc,
                                    void* workspace, size_t workspace_bytes, smgemm_stream_t stream_) {
-  const NvtxRange nvtx_range("smgemm:gemm_bf16_logsoftmax");
+  const CallScope scope("smgemm:gemm_bf16_logsoftmax");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (M < 0 || N < 0 || K < 0) return SMGEMM_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return SMGEMM_OK;
@@ -610,7 +665,7 @@ smgemm_status gemm_bf16_lse_partials(int64_t M, int64_t N, int64_t K, const void
                                      smgemm_layout layout_a, int64_t lda, const void* B, smgemm_layout layout_b,
                                      int64_t ldb, const void* bias, smgemm_dtype bias_dtype, float* C, int64_t ldc,
                                      float* part, void* workspace, size_t workspace_bytes, smgemm_stream_t stream_) {
-  const NvtxRange nvtx_range("smgemm:gemm_bf16_lse_partials");
+  const CallScope scope("smgemm:gemm_bf16_lse_partials");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (M < 0 || N < 0 || K < 0) return SMGEMM_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return SMGEMM_OK;
@@ -628,7 +683,7 @@ smgemm_status gemm_bf16_lse_partials(int64_t M, int64_t N, int64_t K, const void
 
 smgemm_status logsoftmax_apply_partials(float* C, int64_t ldc, int64_t M, int64_t N, const float* part,
                                         int64_t n_parts, float* lse, smgemm_stream_t stream_) {
-  const NvtxRange nvtx_range("smgemm:logsoftmax_apply_partials");
+  const CallScope scope("smgemm:logsoftmax_apply_partials");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (M < 0 || N < 0 || n_parts < 0 || !fits_int(M) || !fits_int(N) || !fits_int(n_parts))
     return SMGEMM_ERR_INVALID_ARG;
@@ -654,6 +709,7 @@ size_t grouped_split_bytes(int clusters) {
 }
 
 size_t smgemm_grouped_workspace_size(int G) {
+  refresh_knobs();
   if (G <= 0) return 0;
   DevInfo d;
   const int P = current_device(d) == SMGEMM_OK ? grouped_max_clusters() : 0;
@@ -666,7 +722,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
                                 const void* const* bias, smgemm_dtype bias_dtype, smgemm_act act, void* const* C,
                                 smgemm_dtype c_dtype, const int64_t* ldc, void* workspace, size_t workspace_bytes,
                                 smgemm_stream_t stream_) {
-  const NvtxRange nvtx_range("smgemm:gemm_bf16_grouped");
+  const CallScope scope("smgemm:gemm_bf16_grouped");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (G < 0 || (G > 0 && (M == nullptr || N == nullptr || K == nullptr || A == nullptr || lda == nullptr ||
                           B == nullptr || ldb == nullptr || C == nullptr || ldc == nullptr)))
@@ -755,7 +811,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   p.groups = dev_table;
   p.G = G;
   p.total_tiles = tiles;
-  p.group_m = static_cast<int>(env_ll("SMGEMM_GROUP_M", 8));
+  p.group_m = static_cast<int>(env_ll(kKnobGroupM, 8));
   p.bias_dtype = bias_dtype;
   p.act = act;
   p.c_dtype = c_dtype;
@@ -769,7 +825,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   const int P = clusters_max;
   const long long R = tiles % P;
   int S = 0;
-  if (R > 0 && env_ll("SMGEMM_SCHED_GROUPED_SPLIT", 1) != 0) {
+  if (R > 0 && env_ll(kKnobGroupedSplit, 1) != 0) {
     int min_kb = 1 << 30;
     long long left = R;
     for (int g = G - 1; g >= 0 && left > 0; --g) {
@@ -797,7 +853,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   std::snprintf(g_last_config, sizeof(g_last_config),
                 "path=grouped groups=%d tiles=%lld grid=%d tile=128x256 split_tiles=%lld splits=%d", G, tiles, clusters,
                 S >= 2 ? R : 0LL, S >= 2 ? S : 0);
-  if (env_ll("SMGEMM_LOG", 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
+  if (env_ll(kKnobLog, 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
   return launch_status(launch_gemm_grouped_split(p, sp, inline_table ? &inl : nullptr, clusters, stream));
 }
 
@@ -805,7 +861,7 @@ smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_
                                    const uint8_t* Bq, const float* sb, const void* bias, smgemm_dtype bias_dtype,
                                    smgemm_act act, void* C, smgemm_dtype c_dtype, int64_t ldc, void* workspace,
                                    size_t workspace_bytes, smgemm_stream_t stream_) {
-  const NvtxRange nvtx_range("smgemm:gemm_fp8_blockscaled");
+  const CallScope scope("smgemm:gemm_fp8_blockscaled");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!fits_int(M) || !fits_int(N) || !fits_int(K)) return SMGEMM_ERR_INVALID_ARG;
   if (!valid_out_dtype(c_dtype) || !valid_act(act)) return SMGEMM_ERR_INVALID_ARG;
@@ -853,7 +909,7 @@ smgemm_status gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_
 smgemm_status quantize_fp8_blockwise(const float* X, int64_t rows, int64_t cols, smgemm_layout layout_x,
                                      int64_t ldx, int group_rows, uint8_t* Q, float* scales,
                                      smgemm_stream_t stream_) {
-  const NvtxRange nvtx_range("smgemm:quantize_fp8_blockwise");
+  const CallScope scope("smgemm:quantize_fp8_blockwise");
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (rows < 0 || cols < 0 || !valid_layout(layout_x)) return SMGEMM_ERR_INVALID_ARG;
   if (group_rows != 1 && group_rows != 128) return SMGEMM_ERR_INVALID_ARG;
@@ -900,6 +956,7 @@ smgemm_status smgemm_selftest_wait_timeout(uint32_t limit_us, smgemm_stream_t st
 
 int64_t smgemm_schedule_dump(int64_t M, int64_t N, int64_t K, int kind, smgemm_layout layout_a, int num_sms,
                              int32_t* out, int64_t cap) {
+  refresh_knobs();
   if (M <= 0 || N <= 0 || K <= 0 || num_sms <= 0) return 0;
   const Plan pl = kind == 1 ? plan_fp8(M, N, K, num_sms, fp8_tile_n(), num_sms / 2).pl
                             : plan_gemm16(M, N, K, layout_a, num_sms, num_sms / 2).pl;

@@ -310,8 +310,7 @@ cudaError_t launch_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& tm_b, co
                             int grid, cudaStream_t stream) {
   constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + kRing * kSlotFloats * 4 + 8 * (2 * STAGES + 5 + 2 * kRing) + 16;
   static_assert(SMEM <= 232448, "shared memory budget");
-  static const cudaError_t attr =
-      cudaFuncSetAttribute(gemm_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  const cudaError_t attr = smem_opt_in<gemm_fp8_kernel>(SMEM);
   if (attr != cudaSuccess) return attr;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);

@@ -366,16 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 namespace {
-// Sets the shared-memory limit and checks that the registers the kernel launches with
-// cover the setmaxnreg split (otherwise the promotion warps' increase would never be
-// granted); a build that breaks the split fails here instead of launching.
+// Checks that the registers the kernel launches with cover the setmaxnreg split
+// (otherwise the promotion warps' increase would never be granted); a build that breaks
+// the split fails here instead of launching.
 template <int TN>
 cudaError_t prepare_once() {
-  cudaError_t e = cudaFuncSetAttribute(gemm_fp8_pair_kernel<TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       PairCfg<TN>::kSmem);
-  if (e != cudaSuccess) return e;
   cudaFuncAttributes attr{};
-  e = cudaFuncGetAttributes(&attr, gemm_fp8_pair_kernel<TN>);
+  const cudaError_t e = cudaFuncGetAttributes(&attr, gemm_fp8_pair_kernel<TN>);
   if (e != cudaSuccess) return e;
   if (attr.numRegs * kThreads < 128 * kRoleRegs + kPromoThreads * kPromoRegs) return cudaErrorInvalidConfiguration;
   return cudaSuccess;
@@ -384,7 +381,8 @@ cudaError_t prepare_once() {
 template <int TN>
 cudaError_t prepare() {
   static cudaError_t st = prepare_once<TN>();
-  return st;
+  if (st != cudaSuccess) return st;
+  return smem_opt_in<gemm_fp8_pair_kernel<TN>>(PairCfg<TN>::kSmem);
 }
 
 template <int TN>

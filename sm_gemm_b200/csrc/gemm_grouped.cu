@@ -342,14 +342,9 @@ constexpr int kSmem = 1024 + kStages * (2 * 128 * kBK * 2) + 8 * (2 * kStages + 
 static_assert(kSmem <= 232448, "shared memory budget");
 
 cudaError_t prepare() {
-  static cudaError_t st = [] {
-    cudaError_t e = cudaFuncSetAttribute(gemm_grouped_kernel<kBK, kStages, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(gemm_grouped_kernel<kBK, kStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                kSmem);
-  }();
-  return st;
+  const cudaError_t e = smem_opt_in<gemm_grouped_kernel<kBK, kStages, false>>(kSmem);
+  if (e != cudaSuccess) return e;
+  return smem_opt_in<gemm_grouped_kernel<kBK, kStages, true>>(kSmem);
 }
 
 cudaLaunchConfig_t config(int clusters, cudaStream_t stream, cudaLaunchAttribute* attr) {

@@ -328,7 +328,7 @@ static cudaError_t launch_tc16(const CUtensorMap& tm_a, const CUtensorMap& tm_b,
   constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5) + 16 + 8 * 32 * 4;
   static_assert(SMEM <= 232448, "shared memory budget");
   auto kern = gemm_tc16_kernel<MMA_N, BK, STAGES, SWAP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  cudaError_t e = smem_opt_in<gemm_tc16_kernel<MMA_N, BK, STAGES, SWAP>>(SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);

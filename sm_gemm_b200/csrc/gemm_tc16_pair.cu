@@ -434,9 +434,7 @@ static_assert(pair_smem<kOutTma>() <= 232448, "shared memory budget");
 
 template <int OUT>
 cudaError_t prepare_pair_kernel() {
-  static cudaError_t st = cudaFuncSetAttribute(gemm_tc16_pair_kernel<kPairBK, kPairStages, OUT>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, pair_smem<OUT>());
-  return st;
+  return smem_opt_in<gemm_tc16_pair_kernel<kPairBK, kPairStages, OUT>>(pair_smem<OUT>());
 }
 
 template <int OUT>

@@ -405,8 +405,7 @@ cudaLaunchConfig_t pdl_config(unsigned grid, unsigned block, size_t smem, cudaSt
 
 cudaError_t launch_quant_1x128_tma(const CUtensorMap& tm_x, long long rows, long long cols, uint8_t* Q, float* S,
                                    int sms, unsigned long long limit, cudaStream_t stream) {
-  static cudaError_t attr = cudaFuncSetAttribute(quant_1x128_tma_kernel,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kQ1Smem);
+  const cudaError_t attr = smem_opt_in<quant_1x128_tma_kernel>(kQ1Smem);
   if (attr != cudaSuccess) return attr;
   static int per_sm = 0;
   if (per_sm == 0 && cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_1x128_tma_kernel, kQThreads,
@@ -440,13 +439,11 @@ cudaError_t launch_quant_128x128_tma(const CUtensorMap& tm_x, bool n_contig, lon
   const cudaLaunchConfig_t cfg = pdl_config(blocks, kQThreads, kQ2Smem, stream, la);
   cudaError_t e;
   if (n_contig) {
-    static cudaError_t attr = cudaFuncSetAttribute(quant_128x128_tma_kernel<true>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kQ2Smem);
+    const cudaError_t attr = smem_opt_in<quant_128x128_tma_kernel<true>>(kQ2Smem);
     if (attr != cudaSuccess) return attr;
     e = cudaLaunchKernelEx(&cfg, quant_128x128_tma_kernel<true>, tm_x, K, N, Q, S, limit);
   } else {
-    static cudaError_t attr = cudaFuncSetAttribute(quant_128x128_tma_kernel<false>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kQ2Smem);
+    const cudaError_t attr = smem_opt_in<quant_128x128_tma_kernel<false>>(kQ2Smem);
     if (attr != cudaSuccess) return attr;
     e = cudaLaunchKernelEx(&cfg, quant_128x128_tma_kernel<false>, tm_x, K, N, Q, S, limit);
   }

@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <cstdlib>
 
 namespace smg {
@@ -185,11 +186,26 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Host side: the launch attribute, unless SMGEMM_PDL=0.
-inline bool pdl_enabled() {
-  const char* v = std::getenv("SMGEMM_PDL");
-  return !(v != nullptr && v[0] == '0');
+// Host side: the launch attribute, unless SMGEMM_PDL=0 (pdl_enabled() reads the switch
+// snapshot the library takes when a call enters it; defined with the C ABI).
+bool pdl_enabled();
+// Opts `Kernel` into `bytes` of dynamic shared memory, once per device: the attribute
+// belongs to the function on the device that is current when it is set, and persists, so
+// later calls on that device skip the runtime call (a per-call cost for small GEMMs).
+template <auto Kernel>
+inline cudaError_t smem_opt_in(int bytes) {
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> set_to[kMaxDev];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool track = dev >= 0 && dev < kMaxDev;
+  if (track && set_to[dev].load(std::memory_order_acquire) == bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && track) set_to[dev].store(bytes, std::memory_order_release);
+  return e;
 }
+
 inline void add_pdl_attr(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attrs) {
   if (!pdl_enabled()) return;
   attrs[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
