@@ -394,3 +394,39 @@ def test_split_counters_need_no_zeroed_workspace(cuda_device, fill):
     # integer inputs: every partial sum is exact, so the split result is the exact product
     exact = (A.double() @ B.double()).float()
     assert torch.equal(ref, exact)
+
+
+# ------------------------------------------------------------------ seeded random sweep
+
+def _sweep_cases(n=120, seed=2024):
+    rs = np.random.RandomState(seed)
+    cases = []
+    for i in range(n):
+        M = int(rs.choice([int(rs.randint(1, 65)), int(rs.randint(65, 700))]))
+        N = int(rs.randint(1, 700))
+        K = int(rs.randint(1, 900))
+        cases.append(dict(
+            M=M, N=N, K=K, ab=[torch.bfloat16, torch.float16][rs.randint(2)],
+            la=["row", "col"][rs.randint(2)], lb=["row", "col"][rs.randint(2)],
+            out_dt=[torch.float32, torch.bfloat16, torch.float16][rs.randint(3)],
+            bias_dt=[None, torch.float32, torch.bfloat16, torch.float16][rs.randint(4)],
+            act=["none", "gelu_tanh", "silu"][rs.randint(3)],
+            integer=bool(rs.randint(2)), sched=["auto", "dp", "sk"][rs.randint(3)],
+            pair=["1", "0"][rs.randint(2)], seed=100 + i))
+    return cases
+
+
+@pytest.mark.parametrize("case", _sweep_cases(), ids=lambda c: "M{M}N{N}K{K}".format(**c))
+def test_seeded_random_sweep(cuda_device, monkeypatch, case):
+    """Random shapes (tiny to several tiles, ragged in M, N and K), operand types,
+    layouts, bias types, activations, output types and schedules: integer inputs without
+    an activation match the oracle bit for bit; everything else meets the contract."""
+    c = dict(case)
+    monkeypatch.setenv("SMGEMM_SCHED", c.pop("sched"))
+    monkeypatch.setenv("SMGEMM_PAIR", c.pop("pair"))
+    M, N, K = c.pop("M"), c.pop("N"), c.pop("K")
+    got, ref, acc = run_case(M, N, K, **c)
+    if c["integer"] and c["act"] == "none" and c["bias_dt"] is None:
+        assert np.array_equal(got, ref), sg.last_config()
+    else:
+        check_tolerance(got, ref, acc, c["out_dt"], what=sg.last_config())
