@@ -23,6 +23,10 @@
  *  - Layouts: SMGEMM_ROW_MAJOR means the second index is contiguous,
  *    SMGEMM_COL_MAJOR the first. C is always row-major with leading dimension ldc.
  *  - No exception crosses this interface. Thread-safe.
+ *  - Tuning and test switches (SMGEMM_FORCE_CONFIG, SMGEMM_SPLITK, SMGEMM_SCHED,
+ *    SMGEMM_GROUP_M, SMGEMM_EPI_STORE, SMGEMM_PDL, SMGEMM_LOG, ...) are read from the
+ *    process environment once each time a call enters the library; each entry point
+ *    opens an NVTX range named after it ("smgemm:<entry point>").
  */
 #ifndef SMGEMM_H
 #define SMGEMM_H
