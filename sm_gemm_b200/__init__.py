@@ -196,6 +196,9 @@ def _layout(t, name):
     if len(st) != 2:
         raise ValueError(f"{name} must be 2-D")
     (rows, cols), (s0, s1) = t.shape, st
+    if rows == 0 or cols == 0:
+        # nothing is read; any strides (numpy gives an empty array zero strides)
+        return ROW_MAJOR, -(-max(cols, 1) // 8) * 8
     if s1 == 1 and (rows <= 1 or s0 >= cols):
         return ROW_MAJOR, max(s0, cols)
     if s0 == 1:
@@ -210,6 +213,8 @@ def _layout_as(t, name, want, g=None):
     in the error message."""
     rows, cols = t.shape
     s0, s1 = t.stride()
+    if rows == 0 or cols == 0:  # nothing is read: any strides, a 16-byte leading dimension
+        return -(-max(cols if want == ROW_MAJOR else rows, 1) // 8) * 8
     if want == ROW_MAJOR and (s1 == 1 or cols <= 1):
         return max(s0, cols) if rows > 1 else -(-max(cols, 1) // 8) * 8
     if want == COL_MAJOR and (s0 == 1 or rows <= 1):

@@ -250,3 +250,16 @@ def test_prepared_grouped_call_marshals_once(monkeypatch):
     assert len(prepared) == 2
     for d in prepared:
         assert d == one_shot
+
+
+def test_layout_accepts_empty_operands_of_any_strides():
+    """An empty operand (M = 0 or K = 0; numpy gives such arrays zero strides) is read
+    by nothing, so it fits either layout, with a 16-byte leading dimension."""
+    import numpy as np
+    e = torch.from_numpy(np.zeros((0, 456), dtype=np.float32)[:, :])
+    z = torch.from_numpy(np.ones((6, 1), dtype=np.float32)[:, :0])
+    for t in (e, z, torch.zeros(0, 0)):
+        lay, ld = sg._layout(t, "t")
+        assert lay == sg.ROW_MAJOR and ld % 8 == 0 and ld >= max(t.shape[1], 1)
+        assert sg._layout_as(t, "t", sg.ROW_MAJOR) % 8 == 0
+        assert sg._layout_as(t, "t", sg.COL_MAJOR) % 8 == 0

@@ -322,3 +322,48 @@ def test_fp8_gemm_output_and_bias_types(cuda_device, monkeypatch, out_dt, bias_d
     ref, acc = oracle.gemm_fp8(qa, sa, qb, sb, bias=bb, bias_dtype=bd, act=oracle.ACT_SILU,
                                out_dtype=TORCH_TO_ORC[out_dt], want_absacc=True)
     check_tolerance(got, ref, acc, out_dt, what=f"fp8 out={out_dt} bias={bias_dt}")
+
+
+# ------------------------------------------------------------------ seeded random sweep
+
+def _fp8_sweep(n=24, seed=4242):
+    rs = np.random.RandomState(seed)
+    cases = []
+    for i in range(n):
+        cases.append(dict(M=int(rs.choice([int(rs.randint(1, 65)), int(rs.randint(65, 600))])),
+                          N=int(rs.randint(1, 600)), K=16 * int(rs.randint(1, 64)),
+                          pair=["1", "0"][rs.randint(2)], sched=["auto", "dp", "sk"][rs.randint(3)],
+                          act=["none", "gelu_tanh", "silu"][rs.randint(3)], bias=bool(rs.randint(2)),
+                          seed=500 + i))
+    return cases
+
+
+@pytest.mark.parametrize("case", _fp8_sweep(), ids=lambda c: "M{M}N{N}K{K}".format(**c))
+def test_fp8_seeded_random_sweep(cuda_device, monkeypatch, case):
+    """Random shapes (K any multiple of 16, so partial last scale groups are common),
+    kernels, schedules, bias and activation: both quantisations on the GPU equal the
+    oracle's bit for bit, and the block-scaled GEMM on those codes meets the contract."""
+    monkeypatch.setenv("SMGEMM_PAIR", case["pair"])
+    monkeypatch.setenv("SMGEMM_SCHED", case["sched"])
+    M, N, K, s = case["M"], case["N"], case["K"], case["seed"]
+    A = synth.normal_with_outliers(s, 0, (M, K))
+    B = synth.normal_with_outliers(s, 1, (K, N))
+    Bd = torch.zeros((K, -(-N // 4) * 4), dtype=torch.float32, device="cuda")  # 16-byte row pitch
+    Bd[:, :N] = torch.from_numpy(B).cuda()
+    qa, sa = sg.quantize_fp8_blockwise(torch.from_numpy(A).cuda(), 1)
+    qb, sb = sg.quantize_fp8_blockwise(Bd[:, :N], 128)
+    assert sg.check() == sg.OK
+    qa_r, sa_r = oracle.quant_1x128(A)
+    qb_r, sb_r = oracle.quant_128x128(B)
+    assert np.array_equal(qa.cpu().numpy(), qa_r)
+    assert np.array_equal(sa.cpu().numpy().view(np.uint32), sa_r.view(np.uint32))
+    assert np.array_equal(qb.cpu().numpy(), qb_r)
+    assert np.array_equal(sb.cpu().numpy().view(np.uint32), sb_r.view(np.uint32))
+    bias = torch.from_numpy(synth.normal(s, 2, (N,), 0.5)).to(torch.bfloat16) if case["bias"] else None
+    out = torch.empty((M, -(-N // 8) * 8), dtype=torch.bfloat16, device="cuda")[:, :N]
+    sg.gemm_fp8_blockscaled(qa, sa, qb, sb, bias=None if bias is None else bias.cuda(), act=case["act"], out=out)
+    assert sg.check() == sg.OK
+    kw = {} if bias is None else dict(zip(("bias", "bias_dtype"), orc_view(bias)))
+    act = {"none": oracle.ACT_NONE, "gelu_tanh": oracle.ACT_GELU_TANH, "silu": oracle.ACT_SILU}[case["act"]]
+    ref, acc = oracle.gemm_fp8(qa_r, sa_r, qb_r, sb_r, act=act, out_dtype=oracle.BF16, want_absacc=True, **kw)
+    check_tolerance(out.float().cpu().numpy(), ref, acc, torch.bfloat16, what=sg.last_config())

@@ -179,3 +179,60 @@ def test_prepared_grouped_gemm_matches_one_shot_calls(cuda_device):
             assert torch.equal(got[g], want[g]), f"step {step} group {g}"
         for A in As:
             A.mul_(-0.5)                       # new contents, same storage
+
+
+def _grouped_sweep(n=12, seed=77):
+    rs = np.random.RandomState(seed)
+    cases = []
+    for i in range(n):
+        G = int(rs.randint(1, 13))
+        shapes = [(int(rs.choice([0, int(rs.randint(1, 65)), int(rs.randint(65, 600))], p=[0.1, 0.3, 0.6])),
+                   8 * int(rs.randint(1, 66)), 8 * int(rs.randint(0, 80))) for _ in range(G)]
+        cases.append(dict(shapes=shapes, la=["row", "col"][rs.randint(2)], lb=["row", "col"][rs.randint(2)],
+                          integer=bool(rs.randint(2)), act=["none", "gelu_tanh", "silu"][rs.randint(3)],
+                          sched_split=["1", "0"][rs.randint(2)], seed=300 + i))
+    return cases
+
+
+@pytest.mark.parametrize("case", _grouped_sweep(), ids=lambda c: "G{}".format(len(c["shapes"])))
+def test_grouped_seeded_random_sweep(cuda_device, monkeypatch, case):
+    """Random group counts and shapes (empty groups, K = 0, one-row groups, ragged tails),
+    layouts, activations, with and without the split tail: integer inputs without an
+    activation are exact in FP32; real inputs with bias and activation meet the contract."""
+    monkeypatch.setenv("SMGEMM_SCHED_GROUPED_SPLIT", case["sched_split"])
+    exact = case["integer"]
+    act = "none" if exact else case["act"]
+    As, Bs, bs, Ah, Bh, bh = [], [], [], [], [], []
+    for g, (M, N, K) in enumerate(case["shapes"]):
+        s = case["seed"]
+        if exact:
+            a = synth.integers(s, 3 * g, (M, K), -3, 3)
+            b = synth.integers(s, 3 * g + 1, (K, N), -3, 3)
+        else:
+            a = synth.normal(s, 3 * g, (M, K))
+            b = synth.normal(s, 3 * g + 1, (K, N), 0.1)
+        As.append(_operand(a, case["la"]))
+        Bs.append(_operand(b, case["lb"]))
+        Ah.append(to_dtype(a, torch.bfloat16))
+        Bh.append(to_dtype(b, torch.bfloat16))
+        bias = None if exact or g % 3 == 1 else to_dtype(synth.normal(s, 3 * g + 2, (N,), 0.5), torch.bfloat16)
+        bs.append(None if bias is None else bias.cuda())
+        bh.append(bias)
+    out_dt = torch.float32 if exact else torch.bfloat16
+    outs = sg.gemm_bf16_grouped(As, Bs, biases=bs, act=act, out_dtype=out_dt)
+    assert sg.check() == sg.OK
+    orc_act = {"none": oracle.ACT_NONE, "gelu_tanh": oracle.ACT_GELU_TANH, "silu": oracle.ACT_SILU}[act]
+    for g, (M, N, K) in enumerate(case["shapes"]):
+        if M == 0 or N == 0:
+            assert outs[g].numel() == 0
+            continue
+        a, ad = orc_view(Ah[g])
+        b, bd = orc_view(Bh[g])
+        kw = {} if bh[g] is None else dict(zip(("bias", "bias_dtype"), orc_view(bh[g])))
+        ref, acc = oracle.gemm(a, b, a_dtype=ad, b_dtype=bd, act=orc_act,
+                               out_dtype=oracle.F32 if exact else oracle.BF16, want_absacc=True, **kw)
+        got = outs[g].float().cpu().numpy()
+        if exact:
+            assert np.array_equal(got, ref.astype(np.float32)), f"group {g} {M}x{N}x{K}"
+        else:
+            check_tolerance(got, ref, acc, out_dt, what=f"group {g} {M}x{N}x{K}")
