@@ -141,3 +141,27 @@ def test_apply_partials_neutral_pairs_and_empty_slice(cuda_device):
     # neutral pairs change nothing but the pairing order of the merge tree (last-bit rounding)
     assert torch.allclose(lse_pad, lse_ref, rtol=0, atol=1e-5) and torch.allclose(o, ref, rtol=0, atol=1e-5)
     assert torch.equal(lse_empty, lse_ref)
+
+
+def _ls_sweep(n=16, seed=909):
+    rs = np.random.RandomState(seed)
+    out = []
+    for i in range(n):
+        out.append(dict(M=int(rs.choice([int(rs.randint(1, 65)), int(rs.randint(65, 300))])),
+                        N=8 * int(rs.randint(1, 400)), K=8 * int(rs.randint(1, 80)), bias=bool(rs.randint(2)),
+                        sched=["auto", "dp", "sk"][rs.randint(3)], seed=700 + i))
+    return out
+
+
+@pytest.mark.parametrize("case", _ls_sweep(), ids=lambda c: "M{M}N{N}K{K}".format(**c))
+def test_logsoftmax_seeded_random_sweep(cuda_device, monkeypatch, case):
+    """Random rows (skinny and large-tile paths), vocabulary widths (not multiples of
+    the 128-column tiles), depths, bias and schedules, within the bound above."""
+    monkeypatch.setenv("SMGEMM_SCHED", case["sched"])
+    M, N, K, s = case["M"], case["N"], case["K"], case["seed"]
+    X = to_dtype(synth.normal(s, 0, (M, K)), torch.bfloat16)
+    W = to_dtype(synth.normal(s, 1, (K, N), 0.2), torch.bfloat16)
+    b = to_dtype(synth.normal(s, 2, (N,), 0.5), torch.bfloat16) if case["bias"] else None
+    out = sg.gemm_bf16_logsoftmax(X.cuda(), W.cuda(), bias=None if b is None else b.cuda())
+    assert sg.check() == sg.OK
+    _check(out, X, W, b)
