@@ -68,15 +68,17 @@ typedef enum { SMGEMM_ACT_NONE = 0, SMGEMM_ACT_GELU_TANH = 1, SMGEMM_ACT_SILU = 
  *            (row-major: ldb >= N; col-major, i.e. W^T stored [N,K]: ldb >= K).
  *   bias     device, nullable; bias_dtype SMGEMM_BF16 / SMGEMM_F16 / SMGEMM_F32; N entries.
  *   act      SMGEMM_ACT_NONE, SMGEMM_ACT_GELU_TANH (0.5x(1+tanh(sqrt(2/pi)(x+0.044715x^3))))
- *            or SMGEMM_ACT_SILU (x/(1+e^-x)); applied in FP32 after the bias add, with the
- *            hardware tanh approximation (relative error ~2^-11) and the fast exponential.
+ *            or SMGEMM_ACT_SILU (x/(1+e^-x)), applied after the bias add, both as
+ *            x*sigmoid(z) without cancellation: in FP32 for 16-bit outputs (relative error
+ *            below 2^-16), in FP64 with one rounding for FP32 outputs (within one FP32 ulp).
  *   C        device, c_dtype SMGEMM_F32 / SMGEMM_BF16 / SMGEMM_F16, row-major, ldc >= N.
  *   workspace  device scratch of at least smgemm_workspace_size(M,N,K,0) bytes,
  *            16-byte aligned (may be NULL when that size is 0). The library uses it
  *            for split-K / stream-K partial tiles and their arrival counters; its
  *            contents on entry do not matter (no zeroing needed: the counters carry a
- *            per-call generation). It must not be shared by calls that can overlap on
- *            the GPU.
+ *            per-call generation), and a completed call leaves every counter at zero, so
+ *            a call captured in a CUDA graph can be replayed on the same workspace any
+ *            number of times. It must not be shared by calls that can overlap on the GPU.
  * Small M (<= 64, row-major A) runs the memory-bound swap-AB path; everything else
  * the persistent tensor-core path. Results are deterministic run to run.
  */

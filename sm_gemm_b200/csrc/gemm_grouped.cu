@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_barrier_sync(1, kEpiThreads);
         if (epi_tid == 0) {
           const bool any_dead = *abort_flag != 0;
-          const int old = any_dead ? -1 : counter_arrive(sp.counters + r_tail * 2 + rank, sp.gen);
+          const int old = any_dead ? -1 : counter_arrive(sp.counters + r_tail * 2 + rank, sp.gen, sp.splits);
           *reduce_flag = (!any_dead && old == sp.splits - 1);
         }
         named_barrier_sync(1, kEpiThreads);

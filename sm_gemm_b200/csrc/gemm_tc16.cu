@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int n = 0;
           for (int c = c_lo; c <= c_hi; ++c) n += sk_bound(s, c) < sk_bound(s, c + 1);
           const bool any_dead = *abort_flag != 0;
-          const int old = any_dead ? -1 : counter_arrive(p.counters + t_sk, p.gen);
+          const int old = any_dead ? -1 : counter_arrive(p.counters + t_sk, p.gen, n);
           *reduce_flag = (!any_dead && old == n - 1);
         }
         named_barrier_sync(1, 128);

@@ -589,22 +589,29 @@ struct WorkIter {
   }
 };
 
-// Arrival of one contributor on a split tile's counter. A counter word holds the call's
-// generation (upper 48 bits, a number the host draws afresh for every call, never 0) and
-// the number of this call's arrivals (lower 16 bits); a word of another generation -
-// left by an earlier call, or whatever a fresh workspace holds - counts as zero arrivals.
-// So the workspace needs no zeroing before a call (the chance that a stale word carries
-// the current generation is 2^-48). Returns the number of earlier arrivals of this call,
-// or -1 if the compare-and-swap kept failing (it cannot fail more often than there are
-// contributors; the bound only keeps the loop finite).
-__device__ __forceinline__ int counter_arrive(unsigned long long* c, unsigned long long gen) {
+// Arrival of one of the n contributors to a split tile on the tile's counter. A counter
+// word holds the call's generation (upper 48 bits, a number the host draws afresh for
+// every call, never 0) and the number of this call's arrivals (lower 16 bits); a word of
+// another generation - left by an earlier call, or whatever a fresh workspace holds -
+// counts as zero arrivals. So the workspace needs no zeroing before a call (the chance
+// that a stale word carries the current generation is 2^-48). The last arrival resets the
+// word to zero: a call replayed from a CUDA graph carries the generation it was captured
+// with, and must find the counters of its previous run back at zero arrivals. Returns the
+// number of earlier arrivals of this call, or -1 if the compare-and-swap kept failing (it
+// cannot fail more often than there are contributors; the bound only keeps the loop
+// finite).
+__device__ __forceinline__ int counter_arrive(unsigned long long* c, unsigned long long gen, int n) {
   unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(c);
 #pragma unroll 1
   for (int i = 0; i < 4096; ++i) {
     const bool same = (cur >> 16) == gen;
     const unsigned long long want = same ? cur + 1ull : ((gen << 16) | 1ull);
     const unsigned long long prev = atomicCAS(c, cur, want);
-    if (prev == cur) return same ? static_cast<int>(cur & 0xffffull) : 0;
+    if (prev == cur) {
+      const int old = same ? static_cast<int>(cur & 0xffffull) : 0;
+      if (old == n - 1) atomicExch(c, 0ull);  // every contributor has arrived
+      return old;
+    }
     cur = prev;
   }
   atomicOr(&g_error_word, kErrTimeout);  // reported by smgemm_check like an abandoned wait
