@@ -126,14 +126,15 @@ smgemm_status gemm_bf16_noalloc(int64_t M, int64_t N, int64_t K,
  *   ab_dtype, layout_a, layout_b, bias_dtype, act, c_dtype: shared by all groups, as in
  *              gemm_bf16. Groups with M or N = 0 are skipped; K = 0 writes act(bias).
  *   workspace  device, 16-byte aligned (else SMGEMM_ERR_ALIGNMENT), at least
- *              smgemm_grouped_workspace_size(G) bytes: the host writes
- *              the groups' TMA descriptors and sizes there (an asynchronous copy on
- *              `stream`, from pageable memory) before the launch; the rest holds the
- *              partial tiles of a split last wave. Calls that can overlap on the GPU
+ *              smgemm_grouped_workspace_size(G) bytes: with more than 16 groups the
+ *              groups' TMA descriptors and sizes are written there before the launch (by
+ *              small kernels on `stream` that carry them as parameters, so the call can be
+ *              captured in a CUDA graph; up to 16 groups travel with the launch itself);
+ *              the rest holds the partial tiles of a split last wave. Calls that can overlap on the GPU
  *              must not share it. A smaller workspace that still holds the table is
  *              accepted; the last wave is then not split.
  * Every group is validated, and every TMA descriptor encoded, before anything is
- * enqueued; the descriptor table is copied first, then groups with K = 0 are filled,
+ * enqueued; the descriptor table is written first, then groups with K = 0 are filled,
  * then the GEMM launches. Errors as in gemm_bf16. Tiles
  * of 256 x 256 run one per CTA pair; when the tiles do not fill a whole last wave, the
  * R tiles of that wave are each split along K into S = min(P / R, KB / 8) pieces (P

@@ -834,12 +834,12 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   const int clusters_max = tiles > 0 ? grouped_max_clusters() : 0;
   if (tiles > 0 && clusters_max <= 0) return SMGEMM_ERR_CUDA;
   GroupDesc* dev_table = reinterpret_cast<GroupDesc*>((reinterpret_cast<uintptr_t>(workspace) + 63) & ~uintptr_t(63));
-  // Pageable source: the copy has consumed `table` by the time the call returns. It is
-  // the first thing enqueued, so a failure here leaves every output untouched.
-  if (!inline_table && tiles > 0 &&
-      cudaMemcpyAsync(dev_table, table, static_cast<size_t>(G) * sizeof(GroupDesc), cudaMemcpyHostToDevice,
-                      stream) != cudaSuccess)
-    return launch_status(cudaGetLastError());
+  // The table goes with small kernels' parameters (captured by value in a CUDA graph);
+  // it is the first thing enqueued, so a failure here leaves every output untouched.
+  if (!inline_table && tiles > 0) {
+    const smgemm_status st = launch_status(launch_upload_group_table(table, G, dev_table, stream));
+    if (st != SMGEMM_OK) return st;
+  }
   for (int g : fills) {
     const GroupDesc& e = table[g];
     smgemm_status st =

@@ -23,6 +23,7 @@
 // tiles are split along K into S pieces (R S <= P) that run side by side; each piece's
 // partial goes to a workspace slot and the last piece to finish sums them in order.
 #include <cuda_bf16.h>
+#include <cstring>
 #include <type_traits>
 #include <cuda_fp16.h>
 
@@ -391,6 +392,40 @@ cudaError_t launch_gemm_grouped_split(const GroupedParams& p, const GroupedSplit
   else e = cudaLaunchKernelEx(&cfg, gemm_grouped_kernel<kBK, kStages, false>, p, sp, NoInlineTable{});
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+namespace {
+// More than kInlineGroups records reach the workspace through kernels whose parameters
+// carry up to kUploadGroups records each (within the 32 KB a launch's parameters may
+// hold): the table travels by value with the launch, so a call captured in a CUDA graph
+// replays it, where a copy from the caller's pageable host memory would be read again at
+// every replay from memory freed after the call.
+constexpr int kUploadGroups = 96;
+struct GroupTableChunk {
+  GroupDesc d[kUploadGroups];
+};
+static_assert(sizeof(GroupTableChunk) <= 32000, "kernel parameter budget");
+
+__global__ void __launch_bounds__(256) upload_group_table_kernel(const __grid_constant__ GroupTableChunk c, int count,
+                                                                 GroupDesc* __restrict__ dst) {
+  const uint4* src = reinterpret_cast<const uint4*>(&c);
+  uint4* out = reinterpret_cast<uint4*>(dst);
+  const int words = count * static_cast<int>(sizeof(GroupDesc) / sizeof(uint4));
+  for (int i = static_cast<int>(threadIdx.x); i < words; i += static_cast<int>(blockDim.x)) out[i] = src[i];
+}
+}  // namespace
+
+cudaError_t launch_upload_group_table(const GroupDesc* table, int G, GroupDesc* dst, cudaStream_t stream) {
+  static_assert(sizeof(GroupDesc) % sizeof(uint4) == 0, "records are whole 16-byte words");
+  for (int first = 0; first < G; first += kUploadGroups) {
+    const int count = G - first < kUploadGroups ? G - first : kUploadGroups;
+    GroupTableChunk c;
+    std::memcpy(c.d, table + first, static_cast<size_t>(count) * sizeof(GroupDesc));
+    upload_group_table_kernel<<<1, 256, 0, stream>>>(c, count, dst + first);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_gemm_grouped(const GroupedParams& p, int clusters, cudaStream_t stream) {

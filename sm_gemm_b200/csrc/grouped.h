@@ -23,6 +23,10 @@ struct GroupTableInline {
   GroupDesc d[kInlineGroups];
 };
 
+// Writes G records to dst (device, 64-byte aligned) on `stream` through kernels whose
+// parameters carry the records (no host-memory copy: graph-capturable).
+cudaError_t launch_upload_group_table(const GroupDesc* table, int G, GroupDesc* dst, cudaStream_t stream);
+
 // `inl` (nullable): the table as a kernel parameter (G <= kInlineGroups); else p.groups.
 cudaError_t launch_gemm_grouped_split(const GroupedParams& p, const GroupedSplit& sp, const GroupTableInline* inl,
                                       int clusters, cudaStream_t stream);

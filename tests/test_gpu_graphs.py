@@ -122,3 +122,17 @@ def test_graph_replay_lm_head_log_softmax(cuda_device):
                          lambda o, ws: sg.gemm_bf16_logsoftmax(X, W, out=o[0], workspace=ws),
                          lambda: [torch.empty(4, 4000, dtype=torch.float32, device="cuda")],
                          lambda: torch.empty(nws, dtype=torch.uint8, device="cuda"))
+
+
+def test_graph_replay_grouped_many_groups(cuda_device):
+    """More groups than travel with the launch itself (16): the table is written into the
+    workspace by kernels that carry it as parameters, which the graph replays."""
+    rs = np.random.RandomState(5)
+    sizes = [(int(rs.randint(1, 300)), 8 * int(rs.randint(1, 40)), 8 * int(rs.randint(1, 60))) for _ in range(40)]
+    As = [torch.empty(m, k, dtype=torch.bfloat16, device="cuda") for m, n, k in sizes]
+    Bs = [torch.empty(k, n, dtype=torch.bfloat16, device="cuda") for m, n, k in sizes]
+    nws = int(sg.lib().smgemm_grouped_workspace_size(len(sizes)))
+    _replays_match_eager(lambda s: _fill(As + Bs, s, 0.1),
+                         lambda o, ws: sg.gemm_bf16_grouped(As, Bs, outs=o, workspace=ws),
+                         lambda: [torch.empty(m, n, dtype=torch.bfloat16, device="cuda") for m, n, k in sizes],
+                         lambda: torch.empty(nws, dtype=torch.uint8, device="cuda"))
