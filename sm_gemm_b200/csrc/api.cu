@@ -798,7 +798,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   const bool b_mn = (layout_b == SMGEMM_ROW_MAJOR);
   const int bk = grouped_bk();
   // Up to kInlineGroups records are passed with the launch (no copy); more go to the
-  // workspace through one host-to-device copy.
+  // workspace (launch_upload_group_table).
   const bool inline_table = G <= kInlineGroups;
   GroupTableInline inl;
   std::vector<GroupDesc> heap;
