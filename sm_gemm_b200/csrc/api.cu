@@ -37,12 +37,12 @@ namespace {
 // environment for each of the dozen switches a GEMM call consults.
 enum Knob {
   kKnobGrid, kKnobSched, kKnobSplitK, kKnobForceConfig, kKnobPair, kKnobForceLarge, kKnobGroupM, kKnobFp8Tn,
-  kKnobLog, kKnobWaitLimitNs, kKnobEpiStore, kKnobGroupedSplit, kKnobPdl, kNumKnobs
+  kKnobLog, kKnobWaitLimitNs, kKnobEpiStore, kKnobGroupedSplit, kKnobPdl, kKnobGroupedTranspose, kNumKnobs
 };
 const char* const kKnobNames[kNumKnobs] = {
     "SMGEMM_GRID", "SMGEMM_SCHED", "SMGEMM_SPLITK", "SMGEMM_FORCE_CONFIG", "SMGEMM_PAIR", "SMGEMM_FORCE_LARGE",
     "SMGEMM_GROUP_M", "SMGEMM_FP8_TN", "SMGEMM_LOG", "SMGEMM_WAIT_LIMIT_NS", "SMGEMM_EPI_STORE",
-    "SMGEMM_SCHED_GROUPED_SPLIT", "SMGEMM_PDL"};
+    "SMGEMM_SCHED_GROUPED_SPLIT", "SMGEMM_PDL", "SMGEMM_GROUPED_TRANSPOSE"};
 thread_local const char* g_knobs[kNumKnobs] = {};
 
 void refresh_knobs() {
@@ -805,7 +805,8 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   if (!inline_table) heap.resize(static_cast<size_t>(G));
   GroupDesc* table = inline_table ? inl.d : heap.data();
   std::vector<int> fills;  // groups with K = 0: filled with act(bias) after the table is enqueued
-  long long tiles = 0;
+  long long tiles = 0, t_tiles = 0;
+  const bool transpose_rem = env_ll(kKnobGroupedTranspose, 1) != 0;
   for (int g = 0; g < G; ++g) {
     GroupDesc& e = table[g];
     std::memset(&e, 0, sizeof(e));
@@ -821,15 +822,19 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
       continue;
     }
     bool ok;
+    // A's boxes are 64 rows (K-major): a normal tile loads two per K slice, the B slot
+    // of a transposed remainder tile one.
     if (a_mn) ok = encode_2d(&e.tm_a, dt, A[g], M[g], K[g], lda[g] * 2, 64, bk);
-    else ok = encode_2d(&e.tm_a, dt, A[g], K[g], M[g], lda[g] * 2, 64, 128);
+    else ok = encode_2d(&e.tm_a, dt, A[g], K[g], M[g], lda[g] * 2, 64, 64);
     if (b_mn) ok = ok && encode_2d(&e.tm_b, dt, B[g], N[g], K[g], ldb[g] * 2, 64, bk);
     else ok = ok && encode_2d(&e.tm_b, dt, B[g], K[g], N[g], ldb[g] * 2, 64, 128);
     if (!ok) return SMGEMM_ERR_CUDA;
     e.m_tiles = static_cast<int>((M[g] + 255) / 256);
     e.n_tiles = static_cast<int>((N[g] + 255) / 256);
     e.kb_total = static_cast<int>((K[g] + bk - 1) / bk);
+    e.rem_t = transpose_rem && M[g] - static_cast<int64_t>(e.m_tiles - 1) * 256 <= 128 ? 1 : 0;
     tiles += static_cast<long long>(e.m_tiles) * e.n_tiles;
+    if (e.rem_t) t_tiles += e.n_tiles;
   }
   const int clusters_max = tiles > 0 ? grouped_max_clusters() : 0;
   if (tiles > 0 && clusters_max <= 0) return SMGEMM_ERR_CUDA;
@@ -858,6 +863,7 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   p.a_mn_major = a_mn ? 1 : 0;
   p.b_mn_major = b_mn ? 1 : 0;
   p.idesc = idesc_f32acc(fmt, fmt, a_mn ? 1u : 0u, b_mn ? 1u : 0u, 256, 256);
+  p.idesc_t = idesc_f32acc(fmt, fmt, b_mn ? 1u : 0u, a_mn ? 1u : 0u, 256, 128);
   p.wait_limit_cycles = wait_limit();
   // A ragged last wave (R = tiles mod P tiles for P co-resident clusters; all tiles when
   // there are fewer than P) is split along K into S pieces when every tail tile keeps at
@@ -891,8 +897,8 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
     sp.gen = next_generation();
   }
   std::snprintf(config_text(), sizeof(g_last_config),
-                "path=grouped groups=%d tiles=%lld grid=%d tile=128x256 split_tiles=%lld splits=%d", G, tiles, clusters,
-                S >= 2 ? R : 0LL, S >= 2 ? S : 0);
+                "path=grouped groups=%d tiles=%lld transposed_tiles=%lld grid=%d tile=128x256 split_tiles=%lld splits=%d",
+                G, tiles, t_tiles, clusters, S >= 2 ? R : 0LL, S >= 2 ? S : 0);
   if (env_ll(kKnobLog, 0)) std::fprintf(stderr, "[smgemm] %s\n", g_last_config);
   return launch_status(launch_gemm_grouped_split(p, sp, inline_table ? &inl : nullptr, clusters, stream));
 }

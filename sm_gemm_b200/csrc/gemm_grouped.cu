@@ -18,10 +18,20 @@
 // Roles as in gemm_tc16_pair.cu: warp 0 TMA producer and warp 1 MMA issuer (warp-wide
 // loops, one elected lane issues; MMA on the rank-0 CTA only), warp 2 TMEM allocator,
 // warps 4-11 epilogue (each CTA drains its own 128 rows of the two TMEM accumulators;
-// warp w takes lanes 32*(w%4).. and the 128 columns 128*((w-4)/4).. of the tile).
+// warp w takes lanes 32*(w%4).. and the 128 columns 128*((w-4)/4).. of the tile, or the
+// 64 columns 64*((w-4)/4).. of a transposed tile).
 // When the tiles leave a ragged last wave (R = T mod P tiles for P clusters), those R
 // tiles are split along K into S pieces (R S <= P) that run side by side; each piece's
 // partial goes to a workspace slot and the last piece to finish sums them in order.
+//
+// A group whose last row of tiles holds at most 128 rows (M mod 256 in 1..128) would
+// leave half of each of those 256-row tiles empty. Those tiles run transposed instead:
+// the pair computes the 256 x 128 tile of C^T = B^T A^T, with 256 columns of B as the
+// MMA's M (128 per CTA, the same load as B's half of a normal tile) and the up to 128
+// remaining rows of A as its N (64 per CTA), and the epilogue writes each TMEM lane (one
+// column of C) down the rows. Half the tensor-core work of the padded tile; the MMA then
+// reads shared memory faster than at N = 256 per unit of work, but still needs fewer
+// cycles per tile than the half-empty one.
 #include <cuda_bf16.h>
 #include <cstring>
 #include <type_traits>
@@ -73,6 +83,7 @@ __device__ __forceinline__ int locate(const GroupedParams& p, long long t, int& 
 struct GItem {
   long long tile;
   int g, mt, nt, kb0, kb1, unit;
+  bool tr;  // transposed remainder tile (C^T = B^T A^T, <= 128 rows of A)
 };
 
 // Work of cluster c: its piece of the split tail (if any) first, so the tail's fix-up
@@ -99,6 +110,7 @@ struct GIter {
       it.kb0 = static_cast<int>(static_cast<long long>(piece) * kbn / sp.splits);
       it.kb1 = static_cast<int>(static_cast<long long>(piece + 1) * kbn / sp.splits);
       it.unit = c;
+      it.tr = p.groups[it.g].rem_t != 0 && it.mt == p.groups[it.g].m_tiles - 1;
       return true;
     }
     if (next_dp < p.total_tiles - sp.split_tiles) {
@@ -107,6 +119,7 @@ struct GIter {
       it.kb0 = 0;
       it.kb1 = p.groups[it.g].kb_total;
       it.unit = -1;
+      it.tr = p.groups[it.g].rem_t != 0 && it.mt == p.groups[it.g].m_tiles - 1;
       next_dp += P;
       return true;
     }
@@ -190,17 +203,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tensormap_acquire(&d->tm_b);
       }
       last_g = it.g;
-      const int a_row = it.mt * 256 + static_cast<int>(rank) * 128;
+      // Normal tile: 128 rows of A and 128 columns of B per CTA. Transposed tile: the
+      // same 128 columns of B in the A slot and 64 rows of A in the B slot.
+      const int a_row = it.mt * 256 + static_cast<int>(rank) * (it.tr ? 64 : 128);
       const int b_row = it.nt * kTileN + static_cast<int>(rank) * 128;
+      const uint32_t tx_bytes = it.tr ? 2 * (A_BYTES + B_BYTES / 2) : 2 * STAGE_BYTES;
       for (int kb = it.kb0; kb < it.kb1; ++kb) {
         const bool w = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         const uint32_t sa = smem_base + stage * STAGE_BYTES;
         const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
         if (elect_one()) {
-          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-          load_operand_pair<128, BK>(sa, &d->tm_a, leader_full, p.a_mn_major, a_row, kb * BK);
-          load_operand_pair<128, BK>(sa + A_BYTES, &d->tm_b, leader_full, p.b_mn_major, b_row, kb * BK);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), tx_bytes);
+          if (!it.tr) {
+            load_operand_pair_r64<128, BK>(sa, &d->tm_a, leader_full, p.a_mn_major, a_row, kb * BK);
+            load_operand_pair<128, BK>(sa + A_BYTES, &d->tm_b, leader_full, p.b_mn_major, b_row, kb * BK);
+          } else {
+            load_operand_pair<128, BK>(sa, &d->tm_b, leader_full, p.b_mn_major, b_row, kb * BK);
+            load_operand_pair_r64<64, BK>(sa + A_BYTES, &d->tm_a, leader_full, p.a_mn_major, a_row, kb * BK);
+          }
         }
         __syncwarp();
         ++issued;
@@ -231,6 +252,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, limit))) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * kTileN;
+      // Transposed tile: B's columns are the MMA's A operand and A's rows its B operand
+      // (64 rows per CTA; for BK = 64 the slice descriptors of a 64- and a 128-row tile
+      // coincide, so only the major-ness flags and the instruction descriptor change).
+      static_assert(BK == 64, "64-row operand tiles share the 128-row slice descriptors");
+      const int amn = it.tr ? p.b_mn_major : p.a_mn_major;
+      const int bmn = it.tr ? p.a_mn_major : p.b_mn_major;
+      const uint32_t idesc = it.tr ? p.idesc_t : p.idesc;
       for (int kb = it.kb0; kb < it.kb1; ++kb) {
         if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, abort_flag, limit))) { ok = false; break; }
         tc_fence_after();
@@ -239,8 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (elect_one()) {
 #pragma unroll
           for (int k = 0; k < KSTEPS; ++k) {
-            umma_f16_pair(d_tmem, operand_desc<128, BK>(sa, p.a_mn_major, k),
-                          operand_desc<128, BK>(sb, p.b_mn_major, k), p.idesc, (kb > it.kb0 || k > 0) ? 1u : 0u);
+            umma_f16_pair(d_tmem, operand_desc<128, BK>(sa, amn, k), operand_desc<128, BK>(sb, bmn, k), idesc,
+                          (kb > it.kb0 || k > 0) ? 1u : 0u);
           }
           umma_commit_pair(empty_bar(stage), 0x3);
         }
@@ -262,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r_local = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     const int epi_tid = threadIdx.x - kEpiWarp0 * 32;
-    const int c_base = ((warp - kEpiWarp0) >> 2) * kEpiCols;  // this warp's first tile column
+    const int cg = (warp - kEpiWarp0) >> 2;  // which half of the tile's columns
     int local = 0;
     bool dead = false;
     GIter wi;
@@ -275,15 +303,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!dead) dead = !mbar_wait(tfull_bar(acc), acc_phase, abort_flag, limit);
       dead = __any_sync(0xffffffffu, dead);
-      const int row = it.mt * 256 + static_cast<int>(rank) * 128 + r_local;
+      // Normal tile: this thread owns row `fixed` of C from column `run0` on (128 tile
+      // columns per warp); transposed tile: column `fixed` of C (its TMEM lane) from row
+      // `run0` down (64 tile columns, i.e. rows of C, per warp).
+      const int cols = it.tr ? kEpiCols / 2 : kEpiCols;
+      const int c_base = cg * cols;
+      const int fixed = (it.tr ? it.nt * kTileN : it.mt * 256) + static_cast<int>(rank) * 128 + r_local;
+      const int run0 = (it.tr ? it.mt * 256 : it.nt * kTileN) + c_base;
+      auto emit = [&](int c, float(&v)[32]) {
+        if (it.tr) epi_col<32>(e, fixed, run0 + c * 32, v);
+        else epi_row32(e, fixed, run0 + c * 32, v);
+      };
       const uint32_t tacc = tmem_base + lane_addr + acc * kTileN + c_base;
-      const int col0 = it.nt * kTileN + c_base;
       const bool split = it.unit >= 0;
       float* my_slot = split ? sp.slots + (static_cast<size_t>(it.unit) * 2 + rank) * SLOT : nullptr;
       if (!dead) {
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < kEpiCols / 32; ++c) {
+        for (int c = 0; c < cols / 32; ++c) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tacc + c * 32, r);
           tmem_ld_wait();
@@ -291,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
           if (split) slot_store<32>(my_slot, r_local, c_base + c * 32, v);
-          else epi_row32(e, row, col0 + c * 32, v);
+          else emit(c, v);
         }
         tc_fence_before();
         __syncwarp();
@@ -312,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*reduce_flag) {
           __threadfence();
 #pragma unroll 1
-          for (int c = 0; c < kEpiCols / 32; ++c) {
+          for (int c = 0; c < cols / 32; ++c) {
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.0f;
@@ -321,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float* src = sp.slots + ((r_tail * sp.splits + pc) * 2 + rank) * static_cast<size_t>(SLOT);
               slot_accumulate<32>(src, r_local, c_base + c * 32, v);
             }
-            epi_row32(e, row, col0 + c * 32, v);
+            emit(c, v);
           }
         }
         named_barrier_sync(1, kEpiThreads);

@@ -63,9 +63,10 @@ cudaError_t launch_lse_tile_partials(const float* C, long long ldc, int M, int N
 // aligned (the TMA descriptors must be). tile0 = index of the group's first tile in the
 // launch's tile order; groups with no tiles share their successor's tile0.
 struct alignas(64) GroupDesc {
-  CUtensorMap tm_a, tm_b;   // A tiles 128 rows x BK, B tiles 128 columns x BK (per CTA)
+  CUtensorMap tm_a, tm_b;   // A: boxes of 64 rows (K-major) or 64 M x BK; B: 128 columns x BK
   long long tile0;
-  int M, N, kb_total, m_tiles, n_tiles, pad0;
+  int M, N, kb_total, m_tiles, n_tiles;
+  int rem_t;                // 1: the last row of tiles (<= 128 rows) runs transposed
   const void* bias;         // nullable
   void* C;
   long long ldc;
@@ -80,6 +81,7 @@ struct GroupedParams {
   int bias_dtype, act, c_dtype;
   int a_mn_major, b_mn_major;
   uint32_t idesc;
+  uint32_t idesc_t;         // transposed remainder tiles: M = 256 (B columns), N = 128 (A rows)
   unsigned long long wait_limit_cycles;
 };
 

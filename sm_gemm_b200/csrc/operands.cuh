@@ -40,6 +40,25 @@ __device__ __forceinline__ void load_operand_pair(uint32_t dst, const CUtensorMa
   }
 }
 
+// The same tile from a map whose K-major box is {64 (K), 64 (rows)}: R/64 boxes per
+// 64-element K slice, stacked 64 * 128 bytes apart (the layout of one R-row box, since
+// each box starts on a 1 KB swizzle atom). The MN-major box is 64 rows wide already.
+template <int R, int BK>
+__device__ __forceinline__ void load_operand_pair_r64(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                      int mn_major, int r0, int k0) {
+  static_assert(R % 64 == 0, "whole 64-row boxes");
+  if (!mn_major) {
+#pragma unroll
+    for (int j = 0; j < BK / 64; ++j)
+#pragma unroll
+      for (int h = 0; h < R / 64; ++h)
+        tma_load_2d_pair(dst + j * R * 128 + h * 64 * 128, map, bar_cluster, k0 + 64 * j, r0 + 64 * h);
+  } else {
+#pragma unroll
+    for (int j = 0; j < R / 64; ++j) tma_load_2d_pair(dst + j * BK * 128, map, bar_cluster, r0 + 64 * j, k0);
+  }
+}
+
 // Descriptor of the i-th 16-element K slice of an operand tile laid out by load_operand.
 template <int R, int BK>
 __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int mn_major, int i) {

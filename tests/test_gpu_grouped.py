@@ -32,8 +32,12 @@ def _operand(x, layout):
     return buf.cuda()[:, :rows].t()
 
 
+@pytest.mark.parametrize("transpose", ["1", "0"])
 @pytest.mark.parametrize("la,lb", [("row", "row"), ("row", "col"), ("col", "row"), ("col", "col")])
-def test_grouped_ragged_all_layouts(cuda_device, la, lb):
+def test_grouped_ragged_all_layouts(cuda_device, monkeypatch, la, lb, transpose):
+    """Ragged groups in every layout pair, with a group's last row of tiles (<= 128 rows)
+    run transposed (the default) or padded to 256 rows."""
+    monkeypatch.setenv("SMGEMM_GROUPED_TRANSPOSE", transpose)
     As, Bs, bs, Ah, Bh, bh = [], [], [], [], [], []
     for g, (M, N, K) in enumerate(SHAPES):
         a = synth.normal(41, 3 * g, (M, K))
@@ -59,8 +63,10 @@ def test_grouped_ragged_all_layouts(cuda_device, la, lb):
         check_tolerance(outs[g].float().cpu().numpy(), ref, acc, torch.bfloat16, what=f"group {g} {M}x{N}x{K}")
 
 
-def test_grouped_integer_exact_and_deterministic(cuda_device):
-    shapes = [(200, 136, 264), (512, 384, 128), (33, 520, 64)]
+@pytest.mark.parametrize("transpose", ["1", "0"])
+def test_grouped_integer_exact_and_deterministic(cuda_device, monkeypatch, transpose):
+    monkeypatch.setenv("SMGEMM_GROUPED_TRANSPOSE", transpose)
+    shapes = [(200, 136, 264), (512, 384, 128), (33, 520, 64), (384, 264, 200)]
     As, Bs, refs = [], [], []
     for g, (M, N, K) in enumerate(shapes):
         a = torch.from_numpy(synth.integers(42, 2 * g, (M, K), -3, 3)).to(torch.bfloat16)
@@ -190,7 +196,8 @@ def _grouped_sweep(n=12, seed=77):
                    8 * int(rs.randint(1, 66)), 8 * int(rs.randint(0, 80))) for _ in range(G)]
         cases.append(dict(shapes=shapes, la=["row", "col"][rs.randint(2)], lb=["row", "col"][rs.randint(2)],
                           integer=bool(rs.randint(2)), act=["none", "gelu_tanh", "silu"][rs.randint(3)],
-                          sched_split=["1", "0"][rs.randint(2)], seed=300 + i))
+                          sched_split=["1", "0"][rs.randint(2)], seed=300 + i,
+                          transpose="0" if i % 4 == 3 else "1"))
     return cases
 
 
@@ -200,6 +207,7 @@ def test_grouped_seeded_random_sweep(cuda_device, monkeypatch, case):
     layouts, activations, with and without the split tail: integer inputs without an
     activation are exact in FP32; real inputs with bias and activation meet the contract."""
     monkeypatch.setenv("SMGEMM_SCHED_GROUPED_SPLIT", case["sched_split"])
+    monkeypatch.setenv("SMGEMM_GROUPED_TRANSPOSE", case["transpose"])
     exact = case["integer"]
     act = "none" if exact else case["act"]
     As, Bs, bs, Ah, Bh, bh = [], [], [], [], [], []
@@ -236,3 +244,51 @@ def test_grouped_seeded_random_sweep(cuda_device, monkeypatch, case):
             assert np.array_equal(got, ref.astype(np.float32)), f"group {g} {M}x{N}x{K}"
         else:
             check_tolerance(got, ref, acc, out_dt, what=f"group {g} {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("la,lb", [("row", "row"), ("row", "col"), ("col", "row"), ("col", "col")])
+def test_grouped_transposed_remainder_tiles(cuda_device, monkeypatch, la, lb):
+    """Groups whose last row of tiles holds 1..128 rows run that row transposed (C^T =
+    B^T A^T, the rows of A as the MMA's N): on integer inputs the result equals the padded
+    tiles' and the oracle's bit for bit, also where those tiles are split along K; with
+    bias and activation into FP32 and FP16 outputs it meets the contract."""
+    shapes = [(1, 264, 136), (128, 256, 64), (129, 520, 200), (300, 40, 72), (384, 256, 4096), (640, 136, 64)]
+    As, Bs, Ah, Bh, refs = [], [], [], [], []
+    for g, (M, N, K) in enumerate(shapes):
+        a = synth.integers(45, 2 * g, (M, K), -3, 3)
+        b = synth.integers(45, 2 * g + 1, (K, N), -3, 3)
+        As.append(_operand(a, la)); Bs.append(_operand(b, lb))
+        Ah.append(to_dtype(a, torch.bfloat16)); Bh.append(to_dtype(b, torch.bfloat16))
+        av, ad = orc_view(Ah[g]); bv, bd = orc_view(Bh[g])
+        refs.append(oracle.gemm(av, bv, a_dtype=ad, b_dtype=bd, out_dtype=oracle.F32))
+    got = {}
+    for t in ("1", "0"):
+        monkeypatch.setenv("SMGEMM_GROUPED_TRANSPOSE", t)
+        got[t] = sg.gemm_bf16_grouped(As, Bs, out_dtype=torch.float32)
+        cfg = sg.last_config()
+        assert sg.check() == sg.OK
+        assert ("transposed_tiles=0" in cfg) == (t == "0"), cfg
+    for g in range(len(shapes)):
+        assert np.array_equal(got["1"][g].cpu().numpy(), refs[g].astype(np.float32)), f"group {g}"
+        assert torch.equal(got["1"][g], got["0"][g])
+    monkeypatch.setenv("SMGEMM_GROUPED_TRANSPOSE", "1")
+    for out_dt, act, bias_dt in ((torch.float32, "silu", torch.float32), (torch.float16, "gelu_tanh", torch.float16)):
+        reals_a, reals_b, biases, hb = [], [], [], []
+        for g, (M, N, K) in enumerate(shapes):
+            a = to_dtype(synth.normal(46, 3 * g, (M, K)), torch.bfloat16)
+            b = to_dtype(synth.normal(46, 3 * g + 1, (K, N), 0.05), torch.bfloat16)
+            bias = to_dtype(synth.normal(46, 3 * g + 2, (N,), 0.5), bias_dt)
+            reals_a.append(a); reals_b.append(b); hb.append(bias)
+            biases.append(bias.cuda())
+        outs = sg.gemm_bf16_grouped([_operand(a.float().numpy(), la) for a in reals_a],
+                                    [_operand(b.float().numpy(), lb) for b in reals_b],
+                                    biases=biases, act=act, out_dtype=out_dt)
+        assert sg.check() == sg.OK
+        orc_act = oracle.ACT_SILU if act == "silu" else oracle.ACT_GELU_TANH
+        orc_out = oracle.F32 if out_dt == torch.float32 else oracle.F16
+        for g, (M, N, K) in enumerate(shapes):
+            av, ad = orc_view(reals_a[g]); bv, bd = orc_view(reals_b[g])
+            kw = dict(zip(("bias", "bias_dtype"), orc_view(hb[g])))
+            ref, acc = oracle.gemm(av, bv, a_dtype=ad, b_dtype=bd, act=orc_act, out_dtype=orc_out, want_absacc=True,
+                                   **kw)
+            check_tolerance(outs[g].float().cpu().numpy(), ref, acc, out_dt, what=f"{out_dt} group {g} {M}x{N}x{K}")
