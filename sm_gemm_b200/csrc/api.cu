@@ -37,12 +37,13 @@ namespace {
 // environment for each of the dozen switches a GEMM call consults.
 enum Knob {
   kKnobGrid, kKnobSched, kKnobSplitK, kKnobForceConfig, kKnobPair, kKnobForceLarge, kKnobGroupM, kKnobFp8Tn,
-  kKnobLog, kKnobWaitLimitNs, kKnobEpiStore, kKnobGroupedSplit, kKnobPdl, kKnobGroupedTranspose, kNumKnobs
+  kKnobLog, kKnobWaitLimitNs, kKnobEpiStore, kKnobGroupedSplit, kKnobPdl, kKnobGroupedTranspose, kKnobGroupedOrder,
+  kNumKnobs
 };
 const char* const kKnobNames[kNumKnobs] = {
     "SMGEMM_GRID", "SMGEMM_SCHED", "SMGEMM_SPLITK", "SMGEMM_FORCE_CONFIG", "SMGEMM_PAIR", "SMGEMM_FORCE_LARGE",
     "SMGEMM_GROUP_M", "SMGEMM_FP8_TN", "SMGEMM_LOG", "SMGEMM_WAIT_LIMIT_NS", "SMGEMM_EPI_STORE",
-    "SMGEMM_SCHED_GROUPED_SPLIT", "SMGEMM_PDL", "SMGEMM_GROUPED_TRANSPOSE"};
+    "SMGEMM_SCHED_GROUPED_SPLIT", "SMGEMM_PDL", "SMGEMM_GROUPED_TRANSPOSE", "SMGEMM_GROUPED_ORDER"};
 thread_local const char* g_knobs[kNumKnobs] = {};
 
 void refresh_knobs() {
@@ -807,8 +808,31 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   std::vector<int> fills;  // groups with K = 0: filled with act(bias) after the table is enqueued
   long long tiles = 0, t_tiles = 0;
   const bool transpose_rem = env_ll(kKnobGroupedTranspose, 1) != 0;
-  for (int g = 0; g < G; ++g) {
-    GroupDesc& e = table[g];
+  // Order of the groups in the table, and so in the tile numbering: by default the
+  // groups with the most work (M N K) first, so that the last, ragged wave holds the
+  // smallest groups' tiles (measured on mixed expert sizes: 1-1.3% faster than the order
+  // given; SMGEMM_GROUPED_ORDER=0 keeps the given order, 2 alternates largest and
+  // smallest). Results do not depend on the order: each tile is computed whole or
+  // summed in K order.
+  std::vector<int> perm(static_cast<size_t>(G));
+  for (int g = 0; g < G; ++g) perm[static_cast<size_t>(g)] = g;
+  const long long order = env_ll(kKnobGroupedOrder, 1);
+  if (order == 1 || order == 2) {
+    auto work = [&](int g) { return M[g] * N[g] * K[g]; };
+    std::stable_sort(perm.begin(), perm.end(), [&](int x, int y) { return work(x) > work(y); });
+    if (order == 2) {  // largest, smallest, second largest, second smallest, ...
+      std::vector<int> z;
+      z.reserve(perm.size());
+      for (size_t lo = 0, hi = perm.size(); lo < hi;) {
+        z.push_back(perm[lo++]);
+        if (lo < hi) z.push_back(perm[--hi]);
+      }
+      perm.swap(z);
+    }
+  }
+  for (int i = 0; i < G; ++i) {
+    const int g = perm[static_cast<size_t>(i)];
+    GroupDesc& e = table[i];
     std::memset(&e, 0, sizeof(e));
     e.tile0 = tiles;
     e.M = static_cast<int>(M[g]);
@@ -846,11 +870,12 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
     if (st != SMGEMM_OK) return st;
   }
   for (int g : fills) {
-    const GroupDesc& e = table[g];
-    smgemm_status st =
-        launch_status(launch_fill_epilogue(e.M, e.N, e.bias, bias_dtype, act, C[g], c_dtype, ldc[g], stream));
+    smgemm_status st = launch_status(launch_fill_epilogue(static_cast<int>(M[g]), static_cast<int>(N[g]),
+                                                          bias != nullptr ? bias[g] : nullptr, bias_dtype, act, C[g],
+                                                          c_dtype, ldc[g], stream));
     if (st != SMGEMM_OK) return st;
   }
+
   if (tiles == 0) return SMGEMM_OK;
   GroupedParams p{};
   p.groups = dev_table;

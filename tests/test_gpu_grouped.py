@@ -292,3 +292,28 @@ def test_grouped_transposed_remainder_tiles(cuda_device, monkeypatch, la, lb):
             ref, acc = oracle.gemm(av, bv, a_dtype=ad, b_dtype=bd, act=orc_act, out_dtype=orc_out, want_absacc=True,
                                    **kw)
             check_tolerance(outs[g].float().cpu().numpy(), ref, acc, out_dt, what=f"{out_dt} group {g} {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("order", ["0", "1", "2"])
+def test_grouped_table_orders_give_identical_results(cuda_device, monkeypatch, order):
+    """The groups' order inside the launch (given, largest work first, or alternating
+    largest and smallest) changes only which cluster computes which tile: integer inputs
+    give the oracle's values bit for bit under every order, including a K = 0 group, an
+    empty group and a split last wave."""
+    monkeypatch.setenv("SMGEMM_GROUPED_ORDER", order)
+    shapes = [(128, 512, 256), (700, 264, 4096), (0, 64, 64), (33, 1000, 200), (300, 136, 0), (512, 256, 1024),
+              (1, 8, 16)]
+    As, Bs, refs = [], [], []
+    for g, (M, N, K) in enumerate(shapes):
+        a = torch.from_numpy(synth.integers(47, 2 * g, (M, K), -3, 3)).to(torch.bfloat16)
+        b = torch.from_numpy(synth.integers(47, 2 * g + 1, (K, N), -3, 3)).to(torch.bfloat16)
+        As.append(a.cuda()); Bs.append(b.cuda())
+        av, ad = orc_view(a); bv, bd = orc_view(b)
+        refs.append(oracle.gemm(av, bv, a_dtype=ad, b_dtype=bd, out_dtype=oracle.F32))
+    outs = sg.gemm_bf16_grouped(As, Bs, out_dtype=torch.float32)
+    assert sg.check() == sg.OK
+    for g, (M, N, K) in enumerate(shapes):
+        if M == 0:
+            assert outs[g].numel() == 0
+            continue
+        assert np.array_equal(outs[g].cpu().numpy(), refs[g].astype(np.float32)), f"group {g} {M}x{N}x{K}"
