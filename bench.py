@@ -177,6 +177,38 @@ def time_steps(torch, step, warmup: int, steps: int, dist=None):
     return max_over_ranks(s.elapsed_time(e), dist)
 
 
+def graph_us_per_call(torch, step, calls: int, replays: int = 3) -> float:
+    """Device time per call (us) of `calls` consecutive calls of step(i) captured in one
+    CUDA graph and replayed (best of `replays` timed replays): the calls' own device time
+    back to back, without the host's per-call cost, which paces kernels of a few
+    microseconds when a Python loop launches them one by one."""
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(0)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for i in range(calls):
+            step(i)
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(replays):
+        graph.replay()
+        torch.cuda.synchronize()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(QUEUE_AHEAD_CYCLES)
+        s.record()
+        graph.replay()
+        e.record()
+        torch.cuda.synchronize()
+        best = min(best, s.elapsed_time(e) * 1e3 / calls)
+    del graph
+    return round(best, 2)
+
+
 def per_call_us(torch, step, start: int, calls: int) -> dict:
     """Median, min and max device time (us) of `calls` further calls of step(i), each
     bracketed by its own CUDA events on the current stream (run after the timed region,
@@ -367,8 +399,13 @@ def wl_tiny_fp16(c: Ctx):
     t = c.synth.tiny_fp16()
     A, B = c.t(t["A"], torch.float16), c.t(t["B"], torch.float16)
     C = torch.empty((64, 64), dtype=torch.float32, device=c.dev)
-    ms = c.time(lambda i: sg.gemm_bf16(A, B, out=C))
-    c.record("tiny_fp16_64", ms, c.K, flops=c.metrics.gemm_flops(64, 64, 64), extra={"plan": sg.last_config()})
+    step = lambda i: sg.gemm_bf16(A, B, out=C)
+    ms = c.time(step)
+    plan = sg.last_config()
+    g_us = graph_us_per_call(torch, step, max(c.K, 20))
+    c.launches += 6 * max(c.K, 20) + 1  # warm-up call + 3 x (warm + timed) replays
+    c.record("tiny_fp16_64", ms, c.K, flops=c.metrics.gemm_flops(64, 64, 64),
+             extra={"plan": plan, "graph_us_per_call": g_us})
 
 
 def wl_ffn(c: Ctx):
@@ -458,10 +495,14 @@ def wl_fp8(c: Ctx, quant=True, gemm=True):
         Afs = [Af] + [Af.clone() for _ in range(na - 1)]
         qas = [qa] + [torch.empty_like(qa) for _ in range(na - 1)]
         sas = [sa] + [torch.empty_like(sa) for _ in range(na - 1)]
-        msa = c.time(lambda i: sg.quantize_fp8_blockwise(Afs[i % na], 1, Q=qas[i % na], scales=sas[i % na]))
+        qstep = lambda i: sg.quantize_fp8_blockwise(Afs[i % na], 1, Q=qas[i % na], scales=sas[i % na])
+        msa = c.time(qstep)
+        ga_us = graph_us_per_call(torch, qstep, max(c.K, 20))
+        c.launches += 6 * max(c.K, 20) + 1  # warm-up call + 3 x (warm + timed) replays
         del Afs, qas[1:], sas[1:]
         msb = c.time(lambda i: sg.quantize_fp8_blockwise(Bf, 128, Q=qb, scales=sb))
-        c.record("quant_1x128_A_2048x4096", msa, c.K, nbytes=m.quant_bytes(2048, 4096, 1))
+        c.record("quant_1x128_A_2048x4096", msa, c.K, nbytes=m.quant_bytes(2048, 4096, 1),
+                 extra={"graph_us_per_call": ga_us})
         c.record("quant_128x128_B_4096x16384", msb, c.K, nbytes=m.quant_bytes(4096, 16384, 128))
     else:
         sg.quantize_fp8_blockwise(Af, 1, Q=qa, scales=sa)
