@@ -326,7 +326,7 @@ def test_fp8_gemm_output_and_bias_types(cuda_device, monkeypatch, out_dt, bias_d
 
 # ------------------------------------------------------------------ seeded random sweep
 
-def _fp8_sweep(n=24, seed=4242):
+def _fp8_sweep(n=64, seed=4242):
     rs = np.random.RandomState(seed)
     cases = []
     for i in range(n):

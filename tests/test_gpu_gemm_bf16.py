@@ -398,7 +398,7 @@ def test_split_counters_need_no_zeroed_workspace(cuda_device, fill):
 
 # ------------------------------------------------------------------ seeded random sweep
 
-def _sweep_cases(n=120, seed=2024):
+def _sweep_cases(n=400, seed=2024):
     rs = np.random.RandomState(seed)
     cases = []
     for i in range(n):

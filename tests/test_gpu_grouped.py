@@ -187,7 +187,7 @@ def test_prepared_grouped_gemm_matches_one_shot_calls(cuda_device):
             A.mul_(-0.5)                       # new contents, same storage
 
 
-def _grouped_sweep(n=12, seed=77):
+def _grouped_sweep(n=40, seed=77):
     rs = np.random.RandomState(seed)
     cases = []
     for i in range(n):

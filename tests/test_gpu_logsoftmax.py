@@ -143,7 +143,7 @@ def test_apply_partials_neutral_pairs_and_empty_slice(cuda_device):
     assert torch.equal(lse_empty, lse_ref)
 
 
-def _ls_sweep(n=16, seed=909):
+def _ls_sweep(n=40, seed=909):
     rs = np.random.RandomState(seed)
     out = []
     for i in range(n):
