@@ -317,3 +317,47 @@ def test_grouped_table_orders_give_identical_results(cuda_device, monkeypatch, o
             assert outs[g].numel() == 0
             continue
         assert np.array_equal(outs[g].cpu().numpy(), refs[g].astype(np.float32)), f"group {g} {M}x{N}x{K}"
+
+
+@pytest.mark.parametrize("la,lb", [("row", "row"), ("col", "col")])
+def test_grouped_fp16_inputs(cuda_device, la, lb):
+    """FP16 operands (the instruction descriptors' other input format) through normal and
+    transposed tiles: integer inputs exact in FP32; real inputs with an FP16 bias and SiLU
+    into FP16 outputs within the contract."""
+    shapes = [(100, 264, 136), (384, 512, 200), (1, 40, 64), (520, 128, 72)]
+
+    def op16(x, layout):
+        t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.float16)
+        if layout == "row":
+            return t.cuda()
+        rows, cols = t.shape
+        ld = max(8, -(-rows // 8) * 8)
+        buf = torch.zeros((cols, ld), dtype=torch.float16)
+        buf[:, :rows] = t.t()
+        return buf.cuda()[:, :rows].t()
+
+    As, Bs, refs = [], [], []
+    for g, (M, N, K) in enumerate(shapes):
+        a = synth.integers(48, 2 * g, (M, K), -3, 3)
+        b = synth.integers(48, 2 * g + 1, (K, N), -3, 3)
+        As.append(op16(a, la)); Bs.append(op16(b, lb))
+        refs.append(oracle.gemm(a.astype(np.float16), b.astype(np.float16), a_dtype=oracle.F16, b_dtype=oracle.F16,
+                                out_dtype=oracle.F32))
+    outs = sg.gemm_bf16_grouped(As, Bs, out_dtype=torch.float32)
+    assert sg.check() == sg.OK
+    for g in range(len(shapes)):
+        assert np.array_equal(outs[g].cpu().numpy(), refs[g].astype(np.float32)), f"group {g}"
+    As, Bs, bs, hs = [], [], [], []
+    for g, (M, N, K) in enumerate(shapes):
+        a = synth.normal(49, 3 * g, (M, K)).astype(np.float16)
+        b = (synth.normal(49, 3 * g + 1, (K, N)) * 0.1).astype(np.float16)
+        bias = synth.normal(49, 3 * g + 2, (N,)).astype(np.float16)
+        As.append(op16(a, la)); Bs.append(op16(b, lb)); bs.append(torch.from_numpy(bias).cuda())
+        hs.append((a, b, bias))
+    outs = sg.gemm_bf16_grouped(As, Bs, biases=bs, act="silu", out_dtype=torch.float16)
+    assert sg.check() == sg.OK
+    for g, (M, N, K) in enumerate(shapes):
+        a, b, bias = hs[g]
+        ref, acc = oracle.gemm(a, b, a_dtype=oracle.F16, b_dtype=oracle.F16, bias=bias, bias_dtype=oracle.F16,
+                               act=oracle.ACT_SILU, out_dtype=oracle.F16, want_absacc=True)
+        check_tolerance(outs[g].float().cpu().numpy(), ref, acc, torch.float16, what=f"group {g} {M}x{N}x{K}")
