@@ -22,25 +22,33 @@ struct MaxSum {
   float m, s;
 };
 
+// One exponential per merge: the pair with the larger max keeps its sum as it is.
 __device__ __forceinline__ MaxSum merge(MaxSum a, MaxSum b) {
   if (a.s == 0.0f) return b;
   if (b.s == 0.0f) return a;
-  const float M = fmaxf(a.m, b.m);
-  return {M, a.s * expf(a.m - M) + b.s * expf(b.m - M)};
+  if (a.m >= b.m) return {a.m, a.s + b.s * expf(b.m - a.m)};
+  return {b.m, a.s * expf(a.m - b.m) + b.s};
 }
 
-// Block-wide merge (256 threads) in a fixed order; the result is returned to thread 0.
-__device__ __forceinline__ MaxSum block_merge(MaxSum v, MaxSum* sh) {
+__device__ __forceinline__ MaxSum warp_merge(MaxSum v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     MaxSum u{__shfl_xor_sync(0xffffffffu, v.m, o), __shfl_xor_sync(0xffffffffu, v.s, o)};
     v = merge(v, u);
   }
-  const int w = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) sh[w] = v;
+  return v;
+}
+
+// Block-wide merge (256 threads) in a fixed order: a butterfly within each warp, then
+// one over the warps' results in warp 0. The result is returned to thread 0.
+__device__ __forceinline__ MaxSum block_merge(MaxSum v, MaxSum* sh) {
+  v = warp_merge(v);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) sh[w] = v;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int i = 1; i < static_cast<int>(blockDim.x >> 5); ++i) v = merge(v, sh[i]);
+  if (w == 0) {
+    v = lane < static_cast<int>(blockDim.x >> 5) ? sh[lane] : MaxSum{-INFINITY, 0.0f};
+    v = warp_merge(v);
   }
   return v;
 }
@@ -120,15 +128,31 @@ __global__ void __launch_bounds__(256) lse_tile_partials_kernel(const float* __r
   if (lane == 0) part[static_cast<long long>(t) * M + m] = v.s > 0.0f ? make_float2(v.m, v.s) : make_float2(-INFINITY, 0.0f);
 }
 
-// Merge and subtract in one launch: CTA (x, m) merges row m's partials (every CTA of the
-// row in the same fixed order, so all get the same lse bit for bit; CTA 0 stores it) and
-// subtracts it from columns [x chunk, (x + 1) chunk) of the row. Each thread issues the
-// loads of its first four float4 of the chunk before the merge, so their latency overlaps
-// it, and loads its partials four at a time.
+__device__ __forceinline__ void st_cluster_f2(uint32_t addr, float a, float b) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
+  float2 r;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(r.x), "=f"(r.y) : "r"(addr) : "memory");
+  return r;
+}
+
+// Merge and subtract in one launch: CTA (x, m) subtracts row m's lse from columns
+// [x chunk, (x + 1) chunk) of the row. The lse comes from the row's partials: with CS = 1
+// every CTA merges all of them; with clusters of CS CTAs along x, CTA rank r merges the
+// r-th of CS equal shares, writes its result to CTA 0's shared memory, and after a cluster
+// barrier every CTA merges the CS results in rank order (the partials, read with a stride
+// of M pairs, then cross from L2 once per cluster instead of once per CTA). Either way
+// every CTA of a row takes the same steps in the same order, so all get the same lse bit
+// for bit (CTA 0 stores it). Each thread issues the loads of its first four float4 of the
+// chunk before the merge, so their latency overlaps it, and loads its partials four at a
+// time.
+template <int CS>
 __global__ void __launch_bounds__(256) lse_merge_subtract_kernel(const float2* __restrict__ part, int n_parts,
                                                                  int M, float* __restrict__ C, long long ldc, int N,
                                                                  int chunk, float* __restrict__ lse) {
   __shared__ MaxSum sh[8];
+  __shared__ float2 shares[CS];  // read in CTA 0 only (cluster ranks' merged shares)
   __shared__ float l_sh;
   pdl_launch_dependents();
   pdl_wait();
@@ -146,20 +170,35 @@ __global__ void __launch_bounds__(256) lse_merge_subtract_kernel(const float2* _
     for (int u = 0; u < 4; ++u)
       if (q0 + u * bd < q1) x[u] = r4[q0 + u * bd];
   }
-  // Partials t = threadIdx.x, + blockDim.x, ... merged in that order (identity pairs past
-  // n_parts change nothing).
+  const int rank = CS > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int per = (n_parts + CS - 1) / CS;
+  const int p0 = rank * per, p1 = p0 + per < n_parts ? p0 + per : n_parts;
+  // Partials p0 + threadIdx.x, + blockDim.x, ... merged in that order (identity pairs
+  // past p1 change nothing).
   MaxSum v{-INFINITY, 0.0f};
-  for (int t0 = static_cast<int>(threadIdx.x); t0 < n_parts; t0 += 4 * bd) {
+  for (int t0 = p0 + static_cast<int>(threadIdx.x); t0 < p1; t0 += 4 * bd) {
     float2 q[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int t = t0 + u * bd;
-      q[u] = t < n_parts ? part[static_cast<size_t>(t) * M + m] : make_float2(-INFINITY, 0.0f);
+      q[u] = t < p1 ? part[static_cast<size_t>(t) * M + m] : make_float2(-INFINITY, 0.0f);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) v = merge(v, MaxSum{q[u].x, q[u].y});
   }
   v = block_merge(v, sh);
+  if constexpr (CS > 1) {
+    if (threadIdx.x == 0) st_cluster_f2(mapa_shared(smem_u32(&shares[rank]), 0), v.m, v.s);
+    cluster_sync();
+    if (threadIdx.x == 0) {
+      v = MaxSum{-INFINITY, 0.0f};
+#pragma unroll
+      for (int i = 0; i < CS; ++i) {
+        const float2 q = ld_cluster_f2(mapa_shared(smem_u32(&shares[i]), 0));
+        v = merge(v, MaxSum{q.x, q.y});
+      }
+    }
+  }
   if (threadIdx.x == 0) {
     const float l = v.s > 0.0f ? v.m + logf(v.s) : -INFINITY;
     l_sh = l;
@@ -184,6 +223,8 @@ __global__ void __launch_bounds__(256) lse_merge_subtract_kernel(const float2* _
   } else {
     for (int n = c0 + static_cast<int>(threadIdx.x); n < c1; n += bd) row[n] -= l;
   }
+  // CTA 0's shares stay in place until every CTA of the cluster has read them.
+  if constexpr (CS > 1) cluster_sync();
 }
 
 }  // namespace
@@ -201,18 +242,35 @@ cudaError_t launch_log_softmax_rows(float* C, long long ldc, int M, int N, const
   if (M <= 0 || (part == nullptr && N <= 0)) return cudaSuccess;
   if (part != nullptr && N > 0 && M <= 65535) {
     // One launch: about four CTAs per SM over the rows' column chunks (multiples of 1024).
+    // With at least kCs chunks per row, the chunks of a row run in clusters of kCs CTAs
+    // that share the merge (the grid's x rounded up to whole clusters; the extra CTAs
+    // merge and subtract nothing).
+    constexpr int kCs = 8;
     const long long ctas_per_row = (4LL * (sms > 0 ? sms : 1) + M - 1) / M;
     long long chunk = (static_cast<long long>(N) + ctas_per_row - 1) / ctas_per_row;
     chunk = (chunk + 1023) / 1024 * 1024;
-    const unsigned gx = static_cast<unsigned>((N + chunk - 1) / chunk);
+    unsigned gx = static_cast<unsigned>((N + chunk - 1) / chunk);
+    const bool clustered = gx >= static_cast<unsigned>(kCs);
+    if (clustered) gx = (gx + kCs - 1) / kCs * kCs;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(gx, static_cast<unsigned>(M), 1);
     cfg.blockDim = dim3(256, 1, 1);
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    if (clustered) {
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = kCs;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+    }
     add_pdl_attr(cfg, attr);
     const cudaError_t e =
-        cudaLaunchKernelEx(&cfg, lse_merge_subtract_kernel, part, n_tiles, M, C, ldc, N, static_cast<int>(chunk), lse);
+        clustered ? cudaLaunchKernelEx(&cfg, lse_merge_subtract_kernel<kCs>, part, n_tiles, M, C, ldc, N,
+                                       static_cast<int>(chunk), lse)
+                  : cudaLaunchKernelEx(&cfg, lse_merge_subtract_kernel<1>, part, n_tiles, M, C, ldc, N,
+                                       static_cast<int>(chunk), lse);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
