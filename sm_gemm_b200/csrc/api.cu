@@ -818,7 +818,9 @@ smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const
   for (int g = 0; g < G; ++g) perm[static_cast<size_t>(g)] = g;
   const long long order = env_ll(kKnobGroupedOrder, 1);
   if (order == 1 || order == 2) {
-    auto work = [&](int g) { return M[g] * N[g] * K[g]; };
+    auto work = [&](int g) {  // in double: the product of three int-sized extents can overflow int64
+      return static_cast<double>(M[g]) * static_cast<double>(N[g]) * static_cast<double>(K[g]);
+    };
     std::stable_sort(perm.begin(), perm.end(), [&](int x, int y) { return work(x) > work(y); });
     if (order == 2) {  // largest, smallest, second largest, second smallest, ...
       std::vector<int> z;
