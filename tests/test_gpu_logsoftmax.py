@@ -72,6 +72,19 @@ def test_logsoftmax_lm_head_full_size(cuda_device):
     _check(out, X, W, None, rows=np.array([0, 15]))
 
 
+@pytest.mark.parametrize("M,N", [(64, 20000), (3, 50000)])
+def test_logsoftmax_cluster_merge_with_padding_ctas(cuda_device, M, N):
+    """Wide rows whose column chunks run in clusters of 8 CTAs sharing the merge, with a
+    chunk count that is not a multiple of 8 (10 and 49 chunks per row: the padding CTAs
+    merge their share and subtract nothing), with bias, against the oracle on every row."""
+    X = to_dtype(synth.normal(51, 0, (M, 256)), torch.bfloat16)
+    W = to_dtype(synth.normal(51, 1, (256, N), 0.05), torch.bfloat16)
+    b = to_dtype(synth.normal(51, 2, (N,), 0.5), torch.bfloat16)
+    out = sg.gemm_bf16_logsoftmax(X.cuda(), W.cuda(), bias=b.cuda())
+    assert sg.check() == sg.OK
+    _check(out, X, W, b)
+
+
 def test_logsoftmax_k0_is_log_softmax_of_bias(cuda_device):
     """K = 0: the logits are the bias alone, so every row is log_softmax(bias)."""
     M, N = 5, 1000
