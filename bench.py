@@ -14,7 +14,8 @@ Timing: W untimed warm-up steps, then K steps between CUDA events on the launchi
 stream, bracketed by a barrier and a device synchronise; the maximum over ranks is
 taken. Workloads whose operands fit in L2 rotate over enough copies that the bytes
 touched between two uses of one copy exceed L2. SM clocks and throttle reasons are
-sampled with nvidia-smi during the headline's timed region. After that region the
+read through NVML over and over while the headline's timed calls run (and by nvidia-smi
+every 200 ms over the same window). After that region the
 headline also times at least 50 further calls one by one (events around each call) and
 reports their median, minimum and maximum.
 
@@ -140,6 +141,62 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+class NvmlClocks:
+    """The SM clock and the active clock-event (throttle) reasons read in-process through
+    NVML (what nvidia-smi reports), so that they can be sampled many times within a timed
+    region of a few milliseconds, shorter than nvidia-smi's sampling period. Reading only:
+    no setting of the GPU is touched."""
+
+    def __init__(self, uuid):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.names = [(getattr(pynvml, "nvmlClocksEventReasonHwSlowdown", 0x8), "hw_slowdown"),
+                          (getattr(pynvml, "nvmlClocksEventReasonHwThermalSlowdown", 0x40), "hw_thermal_slowdown"),
+                          (getattr(pynvml, "nvmlClocksEventReasonSwThermalSlowdown", 0x20), "sw_thermal_slowdown"),
+                          (getattr(pynvml, "nvmlClocksEventReasonSwPowerCap", 0x4), "sw_power_cap")]
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def sample(self):
+        if not self.ok:
+            return
+        try:
+            self.samples.append((float(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)),
+                                 int(self.get_reasons(self.h))))
+        except Exception:
+            self.ok = False
+
+    def summary(self):
+        if not self.samples:
+            return None
+        reasons = sorted({n for _, r in self.samples for bit, n in self.names if r & bit})
+        return {"sm_mhz": float(np.median([m for m, _ in self.samples])), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml, during the timed region"}
+
+
+def merge_clocks(nvml_summary, smi_summary):
+    """The clock record of the JSON line: NVML samples taken while the timed calls ran
+    when there are any, with nvidia-smi's samples (every 200 ms over the same window,
+    often none within a region of a few milliseconds) beside them; else nvidia-smi's."""
+    if nvml_summary is None:
+        return dict(smi_summary, source="nvidia-smi")
+    out = dict(nvml_summary)
+    out["nvidia_smi"] = smi_summary
+    if smi_summary.get("sm_max_mhz"):
+        out["sm_max_mhz"] = smi_summary["sm_max_mhz"]
+    out["reasons"] = sorted(set(out["reasons"]) | set(smi_summary.get("reasons", [])))
+    return out
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 # About 50 us of SM cycles: enough for the host to queue a few calls ahead.
@@ -152,13 +209,15 @@ MIN_TIMED_MS = 2.0
 DEVICE_WARMUP_CYCLES = 100_000_000
 
 
-def time_steps(torch, step, warmup: int, steps: int, dist=None):
+def time_steps(torch, step, warmup: int, steps: int, dist=None, poll=None):
     """Device time of `steps` calls of step(i) after `warmup` calls: CUDA events on the
     current stream, barrier + synchronise on both sides, max over ranks (ms total).
 
     A short spin kernel runs before the start event: while the device is busy with it
     the host queues the first timed calls, so the timed region starts with work queued
-    instead of with the device waiting for the first launch to come through."""
+    instead of with the device waiting for the first launch to come through. With `poll`,
+    the host calls it repeatedly once every timed call is queued, until the end event has
+    completed (to sample clocks while the device runs the timed calls)."""
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
@@ -171,6 +230,9 @@ def time_steps(torch, step, warmup: int, steps: int, dist=None):
     for i in range(steps):
         step(warmup + i)
     e.record()
+    if poll is not None:
+        while not e.query():
+            poll()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -270,7 +332,7 @@ class Ctx:
         self.launches = 0
         self.results = {}
 
-    def time(self, step, launches_per_step=1, warmup=None, steps=None, min_ms="default"):
+    def time(self, step, launches_per_step=1, warmup=None, steps=None, min_ms="default", poll=None):
         """Device time (ms) of K calls of step. With min_ms (and no explicit step
         count), a workload whose K calls took less than min_ms is timed again over
         enough calls to span it, and the result is scaled back to K calls: kernels of a
@@ -280,7 +342,7 @@ class Ctx:
         k = self.K if steps is None else steps
         if min_ms == "default":
             min_ms = self.min_ms
-        ms = time_steps(self.torch, step, w, k, self.dist)
+        ms = time_steps(self.torch, step, w, k, self.dist, poll=poll)
         self.launches += launches_per_step * k
         if steps is None and min_ms is not None and 0 < ms < min_ms:
             k2 = int(math.ceil(k * min_ms / ms))
@@ -331,8 +393,9 @@ def wl_square_bf16(c: Ctx, headline: bool):
         smi_id = "GPU-" + str(torch.cuda.get_device_properties(c.dev).uuid)
     except Exception:
         smi_id = str(c.dev.index)
+    nvml = NvmlClocks(smi_id)
     with ClockSampler(smi_id) as clk:
-        ms = c.time(step, min_ms=None)
+        ms = c.time(step, min_ms=None, poll=nvml.sample)
     dist_us = per_call_us(torch, step, c.W + c.K, max(50, c.K))
     assert sg.check() == sg.OK
     flops = m.gemm_flops(n, n, n)
@@ -340,7 +403,7 @@ def wl_square_bf16(c: Ctx, headline: bool):
     c.record("square_bf16_4096", ms, c.K, flops=flops, peak_tf=c.peaks["bf16_tflops"],
              extra={"plan": plan, "per_call_us": dist_us})
     out = {"ms": ms, "flops": flops, "copies": copies, "set_bytes": set_bytes, "plan": plan,
-           "clocks": clk.summary()}
+           "clocks": merge_clocks(nvml.summary(), clk.summary())}
     if not headline:
         return out
     # End to end through the public API from pinned host buffers: every step uploads its
