@@ -130,17 +130,20 @@ smgemm_status gemm_bf16_noalloc(int64_t M, int64_t N, int64_t K,
  *              groups' TMA descriptors and sizes are written there before the launch (by
  *              small kernels on `stream` that carry them as parameters, so the call can be
  *              captured in a CUDA graph; up to 16 groups travel with the launch itself);
- *              the rest holds the partial tiles of a split last wave. Calls that can overlap on the GPU
- *              must not share it. A smaller workspace that still holds the table is
- *              accepted; the last wave is then not split.
+ *              the rest holds the partial tiles of a split last wave. Calls that can
+ *              overlap on the GPU must not share it. A smaller workspace that still holds
+ *              the table is accepted; the last wave is then not split.
  * Every group is validated, and every TMA descriptor encoded, before anything is
  * enqueued; the descriptor table is written first, then groups with K = 0 are filled,
- * then the GEMM launches. Errors as in gemm_bf16. Tiles
- * of 256 x 256 run one per CTA pair; when the tiles do not fill a whole last wave, the
- * R tiles of that wave are each split along K into S = min(P / R, KB / 8) pieces (P
- * co-resident pairs, KB the smallest K-block count among those tiles) that run side
- * by side; the last piece to finish sums the partials in piece order, so results are
- * deterministic run to run.
+ * then the GEMM launches. Errors as in gemm_bf16. Tiles of 256 x 256 run one per CTA
+ * pair, the groups laid out with the most work (M N K) first; a group's last row of
+ * tiles with at most 128 rows runs as 256 x 128 tiles of C_g^T = B_g^T A_g^T instead (half
+ * the tensor work of a 256-row tile padded with zero rows). When the tiles do not fill a
+ * whole last wave, the R tiles of that wave are each split along K into
+ * S = min(P / R, KB / 8) pieces (P co-resident pairs, KB the smallest K-block count
+ * among those tiles) that run side by side; the last piece to finish sums the partials
+ * in piece order, so results are deterministic run to run and do not depend on the
+ * groups' order.
  */
 size_t smgemm_grouped_workspace_size(int G);
 smgemm_status gemm_bf16_grouped(int G, const int64_t* M, const int64_t* N, const int64_t* K,
