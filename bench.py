@@ -175,6 +175,21 @@ class NvmlClocks:
         except Exception:
             self.ok = False
 
+    # A background thread reads back to back from begin() to end() (NVML calls run
+    # outside the interpreter lock, so the launching thread is not held up).
+    def begin(self):
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+
+    def _run(self):
+        while not self._stop.is_set() and self.ok:
+            self.sample()
+
+    def end(self):
+        self._stop.set()
+        self._thread.join(timeout=5)
+
     def summary(self):
         if not self.samples:
             return None
@@ -209,15 +224,15 @@ MIN_TIMED_MS = 2.0
 DEVICE_WARMUP_CYCLES = 100_000_000
 
 
-def time_steps(torch, step, warmup: int, steps: int, dist=None, poll=None):
+def time_steps(torch, step, warmup: int, steps: int, dist=None, during=None):
     """Device time of `steps` calls of step(i) after `warmup` calls: CUDA events on the
     current stream, barrier + synchronise on both sides, max over ranks (ms total).
 
     A short spin kernel runs before the start event: while the device is busy with it
     the host queues the first timed calls, so the timed region starts with work queued
-    instead of with the device waiting for the first launch to come through. With `poll`,
-    the host calls it repeatedly once every timed call is queued, until the end event has
-    completed (to sample clocks while the device runs the timed calls)."""
+    instead of with the device waiting for the first launch to come through. `during`
+    (optional) has begin() called just before the start event and end() once the end
+    event has completed (clock sampling over the timed region)."""
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
@@ -225,15 +240,16 @@ def time_steps(torch, step, warmup: int, steps: int, dist=None, poll=None):
         dist.barrier()
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
+    if during is not None:
+        during.begin()
     torch.cuda._sleep(QUEUE_AHEAD_CYCLES)
     s.record()
     for i in range(steps):
         step(warmup + i)
     e.record()
-    if poll is not None:
-        while not e.query():
-            poll()
     torch.cuda.synchronize()
+    if during is not None:
+        during.end()
     if dist is not None:
         dist.barrier()
     return max_over_ranks(s.elapsed_time(e), dist)
@@ -332,7 +348,7 @@ class Ctx:
         self.launches = 0
         self.results = {}
 
-    def time(self, step, launches_per_step=1, warmup=None, steps=None, min_ms="default", poll=None):
+    def time(self, step, launches_per_step=1, warmup=None, steps=None, min_ms="default", during=None):
         """Device time (ms) of K calls of step. With min_ms (and no explicit step
         count), a workload whose K calls took less than min_ms is timed again over
         enough calls to span it, and the result is scaled back to K calls: kernels of a
@@ -342,7 +358,7 @@ class Ctx:
         k = self.K if steps is None else steps
         if min_ms == "default":
             min_ms = self.min_ms
-        ms = time_steps(self.torch, step, w, k, self.dist, poll=poll)
+        ms = time_steps(self.torch, step, w, k, self.dist, during=during)
         self.launches += launches_per_step * k
         if steps is None and min_ms is not None and 0 < ms < min_ms:
             k2 = int(math.ceil(k * min_ms / ms))
@@ -395,7 +411,7 @@ def wl_square_bf16(c: Ctx, headline: bool):
         smi_id = str(c.dev.index)
     nvml = NvmlClocks(smi_id)
     with ClockSampler(smi_id) as clk:
-        ms = c.time(step, min_ms=None, poll=nvml.sample)
+        ms = c.time(step, min_ms=None, during=nvml if nvml.ok else None)
     dist_us = per_call_us(torch, step, c.W + c.K, max(50, c.K))
     assert sg.check() == sg.OK
     flops = m.gemm_flops(n, n, n)
