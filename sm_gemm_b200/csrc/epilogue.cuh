@@ -64,12 +64,40 @@ __device__ __forceinline__ float x_sigmoid_f32(float x, float z) {
   return z >= 0.0f ? x * r : (x * e) * r;
 }
 
+// GeLU's z = 2 sqrt(2/pi) (x + 0.044715 x^3) = x (kGeluA + kGeluB x^2).
+constexpr float kGeluA = 1.5957691216057308f;   // 2 sqrt(2/pi)
+constexpr float kGeluB = 0.07135481627260025f;  // 2 sqrt(2/pi) 0.044715
+
 __device__ __forceinline__ float act_apply(float x, int act) {
-  if (act == 1) {
-    const float u = 0.7978845608028654f * (x + 0.044715f * x * x * x);  // sqrt(2/pi) (x + 0.044715 x^3)
-    return x_sigmoid_f32(x, 2.0f * u);
-  }
+  if (act == 1) return x_sigmoid_f32(x, x * fmaf(kGeluB, x * x, kGeluA));
   if (act == 2) return x_sigmoid_f32(x, x);
+  return x;
+}
+
+// The same for two elements: the FP32 arithmetic as packed FP32x2 operations (each half
+// rounded exactly like the scalar operation, so results equal act_apply's), the
+// exponential and the reciprocal on the special-function unit one element at a time.
+__device__ __forceinline__ float2 x_sigmoid_f32x2(float2 x, float2 z) {
+  const float2 t = __fmul2_rn(make_float2(fabsf(z.x), fabsf(z.y)),
+                              make_float2(-1.4426950408889634f, -1.4426950408889634f));
+  const bool tiny0 = t.x < -120.0f, tiny1 = t.y < -120.0f;
+  float e0 = exp2_sfu(tiny0 ? t.x + 64.0f : t.x);
+  float e1 = exp2_sfu(tiny1 ? t.y + 64.0f : t.y);
+  if (tiny0) e0 *= 5.421010862427522e-20f;  // 2^-64
+  if (tiny1) e1 *= 5.421010862427522e-20f;
+  const float2 d = __fadd2_rn(make_float2(1.0f, 1.0f), make_float2(e0, e1));
+  const float2 r = make_float2(rcp_sfu(d.x), rcp_sfu(d.y));
+  // x * r for z >= 0, (x * e) * r below (x * 1 is exact).
+  const float2 xe = __fmul2_rn(x, make_float2(z.x >= 0.0f ? 1.0f : e0, z.y >= 0.0f ? 1.0f : e1));
+  return __fmul2_rn(xe, r);
+}
+
+__device__ __forceinline__ float2 act_apply2(float2 x, int act) {
+  if (act == 1) {
+    const float2 p = __ffma2_rn(make_float2(kGeluB, kGeluB), __fmul2_rn(x, x), make_float2(kGeluA, kGeluA));
+    return x_sigmoid_f32x2(x, __fmul2_rn(x, p));
+  }
+  if (act == 2) return x_sigmoid_f32x2(x, x);
   return x;
 }
 
@@ -105,17 +133,29 @@ __device__ __forceinline__ void store_one(void* C, int dtype, long long off, flo
 // blocks in one step and stays a short, straight run of instructions (the epilogue
 // warps share instruction caches with the producer and MMA-issuer warps).
 // bias[col0 .. col0 + 32) added to v with 16-byte loads (two 16-bit values per word);
-// one branch on the bias type and alignment per chunk, none per element.
+// one branch on the bias type and alignment per chunk, none per element. kPacked: the
+// adds as packed FP32x2 operations (same results, half the instructions; the FP8
+// promotion kernels, short of registers, keep the scalar form).
+template <bool kPacked = true>
 __device__ __forceinline__ void add_bias32_vec(const EpiArgs& e, int col0, float (&v)[32]) {
   if (e.bias_dtype == 0) {
     const float4* b4 = reinterpret_cast<const float4*>(static_cast<const float*>(e.bias) + col0);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const float4 b = __ldg(b4 + q);
-      v[4 * q] += b.x;
-      v[4 * q + 1] += b.y;
-      v[4 * q + 2] += b.z;
-      v[4 * q + 3] += b.w;
+      if constexpr (kPacked) {
+        const float2 lo = __fadd2_rn(make_float2(v[4 * q], v[4 * q + 1]), make_float2(b.x, b.y));
+        const float2 hi = __fadd2_rn(make_float2(v[4 * q + 2], v[4 * q + 3]), make_float2(b.z, b.w));
+        v[4 * q] = lo.x;
+        v[4 * q + 1] = lo.y;
+        v[4 * q + 2] = hi.x;
+        v[4 * q + 3] = hi.y;
+      } else {
+        v[4 * q] += b.x;
+        v[4 * q + 1] += b.y;
+        v[4 * q + 2] += b.z;
+        v[4 * q + 3] += b.w;
+      }
     }
   } else {
     const uint4* b4 = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(e.bias) + col0);
@@ -132,8 +172,14 @@ __device__ __forceinline__ void add_bias32_vec(const EpiArgs& e, int col0, float
         } else {
           f = __half22float2(*reinterpret_cast<const __half2*>(&w[h]));
         }
-        v[8 * q + 2 * h] += f.x;
-        v[8 * q + 2 * h + 1] += f.y;
+        if constexpr (kPacked) {
+          const float2 y = __fadd2_rn(make_float2(v[8 * q + 2 * h], v[8 * q + 2 * h + 1]), f);
+          v[8 * q + 2 * h] = y.x;
+          v[8 * q + 2 * h + 1] = y.y;
+        } else {
+          v[8 * q + 2 * h] += f.x;
+          v[8 * q + 2 * h + 1] += f.y;
+        }
       }
     }
   }
@@ -154,6 +200,7 @@ __device__ __forceinline__ void epi_bias_act32_f64(const EpiArgs& e, int col0, f
   }
 }
 
+template <bool kPacked = true>
 __device__ __forceinline__ void epi_bias_act32(const EpiArgs& e, int col0, float (&v)[32]) {
   if (e.act != 0 && e.c_dtype == 0) {
     epi_bias_act32_f64(e, col0, v);
@@ -163,7 +210,7 @@ __device__ __forceinline__ void epi_bias_act32(const EpiArgs& e, int col0, float
     const int esz = e.bias_dtype == 0 ? 4 : 2;
     const bool aligned = ((reinterpret_cast<uintptr_t>(e.bias) + static_cast<uintptr_t>(col0) * esz) & 15u) == 0;
     if (col0 + 32 <= e.N && aligned) {
-      add_bias32_vec(e, col0, v);
+      add_bias32_vec<kPacked>(e, col0, v);
     } else if (col0 + 32 <= e.N) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += load_bias(e.bias, e.bias_dtype, col0 + j);
@@ -173,12 +220,30 @@ __device__ __forceinline__ void epi_bias_act32(const EpiArgs& e, int col0, float
         if (col0 + j < e.N) v[j] += load_bias(e.bias, e.bias_dtype, col0 + j);
     }
   }
-  if (e.act == 1) {
+  if constexpr (kPacked) {
+    if (e.act == 1) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], 1);
-  } else if (e.act == 2) {
+      for (int j = 0; j < 16; ++j) {
+        const float2 y = act_apply2(make_float2(v[2 * j], v[2 * j + 1]), 1);
+        v[2 * j] = y.x;
+        v[2 * j + 1] = y.y;
+      }
+    } else if (e.act == 2) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], 2);
+      for (int j = 0; j < 16; ++j) {
+        const float2 y = act_apply2(make_float2(v[2 * j], v[2 * j + 1]), 2);
+        v[2 * j] = y.x;
+        v[2 * j + 1] = y.y;
+      }
+    }
+  } else {
+    if (e.act == 1) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], 1);
+    } else if (e.act == 2) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], 2);
+    }
   }
 }
 
@@ -225,8 +290,9 @@ __device__ __forceinline__ void epi_store_row32(const EpiArgs& e, int row, int c
 }
 
 // 32 consecutive columns col0.. of one output row: bias, activation, cast, store.
+template <bool kPacked = true>
 __device__ __forceinline__ void epi_row32(const EpiArgs& e, int row, int col0, float (&v)[32]) {
-  if (e.bias != nullptr || e.act != 0) epi_bias_act32(e, col0, v);
+  if (e.bias != nullptr || e.act != 0) epi_bias_act32<kPacked>(e, col0, v);
   epi_store_row32(e, row, col0, v);
 }
 

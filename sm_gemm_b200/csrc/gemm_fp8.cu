@@ -260,8 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int col0 = nt * BN + c_local0;
       if (whole) {
         if (!dead) {
-          epi_row32(p.e, row, col0, *reinterpret_cast<float(*)[32]>(acc));
-          epi_row32(p.e, row, col0 + 32, *reinterpret_cast<float(*)[32]>(acc + 32));
+          epi_row32<false>(p.e, row, col0, *reinterpret_cast<float(*)[32]>(acc));
+          epi_row32<false>(p.e, row, col0 + 32, *reinterpret_cast<float(*)[32]>(acc + 32));
         }
       } else {
         // Stream-K partial: store, then the last contributor reduces in CTA order.
@@ -292,8 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float* src = p.slots + (static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * (BM * BN);
             slot_accumulate<64>(src, r_local, c_local0, acc);
           }
-          epi_row32(p.e, row, col0, *reinterpret_cast<float(*)[32]>(acc));
-          epi_row32(p.e, row, col0 + 32, *reinterpret_cast<float(*)[32]>(acc + 32));
+          epi_row32<false>(p.e, row, col0, *reinterpret_cast<float(*)[32]>(acc));
+          epi_row32<false>(p.e, row, col0 + 32, *reinterpret_cast<float(*)[32]>(acc + 32));
         }
         named_barrier_sync(1, kPromoThreads);
       }

@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!dead) {
 #pragma unroll
           for (int h = 0; h < CPW / 32; ++h)
-            epi_row32(p.e, row, col0 + 32 * h, *reinterpret_cast<float(*)[32]>(acc + 32 * h));
+            epi_row32<false>(p.e, row, col0 + 32 * h, *reinterpret_cast<float(*)[32]>(acc + 32 * h));
         }
       } else {
         float* my_slot = p.slots + ((static_cast<size_t>(cluster) * 2 + seg.slot) * 2 + rank) * SLOT;
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float* src = p.slots + ((static_cast<size_t>(cc) * 2 + sk_slot_of(s, cc, t_sk)) * 2 + rank) * SLOT;
               slot_accumulate<32>(src, r_local, c_local0 + 32 * h, v);
             }
-            epi_row32(p.e, row, col0 + 32 * h, v);
+            epi_row32<false>(p.e, row, col0 + 32 * h, v);
           }
         }
         named_barrier_sync(1, kPromoThreads);
